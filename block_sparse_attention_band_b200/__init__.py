@@ -1,0 +1,166 @@
+"""Python binding of the Prism B200 library (include/prism.h).
+
+Argument marshalling only: every step of the estimator and the attention runs
+in the CUDA kernels of ``libprism_b200.so``; PyTorch provides device memory and
+streams.  The functions carry the C names; each raises ``PrismError`` when the
+library returns a non-zero status.  There is no CPU fallback: importing this
+package fails if the library has not been built
+(``python -m block_sparse_attention_band_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+__all__ = [
+    "PrismError", "PrismConfig", "lib", "lib_path", "prism_version", "prism_status_str",
+    "prism_workspace_size", "prism_estimate", "prism_sparse_attn", "prism_prefill",
+    "prism_get_last_device_error", "PRISM_TAU_RMS", "PRISM_TAU_EXPLICIT", "EXPORTED_SYMBOLS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libprism_b200.so")
+
+PRISM_TAU_RMS = 0
+PRISM_TAU_EXPLICIT = 1
+
+EXPORTED_SYMBOLS = (
+    "prism_workspace_size", "prism_estimate", "prism_sparse_attn", "prism_prefill",
+    "prism_get_last_device_error", "prism_status_str", "prism_version",
+)
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: build the CUDA library first "
+        "(python -m block_sparse_attention_band_b200.build); there is no CPU fallback")
+
+lib = ctypes.CDLL(_LIB_PATH)
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int), ("hq", ctypes.c_int), ("hkv", ctypes.c_int),
+        ("seqlen", ctypes.c_int), ("head_dim", ctypes.c_int), ("block", ctypes.c_int),
+        ("band_hi", ctypes.POINTER(ctypes.c_int32)), ("n_hi", ctypes.c_int),
+        ("band_lo", ctypes.POINTER(ctypes.c_int32)), ("n_lo", ctypes.c_int),
+        ("p", ctypes.c_float), ("causal", ctypes.c_int), ("tau_mode", ctypes.c_int),
+        ("tau_hi", ctypes.c_float), ("tau_lo", ctypes.c_float), ("softmax_scale", ctypes.c_float),
+    ]
+
+
+_vp = ctypes.c_void_p
+_cfgp = ctypes.POINTER(_Config)
+lib.prism_version.restype = ctypes.c_int
+lib.prism_status_str.restype = ctypes.c_char_p
+lib.prism_status_str.argtypes = [ctypes.c_int]
+lib.prism_workspace_size.restype = ctypes.c_int
+lib.prism_workspace_size.argtypes = [_cfgp, ctypes.POINTER(ctypes.c_size_t)]
+lib.prism_estimate.restype = ctypes.c_int
+lib.prism_estimate.argtypes = [_cfgp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp, _vp, _vp]
+lib.prism_sparse_attn.restype = ctypes.c_int
+lib.prism_sparse_attn.argtypes = [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.prism_prefill.restype = ctypes.c_int
+lib.prism_prefill.argtypes = [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+lib.prism_get_last_device_error.restype = ctypes.c_int
+lib.prism_get_last_device_error.argtypes = [_vp]
+
+
+class PrismError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({prism_status_str(status)})")
+
+
+class PrismConfig:
+    """Owns a ``prism_config`` and the band index arrays it points to."""
+
+    def __init__(self, batch: int, hq: int, hkv: int, seqlen: int, band_hi: Sequence[int],
+                 band_lo: Sequence[int], p: float, head_dim: int = 128, block: int = 128,
+                 causal: int = 1, tau_mode: int = PRISM_TAU_RMS, tau_hi: float = 1.0,
+                 tau_lo: float = 1.0, softmax_scale: float = 0.0):
+        self._hi = (ctypes.c_int32 * max(len(band_hi), 1))(*band_hi)
+        self._lo = (ctypes.c_int32 * max(len(band_lo), 1))(*band_lo)
+        self.c = _Config(batch, hq, hkv, seqlen, head_dim, block,
+                         ctypes.cast(self._hi, ctypes.POINTER(ctypes.c_int32)), len(band_hi),
+                         ctypes.cast(self._lo, ctypes.POINTER(ctypes.c_int32)), len(band_lo),
+                         p, causal, tau_mode, tau_hi, tau_lo, softmax_scale)
+
+    @property
+    def nb(self) -> int:
+        return self.c.seqlen // self.c.block
+
+    @property
+    def words(self) -> int:
+        return (self.nb + 31) // 32
+
+    def ptr(self):
+        return ctypes.byref(self.c)
+
+
+def _addr(x) -> Optional[int]:
+    """Device address of a CUDA tensor (or a raw int address); None -> NULL."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if not x.is_cuda:
+        raise ValueError("tensor arguments must be CUDA tensors (the library takes device pointers)")
+    if not x.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous")
+    return x.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise PrismError(status, where)
+
+
+def prism_version() -> int:
+    return lib.prism_version()
+
+
+def prism_status_str(status: int) -> str:
+    return lib.prism_status_str(status).decode()
+
+
+def prism_workspace_size(cfg: PrismConfig) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.prism_workspace_size(cfg.ptr(), ctypes.byref(n)), "prism_workspace_size")
+    return n.value
+
+
+def prism_estimate(cfg: PrismConfig, q, k, mask, workspace, stream=None, dbg_scores=None,
+                   dbg_tau=None) -> None:
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib.prism_estimate(cfg.ptr(), _addr(q), _addr(k), _addr(mask), _addr(workspace), ws_bytes,
+                              _stream(stream), _addr(dbg_scores), _addr(dbg_tau)), "prism_estimate")
+
+
+def prism_sparse_attn(cfg: PrismConfig, q, k, v, mask, o, stream=None) -> None:
+    _check(lib.prism_sparse_attn(cfg.ptr(), _addr(q), _addr(k), _addr(v), _addr(mask), _addr(o),
+                                 _stream(stream)), "prism_sparse_attn")
+
+
+def prism_prefill(cfg: PrismConfig, q, k, v, mask_out, o, workspace, stream=None) -> None:
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib.prism_prefill(cfg.ptr(), _addr(q), _addr(k), _addr(v), _addr(mask_out), _addr(o),
+                             _addr(workspace), ws_bytes, _stream(stream)), "prism_prefill")
+
+
+def prism_get_last_device_error(stream=None) -> int:
+    return lib.prism_get_last_device_error(_stream(stream))

@@ -1,0 +1,330 @@
+// Host side of the C ABI declared in include/prism.h: argument validation,
+// workspace layout, TMA descriptors and the kernel launch sequence.
+//
+// Method: "Prism: Spectral-Aware Block-Sparse Attention" -- the
+// paper.rainbus.top review's method paragraph, steps (1)-(7), and the
+// gist.science Technical Summary, sections 1, 2A and 2B.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/prism.h"
+#include "attention.cuh"
+#include "estimate.cuh"
+
+namespace {
+
+using namespace prism;
+
+constexpr int kVersion = 100;  // 0.1.0
+
+// ---------------------------------------------------------------------------
+// validated problem description and workspace layout
+// ---------------------------------------------------------------------------
+struct Plan {
+  int b, hq, hkv, n, nb, W;
+  int q_rows, kv_rows;
+  BandLayout bl;
+  float p_eff;
+  int explicit_tau;
+  float tau_hi, tau_lo;
+  float scale;
+  size_t off_pool, off_part, off_tau, off_scores, off_mask, total;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int validate(const prism_config* cfg, Plan* pl) {
+  if (!cfg) return PRISM_ERR_NULL;
+  if (cfg->batch <= 0 || cfg->hq <= 0 || cfg->hkv <= 0 || cfg->seqlen <= 0) return PRISM_ERR_SHAPE;
+  if (cfg->head_dim != 128 || cfg->block != 128 || cfg->causal != 1) return PRISM_ERR_UNSUPPORTED;
+  if (cfg->hq % cfg->hkv != 0) return PRISM_ERR_SHAPE;
+  if (cfg->seqlen % cfg->block != 0) return PRISM_ERR_SHAPE;
+  const long long nb = cfg->seqlen / cfg->block;
+  // TMA row coordinates are 32-bit; Top-P indices are 16-bit
+  if ((long long)cfg->batch * cfg->hq * cfg->seqlen >= (1ll << 31)) return PRISM_ERR_SHAPE;
+  if (nb > 16384) return PRISM_ERR_UNSUPPORTED;
+  if (cfg->tau_mode != PRISM_TAU_RMS && cfg->tau_mode != PRISM_TAU_EXPLICIT) return PRISM_ERR_UNSUPPORTED;
+  if (cfg->tau_mode == PRISM_TAU_EXPLICIT &&
+      (!(cfg->tau_hi > 0.f) || !(cfg->tau_lo > 0.f) || !std::isfinite(cfg->tau_hi) ||
+       !std::isfinite(cfg->tau_lo)))
+    return PRISM_ERR_TAU;
+  if (!(cfg->p > 0.f)) return PRISM_ERR_P;  // also rejects NaN
+  if (!cfg->band_hi || !cfg->band_lo) return PRISM_ERR_NULL;
+  if (cfg->n_hi <= 0 || cfg->n_lo <= 0 || cfg->n_hi > 128 || cfg->n_lo > 128) return PRISM_ERR_BAND;
+  bool in_hi[128] = {}, in_lo[128] = {};
+  for (int x = 0; x < cfg->n_hi; ++x) {
+    const int d = cfg->band_hi[x];
+    if (d < 0 || d >= 128 || in_hi[d]) return PRISM_ERR_BAND;
+    in_hi[d] = true;
+  }
+  for (int x = 0; x < cfg->n_lo; ++x) {
+    const int d = cfg->band_lo[x];
+    if (d < 0 || d >= 128 || in_lo[d]) return PRISM_ERR_BAND;
+    in_lo[d] = true;
+  }
+  if (!pl) return PRISM_OK;
+  Plan& P = *pl;
+  P.b = cfg->batch;
+  P.hq = cfg->hq;
+  P.hkv = cfg->hkv;
+  P.n = cfg->seqlen;
+  P.nb = (int)nb;
+  P.W = (P.nb + 31) / 32;
+  P.q_rows = P.b * P.hq;
+  P.kv_rows = P.b * P.hkv;
+  // pooled column order: [high only | both | low only | neither]
+  int c = 0;
+  for (int d = 0; d < 128; ++d)
+    if (in_hi[d] && !in_lo[d]) P.bl.perm[c++] = (uint8_t)d;
+  P.bl.s1 = c;
+  for (int d = 0; d < 128; ++d)
+    if (in_hi[d] && in_lo[d]) P.bl.perm[c++] = (uint8_t)d;
+  P.bl.s2 = c;
+  for (int d = 0; d < 128; ++d)
+    if (!in_hi[d] && in_lo[d]) P.bl.perm[c++] = (uint8_t)d;
+  P.bl.s3 = c;
+  for (int d = 0; d < 128; ++d)
+    if (!in_hi[d] && !in_lo[d]) P.bl.perm[c++] = (uint8_t)d;
+  P.bl.d_hi = cfg->n_hi;
+  P.bl.d_lo = cfg->n_lo;
+  P.p_eff = cfg->p >= 1.f ? 1.f : cfg->p;
+  P.explicit_tau = cfg->tau_mode == PRISM_TAU_EXPLICIT;
+  P.tau_hi = cfg->tau_hi;
+  P.tau_lo = cfg->tau_lo;
+  P.scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.0f / std::sqrt(128.0f);
+  const size_t rows = (size_t)P.q_rows + P.kv_rows;
+  const size_t tri = (size_t)P.nb * (P.nb + 1) / 2;
+  size_t off = 0;
+  P.off_pool = off;
+  off = align_up(off + rows * P.nb * 128 * sizeof(float), 256);
+  P.off_part = off;
+  off = align_up(off + rows * P.nb * 4 * sizeof(float), 256);
+  P.off_tau = off;
+  off = align_up(off + (size_t)P.q_rows * 4 * sizeof(float), 256);
+  P.off_scores = off;
+  off = align_up(off + (size_t)P.q_rows * 2 * tri * sizeof(float), 256);
+  P.off_mask = off;
+  off = align_up(off + (size_t)P.q_rows * P.nb * P.W * sizeof(uint32_t), 256);
+  P.total = off;
+  return PRISM_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---------------------------------------------------------------------------
+// per-device one-time setup: architecture check and kernel attributes
+// ---------------------------------------------------------------------------
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int g_dev_state[kMaxDevices];  // 0 unknown, 1 ready, <0 error code
+
+int topp_warps(int nb, size_t* smem) {
+  const int W = (nb + 31) / 32;
+  const int nbp = (nb + 3) & ~3;
+  const size_t per = align_up((size_t)nbp * 8 + (size_t)W * 4, 16);
+  int warps = 4;
+  while (warps > 1 && per * warps > 200 * 1024) --warps;
+  *smem = per * warps;
+  return warps;
+}
+
+int ensure_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PRISM_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return PRISM_ERR_DEVICE;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_dev_state[dev] != 0) return g_dev_state[dev] > 0 ? PRISM_OK : g_dev_state[dev];
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return PRISM_ERR_CUDA;
+  if (major != 10 || minor != 0) {
+    g_dev_state[dev] = PRISM_ERR_DEVICE;
+    return PRISM_ERR_DEVICE;
+  }
+  if (cudaFuncSetAttribute(attn::sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)attn::kSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kScoreSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(topp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
+          cudaSuccess)
+    return PRISM_ERR_CUDA;
+  g_dev_state[dev] = 1;
+  return PRISM_OK;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors: a [rows, 128] bf16 matrix, boxes of 128 rows x 64 columns,
+// 128-byte swizzle (the tcgen05 K-major / MN-major operand layout)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int make_map(CUtensorMap* map, const void* base, size_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return PRISM_ERR_CUDA;
+  cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {128 * sizeof(__nv_bfloat16)};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PRISM_OK : PRISM_ERR_CUDA;
+}
+
+int launched() { return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA; }
+
+// ---------------------------------------------------------------------------
+// launch sequences
+// ---------------------------------------------------------------------------
+int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, unsigned char* ws,
+                 cudaStream_t st, float* dbg_scores, float* dbg_tau) {
+  float* pool = reinterpret_cast<float*>(ws + P.off_pool);
+  float* part = reinterpret_cast<float*>(ws + P.off_part);
+  float* tau = reinterpret_cast<float*>(ws + P.off_tau);
+  float* scores = dbg_scores ? dbg_scores : reinterpret_cast<float*>(ws + P.off_scores);
+  const int units = (P.q_rows + P.kv_rows) * P.nb;
+  pool_kernel<<<units, kPoolThreads, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(q),
+                                              reinterpret_cast<const __nv_bfloat16*>(k), P.q_rows,
+                                              P.nb, pool, part, P.bl);
+  if (launched() != PRISM_OK) return PRISM_ERR_CUDA;
+  tau_kernel<<<P.q_rows, kTauThreads, 0, st>>>(part, P.q_rows, P.hq, P.hkv, P.nb, P.bl.d_hi, P.bl.d_lo,
+                                               P.explicit_tau, P.tau_hi, P.tau_lo, tau, dbg_tau);
+  if (launched() != PRISM_OK) return PRISM_ERR_CUDA;
+  const int T = (P.nb + kScoreTile - 1) / kScoreTile;
+  dim3 sgrid(T * (T + 1) / 2, P.q_rows);
+  scores_kernel<<<sgrid, kScoreThreads, kScoreSmemBytes, st>>>(pool, P.q_rows, P.hq, P.hkv, P.nb, tau,
+                                                              P.bl.s1, P.bl.s2, P.bl.s3, scores);
+  if (launched() != PRISM_OK) return PRISM_ERR_CUDA;
+  size_t smem = 0;
+  const int warps = topp_warps(P.nb, &smem);
+  const int rows = P.q_rows * P.nb;
+  topp_kernel<<<(rows + warps - 1) / warps, warps * 32, smem, st>>>(scores, rows, P.nb, P.p_eff, mask);
+  return launched();
+}
+
+int run_attention(const Plan& P, const void* q, const void* k, const void* v, const uint32_t* mask,
+                  void* o, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  if (make_map(&mq, q, (size_t)P.q_rows * P.n) != PRISM_OK ||
+      make_map(&mk, k, (size_t)P.kv_rows * P.n) != PRISM_OK ||
+      make_map(&mv, v, (size_t)P.kv_rows * P.n) != PRISM_OK)
+    return PRISM_ERR_CUDA;
+  const float scale_log2 = P.scale * 1.4426950408889634f;
+  const unsigned grid = (unsigned)P.q_rows * (unsigned)P.nb;
+  attn::sparse_attn_kernel<<<grid, attn::kThreads, attn::kSmemBytes, st>>>(
+      mq, mk, mv, mask, reinterpret_cast<__nv_bfloat16*>(o), P.b, P.hq, P.hkv, P.n, P.nb, scale_log2);
+  return launched();
+}
+
+}  // namespace
+
+extern "C" {
+
+int prism_version(void) { return kVersion; }
+
+const char* prism_status_str(int s) {
+  switch (s) {
+    case PRISM_OK: return "ok";
+    case PRISM_ERR_NULL: return "a required pointer is NULL";
+    case PRISM_ERR_SHAPE: return "invalid shape (sizes, hq % hkv, seqlen % block, or size overflow)";
+    case PRISM_ERR_ALIGN: return "a pointer is not suitably aligned";
+    case PRISM_ERR_BAND: return "invalid band index set";
+    case PRISM_ERR_P: return "p must be > 0";
+    case PRISM_ERR_UNSUPPORTED: return "unsupported configuration (head_dim/block must be 128, causal must be 1)";
+    case PRISM_ERR_WORKSPACE: return "workspace missing or too small";
+    case PRISM_ERR_CUDA: return "a CUDA runtime call failed";
+    case PRISM_ERR_DEVICE: return "the current device is not sm_100 (B200-class)";
+    case PRISM_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+    case PRISM_ERR_TAU: return "explicit temperatures must be finite and > 0";
+    default: return "unknown status";
+  }
+}
+
+int prism_workspace_size(const prism_config* cfg, size_t* bytes) {
+  if (!bytes) return PRISM_ERR_NULL;
+  Plan P;
+  const int s = validate(cfg, &P);
+  if (s != PRISM_OK) return s;
+  *bytes = P.total;
+  return PRISM_OK;
+}
+
+int prism_estimate(const prism_config* cfg, const void* q, const void* k, uint32_t* mask,
+                   void* workspace, size_t workspace_bytes, prism_stream_t stream, float* dbg_scores,
+                   float* dbg_tau) {
+  Plan P;
+  int s = validate(cfg, &P);
+  if (s != PRISM_OK) return s;
+  if (!q || !k || !mask) return PRISM_ERR_NULL;
+  if (!workspace || workspace_bytes < P.total) return PRISM_ERR_WORKSPACE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(mask, 16) || !aligned(workspace, 256) ||
+      (dbg_scores && !aligned(dbg_scores, 16)) || (dbg_tau && !aligned(dbg_tau, 4)))
+    return PRISM_ERR_ALIGN;
+  if ((s = ensure_device()) != PRISM_OK) return s;
+  return run_estimate(P, q, k, mask, static_cast<unsigned char*>(workspace),
+                      reinterpret_cast<cudaStream_t>(stream), dbg_scores, dbg_tau);
+}
+
+int prism_sparse_attn(const prism_config* cfg, const void* q, const void* k, const void* v,
+                      const uint32_t* mask, void* o, prism_stream_t stream) {
+  Plan P;
+  int s = validate(cfg, &P);
+  if (s != PRISM_OK) return s;
+  if (!q || !k || !v || !mask || !o) return PRISM_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(mask, 4) || !aligned(o, 16))
+    return PRISM_ERR_ALIGN;
+  if ((s = ensure_device()) != PRISM_OK) return s;
+  return run_attention(P, q, k, v, mask, o, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int prism_prefill(const prism_config* cfg, const void* q, const void* k, const void* v,
+                  uint32_t* mask_out, void* o, void* workspace, size_t workspace_bytes,
+                  prism_stream_t stream) {
+  Plan P;
+  int s = validate(cfg, &P);
+  if (s != PRISM_OK) return s;
+  if (!q || !k || !v || !o) return PRISM_ERR_NULL;
+  if (!workspace || workspace_bytes < P.total) return PRISM_ERR_WORKSPACE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(workspace, 256) || (mask_out && !aligned(mask_out, 16)))
+    return PRISM_ERR_ALIGN;
+  if ((s = ensure_device()) != PRISM_OK) return s;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  uint32_t* mask = mask_out ? mask_out : reinterpret_cast<uint32_t*>(ws + P.off_mask);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if ((s = run_estimate(P, q, k, mask, ws, st, nullptr, nullptr)) != PRISM_OK) return s;
+  return run_attention(P, q, k, v, mask, o, st);
+}
+
+int prism_get_last_device_error(prism_stream_t stream) {
+  if (ensure_device() != PRISM_OK) return PRISM_ERR_DEVICE;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return PRISM_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, prism::g_device_error, sizeof(int)) != cudaSuccess) return PRISM_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(prism::g_device_error, &zero, sizeof(int)) != cudaSuccess) return PRISM_ERR_CUDA;
+  return v;
+}
+
+}  // extern "C"

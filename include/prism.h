@@ -1,0 +1,171 @@
+/*
+ * prism.h -- C ABI of the B200 (sm_100a) implementation of Prism's
+ * spectral-aware block-importance estimator and the causal block-sparse
+ * attention prefill that consumes its mask.
+ *
+ * Method: "Prism: Spectral-Aware Block-Sparse Attention" (Wang et al., 2026,
+ * arXiv 2602.08426).  Passages cited below:
+ *   [review:method]  paper.rainbus.top review, the paragraph listing the full
+ *                    pipeline, steps (1)-(7);
+ *   [review:repro]   the same page, reproducibility paragraph (B = 128,
+ *                    d_high = 64, d_low = 96, p = 0.95 / 0.93);
+ *   [summary:1], [summary:2A], [summary:2B]  gist.science Technical Summary,
+ *                    sections 1 (mean pooling as coarse proxy, block-sparse
+ *                    attention computes a subset of blocks), 2A (dual band),
+ *                    2B (RMS-based temperature calibration).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor arguments are DEVICE pointers owned by the caller, contiguous,
+ *   16-byte aligned.  The library never allocates device memory, never
+ *   synchronises, and enqueues all work on the caller's `stream` (0 = the
+ *   legacy default stream).  Calls are asynchronous: a 0 return means the work
+ *   was enqueued, not that it finished.
+ * - Layouts (b = batch, hq / hkv = query / key-value heads, N = seqlen,
+ *   D = head_dim = 128, nb = N / 128, W = ceil(nb / 32)):
+ *     q, o        bf16 [b, hq,  N, D]     (Q after RoPE; output O)
+ *     k, v        bf16 [b, hkv, N, D]     (K after RoPE)
+ *     mask        uint32 [b, hq, nb, W]:  bit (j % 32) of word j / 32 of row i
+ *                 set <=> key block j is kept for query block i.  The
+ *                 estimator writes every word (bits j > i are 0).
+ * - GQA: query head h reads key/value head h / (hq / hkv).
+ * - Return value: PRISM_OK (0) or a negative PRISM_ERR_* code.  Argument
+ *   checks run on the host before anything is enqueued; on an error nothing
+ *   is enqueued and no output is touched.  The library never aborts or traps.
+ */
+#ifndef PRISM_B200_H
+#define PRISM_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* prism_stream_t; /* == cudaStream_t */
+
+enum {
+  PRISM_OK = 0,
+  PRISM_ERR_NULL = -1,        /* a required pointer is NULL                        */
+  PRISM_ERR_SHAPE = -2,       /* batch/heads/seqlen non-positive, hq % hkv != 0,
+                                 seqlen % block != 0, or sizes overflow            */
+  PRISM_ERR_ALIGN = -3,       /* a tensor pointer is not 16-byte aligned           */
+  PRISM_ERR_BAND = -4,        /* band index out of [0, head_dim), duplicated, or an
+                                 empty band                                        */
+  PRISM_ERR_P = -5,           /* p is not in (0, 1] (p > 1 is treated as 1), or NaN */
+  PRISM_ERR_UNSUPPORTED = -6, /* head_dim != 128, block != 128, causal != 1, or an
+                                 unknown tau_mode                                  */
+  PRISM_ERR_WORKSPACE = -7,   /* workspace NULL or smaller than prism_workspace_size */
+  PRISM_ERR_CUDA = -8,        /* a CUDA runtime call failed (launch, attribute)     */
+  PRISM_ERR_DEVICE = -9,      /* the device is not sm_100 (B200-class)              */
+  PRISM_ERR_TIMEOUT = -10,    /* a kernel gave up a bounded wait (device error word) */
+  PRISM_ERR_TAU = -11         /* PRISM_TAU_EXPLICIT with a temperature that is not
+                                 finite and > 0                                    */
+};
+
+enum {
+  PRISM_TAU_RMS = 0,      /* tau_z from the pooled RMS energies (reading R1 below) */
+  PRISM_TAU_EXPLICIT = 1  /* tau_hi / tau_lo taken from the config (tests, ablations) */
+};
+
+/*
+ * Problem statement of one attention layer ([review:method]; [review:repro]).
+ * Band sets are HOST arrays of distinct dimension indices in [0, head_dim);
+ * the default Prism split for the half-split RoPE layout is
+ *   band_hi = {0..31} u {64..95}   (d_high = 64: the 32 fastest RoPE pairs)
+ *   band_lo = {16..63} u {80..127} (d_low  = 96: the 48 slowest RoPE pairs)
+ * The library copies what it needs during the call; the arrays may be freed
+ * when the call returns.
+ *
+ * tau (step 4 of [review:method]) -- reading R1:
+ *   tau_z = RMS(Qbar_z) * RMS(Kbar_z) / (RMS(Qbar_full) * RMS(Kbar_full)),
+ *   per (batch, query head), RMS over all pooled blocks and the band's dims,
+ *   Kbar of the head's KV head; tau_z = 1 if any RMS is 0.
+ * Scores (step 5): L_z[i][j] = Qbar_z[i] . Kbar_z[j] / (tau_z sqrt(d_z)), j <= i.
+ * Top-P (step 6): per row and band, keys ranked by (-prob, j); block j kept iff
+ *   the mass ranked strictly ahead of it is < p (the crossing block is kept);
+ *   p >= 1 keeps every causal block.  Union (step 7): M = M_hi | M_lo.
+ */
+typedef struct prism_config {
+  int batch;
+  int hq;
+  int hkv;
+  int seqlen;
+  int head_dim;          /* must be 128 */
+  int block;             /* B; must be 128; seqlen % block == 0 */
+  const int32_t* band_hi;
+  int n_hi;
+  const int32_t* band_lo;
+  int n_lo;
+  float p;               /* Top-P threshold, 0 < p; p >= 1 keeps all causal blocks */
+  int causal;            /* must be 1 */
+  int tau_mode;          /* PRISM_TAU_RMS or PRISM_TAU_EXPLICIT */
+  float tau_hi;          /* used only with PRISM_TAU_EXPLICIT; must be > 0 */
+  float tau_lo;
+  float softmax_scale;   /* attention scale; <= 0 selects 1/sqrt(head_dim) */
+} prism_config;
+
+/*
+ * Device workspace, in bytes, that prism_estimate / prism_prefill need for
+ * `cfg` (prism_sparse_attn needs none).  Host-only; enqueues nothing.
+ * Writes the size to *bytes.  The workspace holds the pooled Q/K means (fp32),
+ * per-block energy partials, the temperatures and the fp32 band scores
+ * (b * hq * 2 * nb(nb+1)/2 floats); its contents on return are unspecified.
+ */
+int prism_workspace_size(const prism_config* cfg, size_t* bytes);
+
+/*
+ * Estimator, steps (1)-(7) of [review:method]: band slicing and mean pooling
+ * per block of B = 128 tokens, RMS energy of each pooled band, temperatures,
+ * dual-band pooled softmax scores, Top-P per query-block row and band, union.
+ *   q, k        inputs (layouts above)
+ *   mask        output, uint32 [b, hq, nb, W]; every word written
+ *   workspace   >= prism_workspace_size(cfg) bytes, 256-byte aligned
+ *   dbg_scores  optional (NULL: unused) fp32 output holding the scaled band
+ *               scores L_z in packed lower-triangular rows:
+ *               [b, hq, 2 (hi, lo), nb(nb+1)/2], row i starting at i(i+1)/2
+ *   dbg_tau     optional fp32 output [b, hq, 2] = (tau_hi, tau_lo)
+ */
+int prism_estimate(const prism_config* cfg, const void* q, const void* k, uint32_t* mask,
+                   void* workspace, size_t workspace_bytes, prism_stream_t stream,
+                   float* dbg_scores, float* dbg_tau);
+
+/*
+ * Causal block-sparse attention ([summary:1]: only the selected blocks are
+ * computed).  For a query token t in block i it attends to all keys of the
+ * kept blocks j < i and to keys s <= t of block i if block i is kept;
+ * O_t = sum_s softmax_s(q_t . k_s * scale) v_s, fp32 accumulation, bf16 out.
+ * Bits of j > i are ignored; a query block with no kept block gets O = 0.
+ * Runs on the tensor cores (tcgen05 MMA, accumulators in tensor memory).
+ */
+int prism_sparse_attn(const prism_config* cfg, const void* q, const void* k, const void* v,
+                      const uint32_t* mask, void* o, prism_stream_t stream);
+
+/*
+ * One prefill layer: prism_estimate followed by prism_sparse_attn on the same
+ * stream, no host synchronisation in between.  mask_out may be NULL, in which
+ * case the mask lives in the workspace (the size then includes it).
+ */
+int prism_prefill(const prism_config* cfg, const void* q, const void* k, const void* v,
+                  uint32_t* mask_out, void* o, void* workspace, size_t workspace_bytes,
+                  prism_stream_t stream);
+
+/*
+ * Reads and clears the device error word that kernels set when a bounded
+ * wait gives up (PRISM_ERR_TIMEOUT) -- synchronises `stream` first.  Returns
+ * PRISM_OK when no kernel reported an error, a PRISM_ERR_* code otherwise.
+ */
+int prism_get_last_device_error(prism_stream_t stream);
+
+/* Static description of a status code; never NULL. */
+const char* prism_status_str(int status);
+
+/* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
+int prism_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PRISM_B200_H */

@@ -1,0 +1,116 @@
+"""The C-ABI library loads, exports every entry point include/prism.h declares,
+and rejects bad arguments on the host before touching the GPU (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from block_sparse_attention_band_b200 import build as _build
+
+_build.build()
+
+import block_sparse_attention_band_b200 as pb  # noqa: E402
+from tests import gen  # noqa: E402
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "prism.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(prism_\w+)\s*\(", text)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    assert set(pb.EXPORTED_SYMBOLS) <= set(names)
+    for must in ("prism_estimate", "prism_sparse_attn", "prism_prefill"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", pb.lib_path()], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT\s+(prism_\w+)$", out, flags=re.M))
+    for name in declared_functions():
+        assert name in exported, f"{name} declared in prism.h but not exported"
+        assert hasattr(pb.lib, name)
+
+
+def test_version_and_status_strings():
+    assert pb.prism_version() >= 100
+    for code in range(0, -12, -1):
+        s = pb.prism_status_str(code)
+        assert s and s != "unknown status"
+    assert pb.prism_status_str(-999) == "unknown status"
+
+
+def _cfg(**kw):
+    hi, lo = gen.default_bands()
+    args = dict(batch=1, hq=4, hkv=2, seqlen=1024, band_hi=hi, band_lo=lo, p=0.95)
+    args.update(kw)
+    return pb.PrismConfig(**args)
+
+
+def _ws_size(cfg):
+    n = ctypes.c_size_t(0)
+    return pb.lib.prism_workspace_size(cfg.ptr(), ctypes.byref(n)), n.value
+
+
+def test_workspace_size_formula():
+    s, n = _ws_size(_cfg())
+    assert s == 0
+    nb, rows, q_rows = 8, 6, 4
+    tri = nb * (nb + 1) // 2
+
+    def up(x):
+        return (x + 255) // 256 * 256
+    expect = up(rows * nb * 128 * 4) + up(rows * nb * 4 * 4) + up(q_rows * 16) + up(q_rows * 2 * tri * 4) \
+        + up(q_rows * nb * 1 * 4)
+    assert n == expect
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(seqlen=1000), -2), (dict(hq=3, hkv=2), -2), (dict(batch=0), -2), (dict(seqlen=0), -2),
+    (dict(head_dim=64), -6), (dict(block=64), -6), (dict(causal=0), -6), (dict(tau_mode=7), -6),
+    (dict(p=0.0), -5), (dict(p=-1.0), -5), (dict(p=float("nan")), -5),
+    (dict(band_hi=[]), -4), (dict(band_lo=[0, 0]), -4), (dict(band_hi=[128]), -4), (dict(band_lo=[-1]), -4),
+    (dict(tau_mode=1, tau_hi=0.0), -11), (dict(tau_mode=1, tau_lo=float("inf")), -11),
+    (dict(seqlen=128 * 16385), -6),
+])
+def test_bad_config_rejected_on_host(kw, code):
+    s, _ = _ws_size(_cfg(**kw))
+    assert s == code, pb.prism_status_str(s)
+    # the compute entry points reject the same config before any CUDA call
+    fake = 1 << 20
+    assert pb.lib.prism_estimate(_cfg(**kw).ptr(), fake, fake, fake, fake, 1 << 40, None, None, None) == code
+    assert pb.lib.prism_sparse_attn(_cfg(**kw).ptr(), fake, fake, fake, fake, fake, None) == code
+    assert pb.lib.prism_prefill(_cfg(**kw).ptr(), fake, fake, fake, None, fake, fake, 1 << 40, None) == code
+
+
+def test_null_pointers_workspace_and_alignment_rejected():
+    cfg = _cfg()
+    _, ws = _ws_size(cfg)
+    a = 1 << 20
+    assert pb.lib.prism_workspace_size(None, ctypes.byref(ctypes.c_size_t())) == -1
+    assert pb.lib.prism_workspace_size(cfg.ptr(), None) == -1
+    assert pb.lib.prism_estimate(cfg.ptr(), None, a, a, a, ws, None, None, None) == -1
+    assert pb.lib.prism_estimate(cfg.ptr(), a, a, None, a, ws, None, None, None) == -1
+    assert pb.lib.prism_estimate(cfg.ptr(), a, a, a, None, ws, None, None, None) == -7
+    assert pb.lib.prism_estimate(cfg.ptr(), a, a, a, a, ws - 1, None, None, None) == -7
+    assert pb.lib.prism_estimate(cfg.ptr(), a + 8, a, a, a, ws, None, None, None) == -3
+    assert pb.lib.prism_estimate(cfg.ptr(), a, a, a, a + 16, ws, None, None, None) == -3
+    assert pb.lib.prism_sparse_attn(cfg.ptr(), a, a, a, a, None, None) == -1
+    assert pb.lib.prism_sparse_attn(cfg.ptr(), a, a, a + 2, a, a, None) == -3
+    assert pb.lib.prism_prefill(cfg.ptr(), a, a, a, None, a, None, ws, None) == -7
+    assert pb.lib.prism_prefill(cfg.ptr(), a, a, a, a + 4, a, a, ws, None) == -3
+
+
+def test_python_binding_rejects_host_tensors():
+    import torch
+    cfg = _cfg()
+    q = torch.zeros(1, 4, 1024, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        pb.prism_sparse_attn(cfg, q, q, q, q, q, stream=0)

@@ -1,0 +1,163 @@
+"""CUDA path vs the fp64 oracle on small seeded workloads (all outputs compared).
+
+Sizes span several 64-wide score tiles, several 32-bit mask words and a ragged
+tail (nb = 1, 2, 3, 17, 33, 70), GQA 1:1 / 2:1 / 4:1, batch 2.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests import gen
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+import block_sparse_attention_band_b200 as pb  # noqa: E402
+
+
+def _inputs(w, device):
+    q, k, v = gen.make_inputs(w)
+    return q, k, v, q.to(device), k.to(device), v.to(device)
+
+
+CASES = [
+    gen.WORKLOADS["tiny_2k"],
+    gen.small_workload("gqa2_nb17", 1, 4, 2, 17 * 128, seed=21),
+    gen.small_workload("gqa4_nb33", 1, 8, 2, 33 * 128, seed=22, p=0.9),
+    gen.small_workload("batch2_nb3", 2, 2, 1, 3 * 128, seed=23),
+    gen.small_workload("nb1", 1, 2, 2, 128, seed=24),
+    gen.small_workload("nb2", 1, 2, 1, 256, seed=25),
+    gen.small_workload("planted_nb70", 1, 4, 2, 70 * 128, seed=26, p=0.93, rope_base=1e6,
+                       stripes=True, slash=True),
+    gen.small_workload("segments_nb40", 1, 8, 2, 40 * 128, seed=27, segment=1024),
+]
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_estimator_parity(w, cuda_device):
+    q, k, v, qd, kd, vd = _inputs(w, cuda_device)
+    cfg = P.make_cfg(w)
+    mask, sc, tau, _ = P.run_estimate(cfg, qd, kd)
+    hi, lo = gen.default_bands()
+    ref = oracle.estimate(q, k, hi, lo, w.p)
+    P.check_tau(tau, ref)
+    P.check_scores(sc, ref)
+    n_diff, n_exempt = P.check_mask(mask, ref, w.p)
+    # Top-P on the GPU's own scores: the oracle's selection must agree exactly
+    # except where fp32 vs fp64 softmax can flip a decision right at p
+    self_mask, self_cx = P.topp_on_scores(sc, w.p)
+    diff = self_mask != mask
+    near = (np.abs(self_cx[..., 0, :, :] - w.p) < P.SELF_WINDOW) | (np.abs(self_cx[..., 1, :, :] - w.p) < P.SELF_WINDOW)
+    assert not np.any(diff & ~near), f"{np.sum(diff & ~near)} bits differ from Top-P on the GPU scores"
+    print(f"{w.name}: density {P.density(mask):.3f} mismatches {n_diff} (exempt {n_exempt})")
+
+
+@pytest.mark.parametrize("w", CASES[:4] + CASES[6:7], ids=lambda w: w.name)
+def test_attention_parity_with_estimator_mask(w, cuda_device):
+    q, k, v, qd, kd, vd = _inputs(w, cuda_device)
+    cfg = P.make_cfg(w)
+    mask, _, _, words = P.run_estimate(cfg, qd, kd, with_scores=False)
+    o = P.run_attention(cfg, qd, kd, vd, torch.from_numpy(words.view(np.int32)).to(cuda_device))
+    rows = [(b, h, i) for b in range(w.batch) for h in range(w.hq) for i in range(w.nb)]
+    if len(rows) > 96:
+        rng = np.random.default_rng(0)
+        rows = [rows[x] for x in sorted(rng.choice(len(rows), 96, replace=False))]
+    P.check_attention_rows(o, q, k, v, mask, rows, w.hq // w.hkv)
+
+
+@pytest.mark.parametrize("w", [gen.small_workload("dense_nb9", 1, 4, 2, 9 * 128, seed=31),
+                               gen.small_workload("dense_b2", 2, 2, 2, 4 * 128, seed=32)],
+                         ids=lambda w: w.name)
+def test_p1_is_dense_causal(w, cuda_device):
+    q, k, v, qd, kd, vd = _inputs(w, cuda_device)
+    cfg = P.make_cfg(w, p=1.0)
+    mask, _, _, words = P.run_estimate(cfg, qd, kd, with_scores=False)
+    assert np.array_equal(mask, np.broadcast_to(np.tril(np.ones((w.nb, w.nb), dtype=bool)), mask.shape))
+    o = P.run_attention(cfg, qd, kd, vd, torch.from_numpy(words.view(np.int32)).to(cuda_device))
+    dense = oracle.dense_causal_attention(q, k, v, group=w.hq // w.hkv)
+    err = np.abs(o.float().cpu().numpy() - dense)
+    assert err.max() <= P.ATTN_MAX_ABS and err.mean() <= P.ATTN_MEAN_ABS, (err.max(), err.mean())
+
+
+def test_attention_arbitrary_masks(cuda_device):
+    """Random masks incl. empty rows, diagonal-only rows and bits above the
+    diagonal (ignored), fed straight to prism_sparse_attn."""
+    w = gen.small_workload("masks_nb37", 1, 4, 2, 37 * 128, seed=33)
+    q, k, v, qd, kd, vd = _inputs(w, cuda_device)
+    nb = w.nb
+    rng = np.random.default_rng(5)
+    m = rng.random((1, 4, nb, nb)) < 0.3
+    m[0, 0, 5, :] = False          # empty row -> zeros
+    m[0, 1, 7, :] = False
+    m[0, 1, 7, 7] = True           # diagonal only
+    m[0, 2, 9, :] = True           # bits above the diagonal too
+    words = oracle.pack_mask(m)
+    o = P.run_attention(P.make_cfg(w), qd, kd, vd, torch.from_numpy(words.view(np.int32)).to(cuda_device))
+    causal_m = m & np.tril(np.ones((nb, nb), dtype=bool))
+    rows = [(0, h, i) for h in range(4) for i in range(nb)]
+    P.check_attention_rows(o, q, k, v, causal_m, rows, 2)
+    assert torch.all(o[0, 0, 5 * 128:6 * 128] == 0)
+
+
+def test_explicit_tau_and_custom_bands(cuda_device):
+    w = gen.small_workload("custom_nb20", 1, 4, 4, 20 * 128, seed=34, p=0.8)
+    q, k, v, qd, kd, vd = _inputs(w, cuda_device)
+    bands = (list(range(0, 64)), list(range(32, 128)))  # the literal first-64 / last-96 reading
+    cfg = P.make_cfg(w, bands=bands, tau_mode=pb.PRISM_TAU_EXPLICIT, tau_hi=0.5, tau_lo=1.5)
+    mask, sc, tau, _ = P.run_estimate(cfg, qd, kd)
+    ref = oracle.estimate(q, k, bands[0], bands[1], w.p, tau_mode="explicit", tau_explicit=(0.5, 1.5))
+    np.testing.assert_allclose(tau, 0 * tau + np.array([0.5, 1.5]), rtol=0)
+    P.check_scores(sc, ref)
+    P.check_mask(mask, ref, w.p)
+
+
+def test_small_p_sparse_rows(cuda_device):
+    w = gen.small_workload("sparse_nb48", 1, 2, 1, 48 * 128, seed=35, p=0.3)
+    q, k, v, qd, kd, vd = _inputs(w, cuda_device)
+    mask, sc, tau, words = P.run_estimate(P.make_cfg(w), qd, kd)
+    hi, lo = gen.default_bands()
+    ref = oracle.estimate(q, k, hi, lo, w.p)
+    P.check_mask(mask, ref, w.p)
+    assert P.density(mask) < 0.9
+    o = P.run_attention(P.make_cfg(w), qd, kd, vd, torch.from_numpy(words.view(np.int32)).to(cuda_device))
+    rows = [(0, h, i) for h in range(2) for i in range(w.nb)]
+    P.check_attention_rows(o, q, k, v, mask, rows, 2)
+
+
+def test_prefill_matches_separate_calls_and_is_deterministic(cuda_device):
+    w = gen.small_workload("prefill_nb25", 1, 8, 2, 25 * 128, seed=36)
+    q, k, v, qd, kd, vd = _inputs(w, cuda_device)
+    cfg = P.make_cfg(w)
+    ws = torch.empty(pb.prism_workspace_size(cfg), dtype=torch.uint8, device=cuda_device)
+    outs, masks = [], []
+    for _ in range(2):
+        mask = torch.empty(1, 8, w.nb, cfg.words, dtype=torch.int32, device=cuda_device)
+        o = torch.empty_like(qd)
+        pb.prism_prefill(cfg, qd, kd, vd, mask, o, ws)
+        outs.append(o)
+        masks.append(mask)
+    torch.cuda.synchronize()
+    assert torch.equal(masks[0], masks[1]) and torch.equal(outs[0], outs[1])
+    m2, _, _, words = P.run_estimate(cfg, qd, kd, with_scores=False)
+    assert np.array_equal(masks[0].cpu().numpy().view(np.uint32), words)
+    o2 = P.run_attention(cfg, qd, kd, vd, masks[0])
+    assert torch.equal(o2, outs[0])
+    # prefill with the mask kept in the workspace gives the same output
+    o3 = torch.empty_like(qd)
+    pb.prism_prefill(cfg, qd, kd, vd, None, o3, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(o3, outs[0])
+    assert pb.prism_get_last_device_error() == 0
+
+
+def test_softmax_scale_argument(cuda_device):
+    w = gen.small_workload("scale_nb6", 1, 2, 1, 6 * 128, seed=37)
+    q, k, v, qd, kd, vd = _inputs(w, cuda_device)
+    nb = w.nb
+    m = np.tril(np.ones((1, 2, nb, nb), dtype=bool))
+    words = oracle.pack_mask(m)
+    cfg = P.make_cfg(w, softmax_scale=0.05)
+    o = P.run_attention(cfg, qd, kd, vd, torch.from_numpy(words.view(np.int32)).to(cuda_device))
+    rows = [(0, h, i) for h in range(2) for i in range(nb)]
+    P.check_attention_rows(o, q, k, v, m, rows, 2, scale=0.05)
