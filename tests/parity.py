@@ -70,7 +70,7 @@ def check_scores(sc_gpu, ref):
     assert np.array_equal(finite, np.isfinite(sc_gpu)), "causal structure of the scores differs"
     rowmax = np.max(np.where(finite, np.abs(lr), 0.0), axis=-1, keepdims=True)
     tol = 1e-3 * np.maximum(np.abs(lr), 1e-3 * rowmax)
-    err = np.where(finite, np.abs(sc_gpu - lr), 0.0)
+    err = np.abs(np.where(finite, sc_gpu, 0.0) - np.where(finite, lr, 0.0))
     bad = err > np.where(finite, tol, 1.0)
     assert not bad.any(), f"{bad.sum()} score entries outside 1e-3 relative (max err {err.max():.3g})"
 
