@@ -16,7 +16,8 @@ from typing import Optional, Sequence
 __all__ = [
     "PrismError", "PrismConfig", "lib", "lib_path", "prism_version", "prism_status_str",
     "prism_workspace_size", "prism_estimate", "prism_sparse_attn", "prism_prefill",
-    "prism_get_last_device_error", "PRISM_TAU_RMS", "PRISM_TAU_EXPLICIT", "EXPORTED_SYMBOLS",
+    "prism_get_last_device_error", "prism_estimate_noalloc", "prism_noalloc_scratch_bytes",
+    "PRISM_TAU_RMS", "PRISM_TAU_EXPLICIT", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -27,7 +28,8 @@ PRISM_TAU_EXPLICIT = 1
 
 EXPORTED_SYMBOLS = (
     "prism_workspace_size", "prism_estimate", "prism_sparse_attn", "prism_prefill",
-    "prism_get_last_device_error", "prism_status_str", "prism_version",
+    "prism_get_last_device_error", "prism_status_str", "prism_version", "prism_estimate_noalloc",
+    "prism_noalloc_scratch_bytes",
 )
 
 
@@ -67,6 +69,10 @@ lib.prism_sparse_attn.restype = ctypes.c_int
 lib.prism_sparse_attn.argtypes = [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.prism_prefill.restype = ctypes.c_int
 lib.prism_prefill.argtypes = [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+lib.prism_estimate_noalloc.restype = ctypes.c_int
+lib.prism_estimate_noalloc.argtypes = [_cfgp, _vp, _vp, _vp, _vp]
+lib.prism_noalloc_scratch_bytes.restype = ctypes.c_size_t
+lib.prism_noalloc_scratch_bytes.argtypes = []
 lib.prism_get_last_device_error.restype = ctypes.c_int
 lib.prism_get_last_device_error.argtypes = [_vp]
 
@@ -160,6 +166,16 @@ def prism_prefill(cfg: PrismConfig, q, k, v, mask_out, o, workspace, stream=None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(lib.prism_prefill(cfg.ptr(), _addr(q), _addr(k), _addr(v), _addr(mask_out), _addr(o),
                              _addr(workspace), ws_bytes, _stream(stream)), "prism_prefill")
+
+
+def prism_estimate_noalloc(cfg: PrismConfig, q, k, mask, stream=None) -> None:
+    """The estimator on the library's built-in scratch (no workspace argument)."""
+    _check(lib.prism_estimate_noalloc(cfg.ptr(), _addr(q), _addr(k), _addr(mask), _stream(stream)),
+           "prism_estimate_noalloc")
+
+
+def prism_noalloc_scratch_bytes() -> int:
+    return lib.prism_noalloc_scratch_bytes()
 
 
 def prism_get_last_device_error(stream=None) -> int:

@@ -237,6 +237,33 @@ int run_attention(const Plan& P, const void* q, const void* k, const void* v, co
   return launched();
 }
 
+// ---------------------------------------------------------------------------
+// Built-in scratch for prism_estimate_noalloc.  A file-scope device array of
+// fixed size: every GPU that loads this library holds it until the process
+// exits.  Host code may not use the symbol itself as a device address (in host
+// code it names a host-side stand-in); the device address is looked up once
+// per device with cudaGetSymbolAddress while that device is current.
+// ---------------------------------------------------------------------------
+constexpr size_t kStaticScratchBytes = 32u << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices];
+
+int static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PRISM_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return PRISM_ERR_DEVICE;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return PRISM_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return PRISM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -257,6 +284,8 @@ const char* prism_status_str(int s) {
     case PRISM_ERR_DEVICE: return "the current device is not sm_100 (B200-class)";
     case PRISM_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
     case PRISM_ERR_TAU: return "explicit temperatures must be finite and > 0";
+    case PRISM_ERR_SCRATCH_LIMIT:
+      return "problem needs more scratch than the 32 MiB built into prism_estimate_noalloc";
     default: return "unknown status";
   }
 }
@@ -316,6 +345,26 @@ int prism_prefill(const prism_config* cfg, const void* q, const void* k, const v
   if ((s = run_estimate(P, q, k, mask, ws, st, nullptr, nullptr)) != PRISM_OK) return s;
   return run_attention(P, q, k, v, mask, o, st);
 }
+
+// Same estimator as prism_estimate, with the library's built-in scratch array in
+// place of a caller-provided workspace.  Nothing in the scratch has to start
+// at zero: every word a kernel reads was written earlier in the same call.
+int prism_estimate_noalloc(const prism_config* cfg, const void* q, const void* k, uint32_t* mask,
+                           prism_stream_t stream) {
+  Plan P;
+  int s = validate(cfg, &P);
+  if (s != PRISM_OK) return s;
+  if (!q || !k || !mask) return PRISM_ERR_NULL;
+  if (P.total > kStaticScratchBytes) return PRISM_ERR_SCRATCH_LIMIT;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(mask, 16)) return PRISM_ERR_ALIGN;
+  if ((s = ensure_device()) != PRISM_OK) return s;
+  void* scratch = nullptr;
+  if ((s = static_scratch(&scratch)) != PRISM_OK) return s;
+  return run_estimate(P, q, k, mask, static_cast<unsigned char*>(scratch),
+                      reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr);
+}
+
+size_t prism_noalloc_scratch_bytes(void) { return kStaticScratchBytes; }
 
 int prism_get_last_device_error(prism_stream_t stream) {
   if (ensure_device() != PRISM_OK) return PRISM_ERR_DEVICE;

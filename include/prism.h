@@ -60,8 +60,10 @@ enum {
   PRISM_ERR_CUDA = -8,        /* a CUDA runtime call failed (launch, attribute)     */
   PRISM_ERR_DEVICE = -9,      /* the device is not sm_100 (B200-class)              */
   PRISM_ERR_TIMEOUT = -10,    /* a kernel gave up a bounded wait (device error word) */
-  PRISM_ERR_TAU = -11         /* PRISM_TAU_EXPLICIT with a temperature that is not
+  PRISM_ERR_TAU = -11,        /* PRISM_TAU_EXPLICIT with a temperature that is not
                                  finite and > 0                                    */
+  PRISM_ERR_SCRATCH_LIMIT = -12 /* prism_estimate_noalloc: the problem needs more
+                                 scratch than prism_noalloc_scratch_bytes()        */
 };
 
 enum {
@@ -150,6 +152,37 @@ int prism_sparse_attn(const prism_config* cfg, const void* q, const void* k, con
 int prism_prefill(const prism_config* cfg, const void* q, const void* k, const void* v,
                   uint32_t* mask_out, void* o, void* workspace, size_t workspace_bytes,
                   prism_stream_t stream);
+
+/*
+ * Allocation-free estimator.  The paper has no counterpart to this entry
+ * point: it exists for callers that cannot allocate device memory -- for
+ * example a plugin inside a host framework that hands out no workspace, or a
+ * serving loop that forbids cudaMalloc after start-up because it can
+ * synchronise the device and fail under memory pressure.
+ *
+ * Computes exactly what prism_estimate computes (same kernels, same mask,
+ * bit for bit) but uses scratch built into the library: a fixed device array
+ * of prism_noalloc_scratch_bytes() = 32 MiB that every GPU loading the library
+ * holds until the process exits.  The caller still passes q, k and mask
+ * (device pointers, layouts as above); no dbg outputs.
+ *   - Problems whose workspace (prism_workspace_size) exceeds 32 MiB are
+ *     rejected with PRISM_ERR_SCRATCH_LIMIT before anything is enqueued
+ *     (the Llama-3-8B shape, 32 Q / 8 KV heads, batch 1, fits up to 54,912
+ *     tokens = 429 blocks).
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress while that device is current; make that first call
+ *     before any stream capture.
+ *   - Calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - Every call on a device shares the one array, which keeps the previous
+ *     call's contents: calls whose work overlaps on the GPU (different streams,
+ *     or host threads, without ordering between them) race on it.  Order them
+ *     on one stream, or synchronise between them.
+ */
+int prism_estimate_noalloc(const prism_config* cfg, const void* q, const void* k, uint32_t* mask,
+                           prism_stream_t stream);
+
+/* Size in bytes of the scratch built into prism_estimate_noalloc. */
+size_t prism_noalloc_scratch_bytes(void);
 
 /*
  * Reads and clears the device error word that kernels set when a bounded

@@ -1,0 +1,58 @@
+"""The allocation-free estimator entry point, prism_estimate_noalloc.
+
+Some callers cannot allocate device memory (a plugin whose host framework
+hands out no workspace, or a serving loop that forbids cudaMalloc after
+start-up because it may synchronise the device and fail under memory
+pressure).  prism_estimate_noalloc serves them from a fixed 32 MiB scratch
+array built into the library.  This file checks, through the C ABI, that it
+returns the same mask as prism_estimate, bit for bit, on two calls in a row
+with different inputs (so stale scratch from the first call cannot leak into
+the second), and that a problem too big for the array is refused on the host.
+It is collected last so a failure here never hides another test's result.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_band_b200 as pb
+from tests import gen
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+def _mask_via_workspace(cfg, qd, kd):
+    ws = torch.empty(pb.prism_workspace_size(cfg), dtype=torch.uint8, device=qd.device)
+    m = torch.zeros(qd.shape[0], qd.shape[1], cfg.nb, cfg.words, dtype=torch.int32, device=qd.device)
+    pb.prism_estimate(cfg, qd, kd, m, ws)
+    return m
+
+
+def test_noalloc_matches_workspace_entry_point_twice(cuda_device):
+    assert pb.prism_noalloc_scratch_bytes() == 32 << 20
+    cases = [gen.small_workload("noalloc_a", 1, 8, 2, 40 * 128, seed=51),
+             gen.small_workload("noalloc_b", 1, 8, 2, 40 * 128, seed=52, p=0.9)]
+    for w in cases:
+        q, k, _ = gen.make_inputs(w, with_v=False)
+        qd, kd = q.to(cuda_device), k.to(cuda_device)
+        cfg = P.make_cfg(w)
+        ref = _mask_via_workspace(cfg, qd, kd)
+        got = torch.full_like(ref, 0x5A5A5A5A)
+        status = pb.lib.prism_estimate_noalloc(cfg.ptr(), qd.data_ptr(), kd.data_ptr(), got.data_ptr(),
+                                               torch.cuda.current_stream().cuda_stream)
+        assert status == 0, pb.prism_status_str(status)
+        torch.cuda.synchronize()
+        assert pb.prism_get_last_device_error() == 0
+        assert torch.equal(got, ref), f"{w.name}: {(got != ref).sum().item()} mask words differ"
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch(cuda_device):
+    hi, lo = gen.default_bands()
+    fits = pb.PrismConfig(1, 32, 8, 429 * 128, hi, lo, 0.95)
+    too_big = pb.PrismConfig(1, 32, 8, 430 * 128, hi, lo, 0.95)
+    assert pb.prism_workspace_size(fits) <= pb.prism_noalloc_scratch_bytes()
+    assert pb.prism_workspace_size(too_big) > pb.prism_noalloc_scratch_bytes()
+    a = 1 << 20  # never dereferenced: the size check runs before anything is enqueued
+    assert pb.lib.prism_estimate_noalloc(too_big.ptr(), a, a, a, None) == -12
