@@ -5,65 +5,136 @@
 // attention blocks; here the subset is the estimator's mask M (one bit per
 // (query block i, key block j)), token-causal inside the diagonal block.
 //
-// One CTA per (batch, Q head, query block i) of 128 queries, 192 threads:
-//   warp 5        TMA producer: Q once, then K_j / V_j of every kept block j
-//                 into a 2-stage ring (128-byte swizzled, 2 x 16 KB halves)
-//   warp 4        MMA issuer (one thread): S = Q K_j^T, then O += P V_j,
-//                 tcgen05.mma kind::f16 (bf16 in, fp32 accumulate in tensor
-//                 memory: S in columns 0-127, O in columns 128-255)
-//   warps 0-3     softmax: thread r owns query row r (tensor-memory lane r),
-//                 reads its S row, keeps the running max / sum (base-2
-//                 exponent), rescales its O row when the max grows, writes
-//                 P (bf16) into shared memory in the MMA operand layout, and
-//                 at the end normalises O and stores it as bf16.
-// Grid order runs query blocks from the last (most key blocks) to the first,
-// so long rows start early.
+// Work item = two 128-query tiles that read the same KV head (for GQA, two Q
+// heads of one group at the same query block), so every K/V tile fetched by
+// TMA serves both.  The key blocks visited are the union of the two tiles'
+// kept sets; each tile computes only its own kept blocks.
+//
+// 320 threads (10 warps):
+//   warp 0      TMA producer: Q_A, Q_B once; K_j, V_j of every visited block
+//               into a 2-stage ring (128-byte swizzled, two 16 KB halves each)
+//   warp 1      MMA issuer (one thread), tcgen05.mma kind::f16, bf16 in /
+//               fp32 accumulate in tensor memory (512 columns):
+//                 S_A = cols [0,128)  S_B = [128,256)  O_A = [256,384)  O_B = [384,512)
+//               S = Q K_j^T (A and B from shared memory), then O += P V_j
+//               with P read from tensor memory (bf16, written over S).
+//               Issue order: PV_A(t), QK_A(t+1), PV_B(t), QK_B(t+1), so one
+//               tile's softmax overlaps the other tile's matrix products.
+//   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B: thread =
+//               query row = tensor-memory lane 32*(warp%4)+lane.  Online
+//               softmax in base 2; O is rescaled in tensor memory only when
+//               the running max grows by more than 8 (a factor 256), so the
+//               unnormalised values stay bounded and most steps skip it.
+// The grid runs items from the last query block (most key blocks) down.
 #pragma once
 #include "ptx.cuh"
 
 namespace prism {
 namespace attn {
 
-constexpr int kThreads = 192;
-constexpr int kStages = 2;
-constexpr uint32_t kHalfBytes = 128 * 64 * 2;     // 128 rows x 64 bf16 (one swizzle span)
-constexpr uint32_t kTileBytes = 2 * kHalfBytes;   // 128 x 128 bf16
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTileBytes;
-constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
-constexpr uint32_t kOffP = kOffV + kStages * kTileBytes;
-constexpr uint32_t kOffBar = kOffP + kTileBytes;
+constexpr int kThreads = 320;
+constexpr uint32_t kHalfBytes = 128 * 64 * 2;    // 128 rows x 64 bf16 (one swizzle span)
+constexpr uint32_t kTileBytes = 2 * kHalfBytes;  // 128 x 128 bf16
+constexpr uint32_t kOffQ = 0;                    // Q_A, Q_B
+constexpr uint32_t kOffK = 2 * kTileBytes;       // 2 stages
+constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;
+constexpr uint32_t kOffBar = kOffV + 2 * kTileBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + slack for 1024-byte alignment
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-// Iterates the kept key blocks j <= i of one mask row in ascending order.
-struct KeptIter {
-  const uint32_t* row;
+// Barrier slots (8 bytes each) after kOffBar.
+enum : uint32_t {
+  kBarQ = 0,
+  kBarKFull = 1,    // [2]
+  kBarVFull = 3,    // [2]
+  kBarKVEmpty = 5,  // [2]
+  kBarSFull = 7,    // [2] per tile
+  kBarPFull = 9,    // [2] per tile
+  kBarODone = 11,   // [2] per tile
+  kNumBars = 13
+};
+
+// One 128-query tile of a work item.
+struct Tile {
+  int valid;  // 0: the item has a single tile
+  int i;      // query block
+  int bh;     // batch * hq + head
+  const uint32_t* mrow;
   int last_word;
   uint32_t last_mask;
-  int w;
-  uint32_t bits;
-  __device__ __forceinline__ void init(const uint32_t* r, int i) {
-    row = r;
-    last_word = i >> 5;
-    last_mask = ((i & 31) == 31) ? 0xffffffffu : ((2u << (i & 31)) - 1u);
-    w = 0;
-    bits = load(0);
-  }
-  __device__ __forceinline__ uint32_t load(int ww) const {
-    uint32_t b = row[ww];
-    return ww == last_word ? (b & last_mask) : b;
-  }
-  __device__ __forceinline__ int next() {
-    while (bits == 0u) {
-      if (++w > last_word) return -1;
-      bits = load(w);
-    }
-    const int b = __ffs(bits) - 1;
-    bits &= bits - 1u;
-    return (w << 5) + b;
+  __device__ __forceinline__ uint32_t word(int w) const {
+    if (!valid || w > last_word) return 0u;
+    const uint32_t b = mrow[w];
+    return w == last_word ? (b & last_mask) : b;
   }
 };
+
+__device__ __forceinline__ void make_tile(Tile& t, int row, int rows_total, int G, int nb, int kv_global,
+                                          int hq, const uint32_t* mask, int W) {
+  t.valid = row < rows_total;
+  const int r = t.valid ? row : 0;
+  t.i = nb - 1 - r / G;
+  const int bi = kv_global / (hq / G);  // batch of this KV head
+  const int kv = kv_global - bi * (hq / G);
+  const int h = kv * G + r % G;
+  t.bh = bi * hq + h;
+  t.mrow = mask + ((size_t)t.bh * nb + t.i) * W;
+  t.last_word = t.i >> 5;
+  t.last_mask = ((t.i & 31) == 31) ? 0xffffffffu : ((2u << (t.i & 31)) - 1u);
+}
+
+// Walks the union of the two tiles' kept blocks in ascending order.
+struct UnionIter {
+  const Tile* a;
+  const Tile* b;
+  int w, last_word;
+  uint32_t bits;
+  __device__ __forceinline__ void init(const Tile* ta, const Tile* tb) {
+    a = ta;
+    b = tb;
+    last_word = max(ta->valid ? ta->last_word : -1, tb->valid ? tb->last_word : -1);
+    w = 0;
+    bits = last_word >= 0 ? (a->word(0) | b->word(0)) : 0u;
+  }
+  // returns j or -1; sets in_a / in_b
+  __device__ __forceinline__ int next(bool& in_a, bool& in_b) {
+    while (bits == 0u) {
+      if (++w > last_word) return -1;
+      bits = a->word(w) | b->word(w);
+    }
+    const int bit = __ffs(bits) - 1;
+    bits &= bits - 1u;
+    in_a = (a->word(w) >> bit) & 1u;
+    in_b = (b->word(w) >> bit) & 1u;
+    return (w << 5) + bit;
+  }
+};
+
+__device__ __forceinline__ int count_kept(const Tile& t) {
+  if (!t.valid) return 0;
+  int n = 0;
+  for (int w = 0; w <= t.last_word; ++w) n += __popc(t.word(w));
+  return n;
+}
+
+__device__ __forceinline__ void mma_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);  // Q K-major, K K-major
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+    mma_bf16_ss(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024), smem_desc_sw128(k_smem + off, 16, 1024),
+                idesc, kk > 0);
+  }
+}
+
+__device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 1);  // P K-major (TMEM), V MN-major
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_bf16_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(v_smem + kk * 2048, kHalfBytes, 1024), idesc,
+                (accumulate || kk > 0) ? 1u : 0u);
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -74,44 +145,30 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   unsigned char* sgen = smem_raw + (sbase - raw);
-  const uint32_t bar_q = sbase + kOffBar;
-  const uint32_t bar_kv_full = bar_q + 8;    // [2]
-  const uint32_t bar_kv_empty = bar_q + 24;  // [2]
-  const uint32_t bar_s_full = bar_q + 40;
-  const uint32_t bar_p_full = bar_q + 48;
-  const uint32_t bar_o_full = bar_q + 56;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sgen + kOffBar + 128);
+  const uint32_t bars = sbase + kOffBar;
+  auto bar = [&](uint32_t slot) { return bars + 8u * slot; };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sgen + kOffBar + 8 * kNumBars + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = batch * hq;
-  const int i = nb - 1 - (int)(blockIdx.x / BH);
-  const int bh = (int)(blockIdx.x % BH);
-  const int bi = bh / hq, h = bh - bi * hq;
-  const int kvh = bi * hkv + h / (hq / hkv);
+  const int G = hq / hkv;
+  const int rows_per_kv = G * nb;
+  const int items_per_kv = (rows_per_kv + 1) >> 1;
+  const int kv_total = batch * hkv;
+  const int m = (int)(blockIdx.x / kv_total);
+  const int kv_global = (int)(blockIdx.x % kv_total);
   const int W = (nb + 31) >> 5;
-  const uint32_t* mrow = mask + ((size_t)bh * nb + i) * W;
-
-  // number of kept blocks j <= i (same value in every thread)
-  int n_kept = 0;
-  {
-    KeptIter it;
-    it.init(mrow, i);
-    n_kept = __popc(it.bits);
-    for (int ww = 1; ww <= it.last_word; ++ww) n_kept += __popc(it.load(ww));
-  }
+  (void)items_per_kv;
+  Tile tiles[2];
+  make_tile(tiles[0], 2 * m, rows_per_kv, G, nb, kv_global, hq, mask, W);
+  make_tile(tiles[1], 2 * m + 1, rows_per_kv, G, nb, kv_global, hq, mask, W);
+  const int kv_row0 = kv_global * seqlen;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 1);
-    mbar_init(bar_kv_full, 1);
-    mbar_init(bar_kv_full + 8, 1);
-    mbar_init(bar_kv_empty, 1);
-    mbar_init(bar_kv_empty + 8, 1);
-    mbar_init(bar_s_full, 1);
-    mbar_init(bar_p_full, 128);
-    mbar_init(bar_o_full, 1);
+    for (uint32_t s = 0; s < kNumBars; ++s)
+      mbar_init(bar(s), (s == kBarPFull || s == kBarPFull + 1) ? 128u : 1u);
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), kTmemCols);
     tmem_relinquish();
   }
@@ -119,161 +176,202 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tS = tmem, tO = tmem + 128;
 
-  if (warp == 5) {
+  if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && n_kept > 0) {
+    if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      const int q_row = bh * seqlen + i * 128;
-      mbar_arrive_expect_tx(bar_q, kTileBytes);
-      tma_load_2d(sbase + kOffQ, &tmQ, 0, q_row, bar_q);
-      tma_load_2d(sbase + kOffQ + kHalfBytes, &tmQ, 64, q_row, bar_q);
-      KeptIter it;
-      it.init(mrow, i);
-      for (int t = 0;; ++t) {
-        const int j = it.next();
-        if (j < 0) break;
-        const int s = t & 1;
-        if (t >= kStages && !mbar_wait(bar_kv_empty + 8 * s, ((t >> 1) - 1) & 1)) break;
-        const uint32_t full = bar_kv_full + 8 * s;
-        mbar_arrive_expect_tx(full, 2 * kTileBytes);
-        const int kr = kvh * seqlen + j * 128;
-        const uint32_t kd = sbase + kOffK + s * kTileBytes, vd = sbase + kOffV + s * kTileBytes;
-        tma_load_2d(kd, &tmK, 0, kr, full);
-        tma_load_2d(kd + kHalfBytes, &tmK, 64, kr, full);
-        tma_load_2d(vd, &tmV, 0, kr, full);
-        tma_load_2d(vd + kHalfBytes, &tmV, 64, kr, full);
+      const int nA = count_kept(tiles[0]), nB = count_kept(tiles[1]);
+      if (nA + nB > 0) {
+        mbar_arrive_expect_tx(bar(kBarQ), (nA > 0 ? kTileBytes : 0) + (nB > 0 ? kTileBytes : 0));
+        for (int x = 0; x < 2; ++x) {
+          if ((x == 0 ? nA : nB) == 0) continue;
+          const int q_row = tiles[x].bh * seqlen + tiles[x].i * 128;
+          tma_load_2d(sbase + kOffQ + x * kTileBytes, &tmQ, 0, q_row, bar(kBarQ));
+          tma_load_2d(sbase + kOffQ + x * kTileBytes + kHalfBytes, &tmQ, 64, q_row, bar(kBarQ));
+        }
+        UnionIter it;
+        it.init(&tiles[0], &tiles[1]);
+        bool ia, ib;
+        for (int t = 0;; ++t) {
+          const int j = it.next(ia, ib);
+          if (j < 0) break;
+          const int s = t & 1;
+          if (t >= 2 && !mbar_wait(bar(kBarKVEmpty + s), ((t >> 1) - 1) & 1)) break;
+          const int kr = kv_row0 + j * 128;
+          const uint32_t kd = sbase + kOffK + s * kTileBytes, vd = sbase + kOffV + s * kTileBytes;
+          mbar_arrive_expect_tx(bar(kBarKFull + s), kTileBytes);
+          tma_load_2d(kd, &tmK, 0, kr, bar(kBarKFull + s));
+          tma_load_2d(kd + kHalfBytes, &tmK, 64, kr, bar(kBarKFull + s));
+          mbar_arrive_expect_tx(bar(kBarVFull + s), kTileBytes);
+          tma_load_2d(vd, &tmV, 0, kr, bar(kBarVFull + s));
+          tma_load_2d(vd + kHalfBytes, &tmV, 64, kr, bar(kBarVFull + s));
+        }
       }
     }
-  } else if (warp == 4) {
+  } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_kept > 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);  // Q K-major, K K-major
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);  // P K-major, V MN-major
-      if (mbar_wait(bar_q, 0)) {
-        for (int t = 0; t < n_kept; ++t) {
+    if (lane == 0) {
+      const int nA = count_kept(tiles[0]), nB = count_kept(tiles[1]);
+      if (nA + nB > 0 && mbar_wait(bar(kBarQ), 0)) {
+        const uint32_t tS[2] = {tmem, tmem + 128};
+        const uint32_t tO[2] = {tmem + 256, tmem + 384};
+        const uint32_t qs[2] = {sbase + kOffQ, sbase + kOffQ + kTileBytes};
+        int u[2] = {0, 0};  // per-tile count of P V products issued
+        UnionIter it;
+        it.init(&tiles[0], &tiles[1]);
+        bool in_cur[2], in_nxt[2];
+        int j = it.next(in_cur[0], in_cur[1]);
+        bool ok = mbar_wait(bar(kBarKFull + 0), 0);
+        if (ok) {
+          tc_fence_after();
+          for (int x = 0; x < 2; ++x)
+            if (in_cur[x]) {
+              mma_qk(tS[x], qs[x], sbase + kOffK);
+              mma_commit(bar(kBarSFull + x));
+            }
+        }
+        for (int t = 0; ok && j >= 0; ++t) {
           const int s = t & 1;
-          if (!mbar_wait(bar_kv_full + 8 * s, (t >> 1) & 1)) break;
-          tc_fence_after();
-          const uint32_t kb = sbase + kOffK + s * kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-            mma_bf16_ss(tS, smem_desc_sw128(sbase + kOffQ + off, 16, 1024),
-                        smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0);
+          const int jn = it.next(in_nxt[0], in_nxt[1]);
+          if (!(ok = mbar_wait(bar(kBarVFull + s), (t >> 1) & 1))) break;
+          bool k_ready = false;
+          for (int x = 0; x < 2; ++x) {
+            if (in_cur[x]) {
+              if (!(ok = mbar_wait(bar(kBarPFull + x), u[x] & 1))) break;
+              tc_fence_after();
+              mma_pv(tO[x], tS[x], sbase + kOffV + s * kTileBytes, u[x] > 0);
+              mma_commit(bar(kBarODone + x));
+              ++u[x];
+            }
+            if (jn >= 0 && in_nxt[x]) {
+              if (!k_ready) {
+                if (!(ok = mbar_wait(bar(kBarKFull + (s ^ 1)), ((t + 1) >> 1) & 1))) break;
+                tc_fence_after();
+                k_ready = true;
+              }
+              mma_qk(tS[x], qs[x], sbase + kOffK + (s ^ 1) * kTileBytes);
+              mma_commit(bar(kBarSFull + x));
+            }
           }
-          mma_commit(bar_s_full);
-          if (!mbar_wait(bar_p_full, t & 1)) break;
-          tc_fence_after();
-          const uint32_t vb = sbase + kOffV + s * kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t aoff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-            mma_bf16_ss(tO, smem_desc_sw128(sbase + kOffP + aoff, 16, 1024),
-                        smem_desc_sw128(vb + kk * 2048, kHalfBytes, 1024), idesc_pv,
-                        (t > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(bar_kv_empty + 8 * s);
-          mma_commit(bar_o_full);
+          if (!ok) break;
+          mma_commit(bar(kBarKVEmpty + s));
+          j = jn;
+          in_cur[0] = in_nxt[0];
+          in_cur[1] = in_nxt[1];
         }
       }
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int r = threadIdx.x;  // query row within the block == TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    __nv_bfloat16* orow = out + ((size_t)bh * seqlen + (size_t)i * 128 + r) * 128;
+    const int x = (warp - 2) >> 2;          // tile
+    const int qw = warp & 3;                // TMEM lane quarter of this warp
+    const int r = qw * 32 + lane;           // query row == TMEM lane
+    const uint32_t lane_base = (uint32_t)(qw * 32) << 16;
+    const uint32_t tS = tmem + 128 * x + lane_base;
+    const uint32_t tO = tmem + 256 + 128 * x + lane_base;
+    const Tile& T = tiles[x];
+    const int n = count_kept(T);
     bool ok = true;
     float m_run = -INFINITY, l_run = 0.f;
-    KeptIter it;
-    it.init(mrow, i);
-    for (int t = 0; t < n_kept; ++t) {
-      const int j = it.next();
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, t & 1));
+    int w = 0;
+    uint32_t bits = T.word(0);
+    for (int u = 0; u < n; ++u) {
+      while (bits == 0u) bits = T.word(++w);
+      const int j = (w << 5) + __ffs(bits) - 1;
+      bits &= bits - 1u;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarSFull + x), u & 1));
       if (!ok) break;
       tc_fence_after();
-      float x[128];
+      // pass 1 over S: the row max (diagonal block: keys c <= r only)
+      const bool diag = (j == T.i);
+      float mx = -INFINITY;
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
         uint32_t v[32];
-        tmem_ld32(tS + lane_base + c4 * 32, v);
+        tmem_ld32(tS + c4 * 32, v);
         tmem_wait_ld_dep(v);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[c4 * 32 + e] = __uint_as_float(v[e]) * scale_log2;
+        for (int e = 0; e < 32; ++e) {
+          const float val = __uint_as_float(v[e]);
+          mx = (diag && c4 * 32 + e > r) ? mx : fmaxf(mx, val);
+        }
       }
-      if (j == i) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c > r) x[c] = -INFINITY;
-      }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, x[c]);
-      const float m_new = fmaxf(m_run, mx);
-      float rs = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        x[c] = exp2f(x[c] - m_new);
-        rs += x[c];
-      }
-      if (t > 0) {
-        // the previous P V must be done before O is rescaled and P is rewritten
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_o_full, (t - 1) & 1));
+      mx *= scale_log2;
+      // lazy rescale: move the reference max only when it grows by > threshold
+      const bool grow = (u == 0) || (mx > m_run + kRescaleThreshold);
+      const float m_new = grow ? fmaxf(mx, m_run) : m_run;
+      if (u > 0) {
+        // P V of the previous step must finish before O is touched or P rewritten
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarODone + x), (u - 1) & 1));
         if (!ok) break;
         tc_fence_after();
-        const float alpha = exp2f(m_run - m_new);
-        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+        if (__any_sync(0xffffffffu, grow)) {
+          const float alpha = grow ? exp2f(m_run - m_new) : 1.0f;
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
             uint32_t v[32];
-            tmem_ld32(tO + lane_base + c4 * 32, v);
+            tmem_ld32(tO + c4 * 32, v);
             tmem_wait_ld_dep(v);
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-            tmem_st32(tO + lane_base + c4 * 32, v);
+            tmem_st32(tO + c4 * 32, v);
           }
-          tmem_wait_st();
+          l_run *= alpha;
         }
-        l_run = l_run * alpha + rs;
-      } else {
-        l_run = rs;
       }
       m_run = m_new;
-      // P row r -> shared memory, 128-byte swizzled K-major layout:
-      // half ch holds keys 64ch..64ch+63; row r at (r/8)*1024 + (r%8)*128;
-      // 16-byte chunk u stored at chunk position u ^ (r % 8).
-      unsigned char* prow = sgen + kOffP + (r >> 3) * 1024 + (r & 7) * 128;
+      // pass 2 over S: P = exp2(S * scale - m) in bf16, written over S[:, 0:64)
+      float rs = 0.f;
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch)
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t v0[32], v1[32], pk[32];
+        tmem_ld32(tS + h2 * 64, v0);
+        tmem_ld32(tS + h2 * 64 + 32, v1);
+        tmem_wait_ld_dep(v0);
+        tmem_wait_ld_dep(v1);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int c0 = ch * 64 + u * 8;
-          uint4 pk;
-          pk.x = pack_bf16x2(x[c0 + 0], x[c0 + 1]);
-          pk.y = pack_bf16x2(x[c0 + 2], x[c0 + 3]);
-          pk.z = pack_bf16x2(x[c0 + 4], x[c0 + 5]);
-          pk.w = pack_bf16x2(x[c0 + 6], x[c0 + 7]);
-          *reinterpret_cast<uint4*>(prow + ch * kHalfBytes + ((u ^ (r & 7)) << 4)) = pk;
+        for (int e = 0; e < 16; ++e) {
+          const int c = h2 * 64 + 2 * e;
+          float p0 = exp2f(fmaf(__uint_as_float(v0[2 * e]), scale_log2, -m_run));
+          float p1 = exp2f(fmaf(__uint_as_float(v0[2 * e + 1]), scale_log2, -m_run));
+          if (diag && c > r) p0 = 0.f;
+          if (diag && c + 1 > r) p1 = 0.f;
+          rs += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
         }
-      fence_proxy_async_smem();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c = h2 * 64 + 32 + 2 * e;
+          float p0 = exp2f(fmaf(__uint_as_float(v1[2 * e]), scale_log2, -m_run));
+          float p1 = exp2f(fmaf(__uint_as_float(v1[2 * e + 1]), scale_log2, -m_run));
+          if (diag && c > r) p0 = 0.f;
+          if (diag && c + 1 > r) p1 = 0.f;
+          rs += p0 + p1;
+          pk[16 + e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS + h2 * 32, pk);
+      }
+      l_run += rs;
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_p_full);
+      mbar_arrive(bar(kBarPFull + x));
     }
     // ------------------------------------------------------------ epilogue
-    if (n_kept == 0) {
+    __nv_bfloat16* orow = T.valid ? out + ((size_t)T.bh * seqlen + (size_t)T.i * 128 + r) * 128 : nullptr;
+    if (T.valid && n == 0) {
       const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
       for (int c = 0; c < 16; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
-    } else if (ok && __all_sync(0xffffffffu, mbar_wait(bar_o_full, (n_kept - 1) & 1))) {
+    } else if (T.valid && ok && __all_sync(0xffffffffu, mbar_wait(bar(kBarODone + x), (n - 1) & 1))) {
       tc_fence_after();
       const float inv = 1.0f / l_run;
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
         uint32_t v[32];
-        tmem_ld32(tO + lane_base + c4 * 32, v);
+        tmem_ld32(tO + c4 * 32, v);
         tmem_wait_ld_dep(v);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
@@ -289,10 +387,16 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// Number of work items (CTAs) for a problem.
+__host__ __forceinline__ unsigned grid_size(int batch, int hq, int hkv, int nb) {
+  const int G = hq / hkv;
+  return (unsigned)batch * hkv * (unsigned)((G * nb + 1) / 2);
 }
 
 }  // namespace attn

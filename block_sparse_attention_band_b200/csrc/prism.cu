@@ -231,7 +231,7 @@ int run_attention(const Plan& P, const void* q, const void* k, const void* v, co
       make_map(&mv, v, (size_t)P.kv_rows * P.n) != PRISM_OK)
     return PRISM_ERR_CUDA;
   const float scale_log2 = P.scale * 1.4426950408889634f;
-  const unsigned grid = (unsigned)P.q_rows * (unsigned)P.nb;
+  const unsigned grid = attn::grid_size(P.b, P.hq, P.hkv, P.nb);
   attn::sparse_attn_kernel<<<grid, attn::kThreads, attn::kSmemBytes, st>>>(
       mq, mk, mv, mask, reinterpret_cast<__nv_bfloat16*>(o), P.b, P.hq, P.hkv, P.n, P.nb, scale_log2);
   return launched();

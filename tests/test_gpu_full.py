@@ -1,0 +1,74 @@
+"""Full-size workloads in the launch configuration bench.py times
+(prism_prefill, workspace, mask out), checked on samples the oracle can
+compute one by one, plus properties that hold at any size.
+
+Sampling: the estimator oracle runs on 4 Q heads (one from each of 4 KV
+groups, the seed picks the head within the group); the attention oracle on
+those heads x query blocks {0, 1, nb/2, nb-1} and two seeded random blocks.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_band_b200 as pb
+import oracle
+from tests import gen
+from tests import parity as P
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+FULL = ["llama3_8b_32k", "llama3_8b_128k", "qwen3_8b_64k_planted", "sweep_8k", "sweep_256k"]
+
+
+def _sample_heads(w, rng):
+    g = w.hq // w.hkv
+    groups = sorted(rng.choice(w.hkv, min(4, w.hkv), replace=False).tolist())
+    return [kv * g + int(rng.integers(g)) for kv in groups]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled_parity(name, cuda_device):
+    w = gen.WORKLOADS[name]
+    rng = np.random.default_rng(zlib.crc32(name.encode()))
+    q, k, v = gen.make_inputs(w)
+    qd, kd, vd = q.to(cuda_device), k.to(cuda_device), v.to(cuda_device)
+    cfg = P.make_cfg(w)
+    nb, W = w.nb, cfg.words
+    ws = torch.empty(pb.prism_workspace_size(cfg), dtype=torch.uint8, device=cuda_device)
+    mask = torch.empty(w.batch, w.hq, nb, W, dtype=torch.int32, device=cuda_device)
+    o = torch.empty_like(qd)
+    pb.prism_prefill(cfg, qd, kd, vd, mask, o, ws)
+    torch.cuda.synchronize()
+    assert pb.prism_get_last_device_error() == 0
+    words = mask.cpu().numpy().view(np.uint32)
+
+    # properties at full size: causal, >= 1 block per row, finite output
+    mb = oracle.unpack_mask(words, nb)
+    assert not np.any(mb & ~np.tril(np.ones((nb, nb), dtype=bool)))
+    assert np.all(mb.sum(-1) >= 1)
+    assert torch.isfinite(o.float()).all()
+
+    # scores / tau on sampled heads (same estimator launch, debug outputs on)
+    heads = _sample_heads(w, rng)
+    tri = nb * (nb + 1) // 2
+    scores = torch.empty(w.batch, w.hq, 2, tri, dtype=torch.float32, device=cuda_device)
+    tau = torch.empty(w.batch, w.hq, 2, dtype=torch.float32, device=cuda_device)
+    mask2 = torch.empty_like(mask)
+    pb.prism_estimate(cfg, qd, kd, mask2, ws, dbg_scores=scores, dbg_tau=tau)
+    torch.cuda.synchronize()
+    assert torch.equal(mask2, mask), "estimate and prefill disagree on the mask"
+    hi, lo = gen.default_bands()
+    ref = P.oracle_estimate_streamed(q, k, (hi, lo), w.p, heads=heads)
+    sc = P.unpack_tri(scores[0, heads].cpu().double().numpy(), nb)
+    P.check_tau(tau[0, heads].cpu().double().numpy(), ref)
+    P.check_scores(sc, ref)
+    n_diff, n_exempt = P.check_mask(mb[0, heads], ref, w.p)
+    print(f"{name}: density {P.density(mb):.4f}, sampled-head mask mismatches {n_diff} (all exempt: {n_exempt})")
+
+    # attention on sampled (head, query block) rows with the GPU's mask
+    blocks = sorted({0, 1, nb // 2, nb - 1} | set(rng.integers(0, nb, 2).tolist()))
+    rows = [(0, h, i) for h in heads for i in blocks]
+    worst = P.check_attention_rows(o, q, k, v, mb, rows, w.hq // w.hkv)
+    print(f"{name}: attention rows {len(rows)}, max-abs {worst[0]:.3g}, mean-abs {worst[1]:.3g}")

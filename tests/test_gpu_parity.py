@@ -31,6 +31,8 @@ CASES = [
     gen.small_workload("planted_nb70", 1, 4, 2, 70 * 128, seed=26, p=0.93, rope_base=1e6,
                        stripes=True, slash=True),
     gen.small_workload("segments_nb40", 1, 8, 2, 40 * 128, seed=27, segment=1024),
+    gen.small_workload("gqa3_nb9", 1, 3, 1, 9 * 128, seed=28),
+    gen.small_workload("mha_b2_nb5", 2, 3, 3, 5 * 128, seed=29),
 ]
 
 
@@ -53,7 +55,7 @@ def test_estimator_parity(w, cuda_device):
     print(f"{w.name}: density {P.density(mask):.3f} mismatches {n_diff} (exempt {n_exempt})")
 
 
-@pytest.mark.parametrize("w", CASES[:4] + CASES[6:7], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", CASES[:4] + CASES[6:7] + CASES[8:], ids=lambda w: w.name)
 def test_attention_parity_with_estimator_mask(w, cuda_device):
     q, k, v, qd, kd, vd = _inputs(w, cuda_device)
     cfg = P.make_cfg(w)
