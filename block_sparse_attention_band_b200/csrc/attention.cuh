@@ -136,6 +136,47 @@ __device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_
                 (accumulate || kk > 0) ? 1u : 0u);
 }
 
+// Writes P = exp2(S * scale_log2 - m) as bf16 over columns [0, 64) of this
+// thread's S row and returns the row sum of the fp32 values.  Packed f32x2
+// arithmetic for the scale/shift and the sum; four independent partial sums
+// keep the dependency chains short.  DIAG zeroes keys c > r (causal diagonal).
+template <bool DIAG>
+__device__ __forceinline__ float softmax_p(uint32_t tS, float scale_log2, float m, int r) {
+  const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
+  const uint64_t nm2 = f2_pack(-m, -m);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+    uint32_t v0[32], v1[32], pk[32];
+    tmem_ld32(tS + h2 * 64, v0);
+    tmem_ld32(tS + h2 * 64 + 32, v1);
+    tmem_wait_ld_dep(v0);
+    tmem_wait_ld_dep(v1);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const uint32_t* src = e < 16 ? v0 : v1;
+      const int ee = e & 15;
+      const uint64_t x2 =
+          f2_fma(f2_pack(__uint_as_float(src[2 * ee]), __uint_as_float(src[2 * ee + 1])), sc2, nm2);
+      float x0, x1;
+      f2_unpack(x2, x0, x1);
+      float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+      if (DIAG) {
+        const int c = h2 * 64 + 2 * e;
+        if (c > r) p0 = 0.f;
+        if (c + 1 > r) p1 = 0.f;
+      }
+      acc[e & 3] = f2_add(acc[e & 3], f2_pack(p0, p1));
+      pk[e] = pack_bf16x2(p0, p1);
+    }
+    tmem_st32(tS + h2 * 32, pk);
+  }
+  const uint64_t t2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+  float a0, a1;
+  f2_unpack(t2, a0, a1);
+  return a0 + a1;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const uint32_t* __restrict__ mask,
@@ -287,16 +328,37 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc_fence_after();
       // pass 1 over S: the row max (diagonal block: keys c <= r only)
       const bool diag = (j == T.i);
-      float mx = -INFINITY;
+      float mx;
+      if (!diag) {
+        float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t v[32];
-        tmem_ld32(tS + c4 * 32, v);
-        tmem_wait_ld_dep(v);
+        for (int c8 = 0; c8 < 2; ++c8) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tS + c8 * 64, v0);
+          tmem_ld32(tS + c8 * 64 + 32, v1);
+          tmem_wait_ld_dep(v0);
+          tmem_wait_ld_dep(v1);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float val = __uint_as_float(v[e]);
-          mx = (diag && c4 * 32 + e > r) ? mx : fmaxf(mx, val);
+          for (int e = 0; e < 16; ++e) {
+            mc[e & 1] = max3f(mc[e & 1], __uint_as_float(v0[2 * e]), __uint_as_float(v0[2 * e + 1]));
+            mc[2 + (e & 1)] = max3f(mc[2 + (e & 1)], __uint_as_float(v1[2 * e]), __uint_as_float(v1[2 * e + 1]));
+          }
+        }
+        mx = fmaxf(max3f(mc[0], mc[1], mc[2]), mc[3]);
+      } else {
+        mx = -INFINITY;
+#pragma unroll
+        for (int c8 = 0; c8 < 2; ++c8) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tS + c8 * 64, v0);
+          tmem_ld32(tS + c8 * 64 + 32, v1);
+          tmem_wait_ld_dep(v0);
+          tmem_wait_ld_dep(v1);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            mx = (c8 * 64 + e > r) ? mx : fmaxf(mx, __uint_as_float(v0[e]));
+            mx = (c8 * 64 + 32 + e > r) ? mx : fmaxf(mx, __uint_as_float(v1[e]));
+          }
         }
       }
       mx *= scale_log2;
@@ -309,7 +371,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (!ok) break;
         tc_fence_after();
         if (__any_sync(0xffffffffu, grow)) {
-          const float alpha = grow ? exp2f(m_run - m_new) : 1.0f;
+          const float alpha = grow ? fast_exp2(m_run - m_new) : 1.0f;
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
             uint32_t v[32];
@@ -324,36 +386,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
       m_run = m_new;
       // pass 2 over S: P = exp2(S * scale - m) in bf16, written over S[:, 0:64)
-      float rs = 0.f;
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t v0[32], v1[32], pk[32];
-        tmem_ld32(tS + h2 * 64, v0);
-        tmem_ld32(tS + h2 * 64 + 32, v1);
-        tmem_wait_ld_dep(v0);
-        tmem_wait_ld_dep(v1);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c = h2 * 64 + 2 * e;
-          float p0 = exp2f(fmaf(__uint_as_float(v0[2 * e]), scale_log2, -m_run));
-          float p1 = exp2f(fmaf(__uint_as_float(v0[2 * e + 1]), scale_log2, -m_run));
-          if (diag && c > r) p0 = 0.f;
-          if (diag && c + 1 > r) p1 = 0.f;
-          rs += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
-        }
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c = h2 * 64 + 32 + 2 * e;
-          float p0 = exp2f(fmaf(__uint_as_float(v1[2 * e]), scale_log2, -m_run));
-          float p1 = exp2f(fmaf(__uint_as_float(v1[2 * e + 1]), scale_log2, -m_run));
-          if (diag && c > r) p0 = 0.f;
-          if (diag && c + 1 > r) p1 = 0.f;
-          rs += p0 + p1;
-          pk[16 + e] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(tS + h2 * 32, pk);
-      }
+      const float rs = diag ? softmax_p<true>(tS, scale_log2, m_run, r) : softmax_p<false>(tS, scale_log2, m_run, r);
       l_run += rs;
       tmem_wait_st();
       tc_fence_before();
