@@ -10,7 +10,8 @@
 // TMA serves both.  The key blocks visited are the union of the two tiles'
 // kept sets; each tile computes only its own kept blocks.
 //
-// 320 threads (10 warps):
+// 384 threads (12 warps; registers re-split per warpgroup: warps 0-3 keep 72,
+// the two softmax warpgroups get 216 so a whole S row stays in registers):
 //   warp 0      TMA producer: Q_A, Q_B once; K_j, V_j of every visited block
 //               into a 2-stage ring (128-byte swizzled, two 16 KB halves each)
 //   warp 1      MMA issuer (one thread), tcgen05.mma kind::f16, bf16 in /
@@ -20,7 +21,8 @@
 //               with P read from tensor memory (bf16, written over S).
 //               Issue order: PV_A(t), QK_A(t+1), PV_B(t), QK_B(t+1), so one
 //               tile's softmax overlaps the other tile's matrix products.
-//   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B: thread =
+//   warps 2-3   idle
+//   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: thread =
 //               query row = tensor-memory lane 32*(warp%4)+lane.  Online
 //               softmax in base 2; O is rescaled in tensor memory only when
 //               the running max grows by more than 8 (a factor 256), so the
@@ -32,7 +34,13 @@
 namespace prism {
 namespace attn {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+// register split: 128 * kRegsLow + 256 * kRegsHigh must not exceed the
+// 384 * (registers per thread at launch) the CTA is given
+constexpr uint32_t kRegsLow = 72;
+constexpr uint32_t kRegsHigh = 216;
+constexpr int kMinLaunchRegs = (128 * kRegsLow + 256 * kRegsHigh + 383) / 384;
+static_assert(kMinLaunchRegs <= 168, "register split exceeds what a 384-thread CTA can be given");
 constexpr uint32_t kHalfBytes = 128 * 64 * 2;    // 128 rows x 64 bf16 (one swizzle span)
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;  // 128 x 128 bf16
 constexpr uint32_t kOffQ = 0;                    // Q_A, Q_B
@@ -52,7 +60,8 @@ enum : uint32_t {
   kBarSFull = 7,    // [2] per tile
   kBarPFull = 9,    // [2] per tile
   kBarODone = 11,   // [2] per tile
-  kNumBars = 13
+  kBarDone = 13,    // softmax threads finished with tensor memory
+  kNumBars = 14
 };
 
 // One 128-query tile of a work item.
@@ -136,33 +145,43 @@ __device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_
                 (accumulate || kk > 0) ? 1u : 0u);
 }
 
+// Row max of this thread's S row held in registers; DIAG skips keys c > r.
+template <bool DIAG>
+__device__ __forceinline__ float row_max(const uint32_t (&sv)[128], int r) {
+  if (DIAG) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 128; ++c) mx = (c > r) ? mx : fmaxf(mx, __uint_as_float(sv[c]));
+    return mx;
+  }
+  float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int e = 0; e < 64; ++e)
+    mc[e & 3] = max3f(mc[e & 3], __uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1]));
+  return fmaxf(max3f(mc[0], mc[1], mc[2]), mc[3]);
+}
+
 // Writes P = exp2(S * scale_log2 - m) as bf16 over columns [0, 64) of this
 // thread's S row and returns the row sum of the fp32 values.  Packed f32x2
 // arithmetic for the scale/shift and the sum; four independent partial sums
 // keep the dependency chains short.  DIAG zeroes keys c > r (causal diagonal).
 template <bool DIAG>
-__device__ __forceinline__ float softmax_p(uint32_t tS, float scale_log2, float m, int r) {
+__device__ __forceinline__ float softmax_p(const uint32_t (&sv)[128], uint32_t tS, float scale_log2, float m,
+                                           int r) {
   const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
   const uint64_t nm2 = f2_pack(-m, -m);
   uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
   for (int h2 = 0; h2 < 2; ++h2) {
-    uint32_t v0[32], v1[32], pk[32];
-    tmem_ld32(tS + h2 * 64, v0);
-    tmem_ld32(tS + h2 * 64 + 32, v1);
-    tmem_wait_ld_dep(v0);
-    tmem_wait_ld_dep(v1);
+    uint32_t pk[32];
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
-      const uint32_t* src = e < 16 ? v0 : v1;
-      const int ee = e & 15;
-      const uint64_t x2 =
-          f2_fma(f2_pack(__uint_as_float(src[2 * ee]), __uint_as_float(src[2 * ee + 1])), sc2, nm2);
+      const int c = h2 * 64 + 2 * e;
+      const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sc2, nm2);
       float x0, x1;
       f2_unpack(x2, x0, x1);
       float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
       if (DIAG) {
-        const int c = h2 * 64 + 2 * e;
         if (c > r) p0 = 0.f;
         if (c + 1 > r) p1 = 0.f;
       }
@@ -206,7 +225,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   if (threadIdx.x == 0) {
     for (uint32_t s = 0; s < kNumBars; ++s)
-      mbar_init(bar(s), (s == kBarPFull || s == kBarPFull + 1) ? 128u : 1u);
+      mbar_init(bar(s), (s == kBarPFull || s == kBarPFull + 1) ? 128u : (s == kBarDone ? 256u : 1u));
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -217,7 +236,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-
+  // Each warpgroup sets its register budget first and then runs only its own
+  // roles (no code is shared across the split); warp 1 frees tensor memory
+  // once the 256 softmax threads are done with it.
+  if (warp < 4) {
+  regs_dec<kRegsLow>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -305,9 +328,17 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
       }
     }
+    __syncwarp();
+    mbar_wait(bar(kBarDone), 0);
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  return;
   } else {
+    regs_inc<kRegsHigh>();
     // ------------------------------------------------------------ softmax
-    const int x = (warp - 2) >> 2;          // tile
+    const int x = (warp - 4) >> 2;          // tile
     const int qw = warp & 3;                // TMEM lane quarter of this warp
     const int r = qw * 32 + lane;           // query row == TMEM lane
     const uint32_t lane_base = (uint32_t)(qw * 32) << 16;
@@ -326,41 +357,19 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarSFull + x), u & 1));
       if (!ok) break;
       tc_fence_after();
-      // pass 1 over S: the row max (diagonal block: keys c <= r only)
+      // the S row (128 fp32) into registers, one tensor-memory round trip
       const bool diag = (j == T.i);
-      float mx;
-      if (!diag) {
-        float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int c8 = 0; c8 < 2; ++c8) {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(tS + c8 * 64, v0);
-          tmem_ld32(tS + c8 * 64 + 32, v1);
-          tmem_wait_ld_dep(v0);
-          tmem_wait_ld_dep(v1);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            mc[e & 1] = max3f(mc[e & 1], __uint_as_float(v0[2 * e]), __uint_as_float(v0[2 * e + 1]));
-            mc[2 + (e & 1)] = max3f(mc[2 + (e & 1)], __uint_as_float(v1[2 * e]), __uint_as_float(v1[2 * e + 1]));
-          }
-        }
-        mx = fmaxf(max3f(mc[0], mc[1], mc[2]), mc[3]);
-      } else {
-        mx = -INFINITY;
-#pragma unroll
-        for (int c8 = 0; c8 < 2; ++c8) {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(tS + c8 * 64, v0);
-          tmem_ld32(tS + c8 * 64 + 32, v1);
-          tmem_wait_ld_dep(v0);
-          tmem_wait_ld_dep(v1);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            mx = (c8 * 64 + e > r) ? mx : fmaxf(mx, __uint_as_float(v0[e]));
-            mx = (c8 * 64 + 32 + e > r) ? mx : fmaxf(mx, __uint_as_float(v1[e]));
-          }
-        }
-      }
+      uint32_t sv[128];
+      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(sv + 0));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(sv + 64));
+      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(sv + 96));
+      tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(sv + 0));
+      tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+      tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(sv + 64));
+      tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(sv + 96));
+      // row max (diagonal block: keys c <= r only)
+      float mx = diag ? row_max<true>(sv, r) : row_max<false>(sv, r);
       mx *= scale_log2;
       // lazy rescale: move the reference max only when it grows by > threshold
       const bool grow = (u == 0) || (mx > m_run + kRescaleThreshold);
@@ -386,7 +395,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
       m_run = m_new;
       // pass 2 over S: P = exp2(S * scale - m) in bf16, written over S[:, 0:64)
-      const float rs = diag ? softmax_p<true>(tS, scale_log2, m_run, r) : softmax_p<false>(tS, scale_log2, m_run, r);
+      const float rs = diag ? softmax_p<true>(sv, tS, scale_log2, m_run, r)
+                            : softmax_p<false>(sv, tS, scale_log2, m_run, r);
       l_run += rs;
       tmem_wait_st();
       tc_fence_before();
@@ -417,12 +427,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
       }
     }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tc_fence_before();
+    mbar_arrive(bar(kBarDone));
   }
 }
 

@@ -146,6 +146,15 @@ int ensure_device() {
     g_dev_state[dev] = PRISM_ERR_DEVICE;
     return PRISM_ERR_DEVICE;
   }
+  // The attention kernel re-splits its registers per warpgroup (setmaxnreg);
+  // the increase can only be granted if the CTA was launched with at least
+  // kMinLaunchRegs per thread, so refuse to run a build that has fewer.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, attn::sparse_attn_kernel) != cudaSuccess) return PRISM_ERR_CUDA;
+  if (fa.numRegs < attn::kMinLaunchRegs) {
+    g_dev_state[dev] = PRISM_ERR_UNSUPPORTED;
+    return PRISM_ERR_UNSUPPORTED;
+  }
   if (cudaFuncSetAttribute(attn::sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)attn::kSmemBytes) != cudaSuccess ||
       cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
