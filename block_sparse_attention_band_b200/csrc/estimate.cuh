@@ -4,15 +4,26 @@
 // each pooled band, temperatures tau_z, dual-band pooled softmax, Top-P per
 // query-block row and band, union of the two masks.
 //
-// Four kernels, all on CUDA cores (the work is HBM-bound or small):
-//   pool_kernel    (1)+(2)+(3 partials)  reads Q and K once (the HBM-bound part)
-//   tau_kernel     (3)+(4)               one CTA per (batch, Q head)
-//   scores_kernel  (5, logits)           fp32 register-tiled pooled Q K^T, both bands
-//   topp_kernel    (5 softmax)+(6)+(7)   one warp per (batch, Q head, query block)
+// One persistent kernel.  CTAs take work items from a device queue in a fixed
+// order that interleaves the two kinds of work per KV group g (the Q heads
+// that share one KV head):
 //
-// Band slicing is folded into the pooled layout: the pooling kernel writes the
-// 128 pooled dims in a permuted order [high-only | both | low-only | neither],
-// so each band is a contiguous column range: high = [0, s2), low = [s1, s3).
+//   pool(0), pool(1), score(0), pool(2), score(1), ..., pool(n-1), score(n-2), score(n-1)
+//
+// pool items (HBM-bound) stream 128x128 bf16 tiles of Q and K once and write
+// the fp32 block means (steps 1-2) and per-block energy partials (step 3);
+// the CTA that finishes the last pool item of a group also computes the
+// group's temperatures (steps 3-4) and publishes "group ready".  score items
+// (ALU-bound) wait for their group, compute both bands' pooled logits with an
+// fp32 register-tiled product (step 5) and run softmax + Top-P + union per
+// row (steps 5-7).  Scoring of group g overlaps pooling of group g+1.  An
+// item only ever waits for items earlier in the queue, which running CTAs
+// hold and which never wait, so the schedule cannot deadlock; the wait is
+// bounded all the same.
+//
+// Band slicing is folded into the pooled layout: the pool items write the 128
+// pooled dims in a permuted order [high-only | both | low-only | neither], so
+// each band is a contiguous column range: high = [0, s2), low = [s1, s3).
 #pragma once
 #include "ptx.cuh"
 
@@ -24,31 +35,89 @@ struct BandLayout {
   int d_hi, d_lo;     // band sizes
 };
 
-// ---------------------------------------------------------------------------
-// (1)+(2)+(3a): mean pool each 128x128 bf16 tile, write fp32 means in band
-// order, and per-block energy partials sum(mean^2) over hi / lo / all dims.
-// One CTA per (head row, block); 256 threads; thread t reads 16-byte vectors
-// of rows t/16, t/16+16, ... at dims 8*(t%16) .. +7 (fully coalesced).
-// ---------------------------------------------------------------------------
-constexpr int kPoolThreads = 256;
+constexpr int kEstThreads = 512;      // 16 warps, one CTA per SM
+constexpr int kHalfThreads = 256;     // a pool item is reduced by two halves, one tile each
+constexpr int kPoolTilesPerItem = 8;  // 8 x 32 KB of Q or K per pool item
+constexpr int kScoreRows = 64;        // (head, query block) rows per score item
+constexpr int kColTile = 128;         // key blocks per product column tile
+constexpr int kStageLD = kColTile + 1;
+constexpr int kGemmSmemBytes = (128 * kScoreRows + 128 * kColTile + 2 * kScoreRows * kStageLD + 2 * kScoreRows) * 4;
+constexpr int kMaxGroupHeads = 64;    // Q heads per KV head supported by the tau step
+constexpr float kLog2e = 1.4426950408889634f;
 
-__global__ void __launch_bounds__(kPoolThreads)
-pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, int q_rows,
-            int nb, float* __restrict__ pool, float* __restrict__ part, const BandLayout bl) {
-  __shared__ float red[16][128];
-  __shared__ float mean[128];
-  __shared__ float wsum[4][3];
-  const int unit = blockIdx.x;
-  const int hr = unit / nb;  // head row: q heads first, then k heads
-  const int blk = unit - hr * nb;
-  const __nv_bfloat16* src = hr < q_rows ? q + ((size_t)hr * nb + blk) * (128 * 128)
-                                         : k + ((size_t)(hr - q_rows) * nb + blk) * (128 * 128);
-  const int t = threadIdx.x;
-  const int c8 = t & 15;
-  const int rg = t >> 4;
-  uint4 v[8];
+struct EstParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  float* pool;    // [q_rows + kv_rows, nb, 128] band-ordered means
+  float* part;    // [q_rows + kv_rows, nb, 4] sum(mean^2): hi, lo, all
+  float* tau;     // [q_rows, 4]: tau_hi, tau_lo, 1/(tau_hi sqrt d_hi), 1/(tau_lo sqrt d_lo)
+  float* scores;  // [q_rows, 2, nb(nb+1)/2] scaled band logits, packed rows
+  uint32_t* mask;
+  float* dbg_tau;
+  uint32_t* sync;  // [0] queue head, [1 + g] pool items done, [1 + n_groups + g] group ready
+  int hq, hkv, G, nb, W, q_rows, n_groups;
+  int pool_items;      // per group
+  int score_items;     // per group
+  int pool_item_span;  // pool items per head row
+  int topp_warps;
+  int topp_stride;  // bytes of shared memory per Top-P warp
+  float p;
+  int explicit_tau;
+  float tau_hi, tau_lo;
+  BandLayout bl;
+};
+
+// ---------------------------------------------------------------------------
+// warp / ordering helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
-  for (int r = 0; r < 8; ++r) v[r] = ldg_nc_v4(src + (size_t)(rg + 16 * r) * 128 + c8 * 8);
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ void named_barrier(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// steps (1)-(3a): mean of one 128 x 128 bf16 tile, band-ordered fp32 write,
+// energy partials.  Thread t holds 16-byte vectors of rows t/16 + 16 r at
+// dims 8 (t % 16) .. +7: each warp reads two full 256-byte rows.
+// ---------------------------------------------------------------------------
+struct PoolHalf {
+  float red[16][128];
+  float mean[128];
+  float wsum[4][3];
+};
+struct PoolSmem {
+  PoolHalf half[2];
+  float sums[kMaxGroupHeads + 1][3];
+  int flag;
+};
+
+__device__ __forceinline__ void pool_load(uint4 (&v)[8], const __nv_bfloat16* tile) {
+  const int t = threadIdx.x & (kHalfThreads - 1);
+#pragma unroll
+  for (int r = 0; r < 8; ++r) v[r] = ldg_nc_v4(tile + (size_t)((t >> 4) + 16 * r) * 128 + (t & 15) * 8);
+}
+
+__device__ __forceinline__ void pool_reduce(const uint4 (&v)[8], const EstParams& P, int hr, int blk,
+                                            PoolHalf& sm) {
+  const int t = threadIdx.x & (kHalfThreads - 1);
+  const int bar_id = 1 + (threadIdx.x >> 8);
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -60,21 +129,21 @@ pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict
     acc[6] += bf16lo(v[r].w); acc[7] += bf16hi(v[r].w);
   }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) red[rg][c8 * 8 + e] = acc[e];
-  __syncthreads();
+  for (int e = 0; e < 8; ++e) sm.red[t >> 4][(t & 15) * 8 + e] = acc[e];
+  named_barrier(bar_id, kHalfThreads);
   if (t < 128) {
     float s = 0.f;
 #pragma unroll
-    for (int g = 0; g < 16; ++g) s += red[g][t];
-    mean[t] = s * (1.0f / 128.0f);
+    for (int g = 0; g < 16; ++g) s += sm.red[g][t];
+    sm.mean[t] = s * (1.0f / 128.0f);
   }
-  __syncthreads();
+  named_barrier(bar_id, kHalfThreads);
   if (t < 128) {
-    const float m = mean[bl.perm[t]];
-    pool[((size_t)hr * nb + blk) * 128 + t] = m;
+    const float m = sm.mean[P.bl.perm[t]];
+    P.pool[((size_t)hr * P.nb + blk) * 128 + t] = m;
     const float sq = m * m;
-    float hi = t < bl.s2 ? sq : 0.f;
-    float lo = (t >= bl.s1 && t < bl.s3) ? sq : 0.f;
+    float hi = t < P.bl.s2 ? sq : 0.f;
+    float lo = (t >= P.bl.s1 && t < P.bl.s3) ? sq : 0.f;
     float all = sq;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -83,358 +152,682 @@ pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict
       all += __shfl_xor_sync(0xffffffffu, all, o);
     }
     if ((t & 31) == 0) {
-      wsum[t >> 5][0] = hi;
-      wsum[t >> 5][1] = lo;
-      wsum[t >> 5][2] = all;
+      sm.wsum[t >> 5][0] = hi;
+      sm.wsum[t >> 5][1] = lo;
+      sm.wsum[t >> 5][2] = all;
     }
   }
-  __syncthreads();
-  if (t < 3) {
-    const float s = (wsum[0][t] + wsum[1][t]) + (wsum[2][t] + wsum[3][t]);
-    part[((size_t)hr * nb + blk) * 4 + t] = s;
-  }
+  named_barrier(bar_id, kHalfThreads);
+  if (t < 3)
+    P.part[((size_t)hr * P.nb + blk) * 4 + t] =
+        (sm.wsum[0][t] + sm.wsum[1][t]) + (sm.wsum[2][t] + sm.wsum[3][t]);
 }
 
-// ---------------------------------------------------------------------------
-// (3)+(4): RMS of each pooled band over all blocks and the temperatures.
-// One CTA (256 threads) per (batch, Q head).  Output tau[row] =
-// (tau_hi, tau_lo, 1/(tau_hi sqrt d_hi), 1/(tau_lo sqrt d_lo)).
-// ---------------------------------------------------------------------------
-constexpr int kTauThreads = 256;
-
-__global__ void __launch_bounds__(kTauThreads)
-tau_kernel(const float* __restrict__ part, int q_rows, int hq, int hkv, int nb, int d_hi, int d_lo,
-           int explicit_tau, float tau_hi_x, float tau_lo_x, float* __restrict__ tau,
-           float* __restrict__ dbg_tau) {
-  __shared__ float red[kTauThreads / 32][6];
-  const int row = blockIdx.x;  // batch * hq + h
-  const int bi = row / hq;
-  const int h = row - bi * hq;
-  const int kvrow = q_rows + bi * hkv + h / (hq / hkv);
-  float s[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  if (!explicit_tau) {
-    for (int i = threadIdx.x; i < nb; i += kTauThreads) {
-      const float* pq = part + ((size_t)row * nb + i) * 4;
-      const float* pk = part + ((size_t)kvrow * nb + i) * 4;
-      s[0] += pq[0]; s[1] += pq[1]; s[2] += pq[2];
-      s[3] += pk[0]; s[4] += pk[1]; s[5] += pk[2];
+// steps (3b)-(4): RMS of every pooled band of the group's heads over all
+// blocks and the temperatures of its Q heads (reading R1 of the pages: the
+// band's pooled Q x K energy relative to the full spectrum's).
+__device__ void group_temperatures(const EstParams& P, int g, PoolSmem& sm) {
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int bi = g / P.hkv, kv = g - bi * P.hkv;
+  for (int slot = 0; slot <= P.G; ++slot) {  // slots 0..G-1: Q heads, G: the KV head
+    const int hr = slot < P.G ? bi * P.hq + kv * P.G + slot : P.q_rows + g;
+    float s[3] = {0.f, 0.f, 0.f};
+    for (int i = t; i < P.nb; i += kEstThreads) {
+      const float* pp = P.part + ((size_t)hr * P.nb + i) * 4;
+      s[0] += pp[0];
+      s[1] += pp[1];
+      s[2] += pp[2];
     }
+#pragma unroll
+    for (int e = 0; e < 3; ++e) s[e] = warp_sum(s[e]);
+    if (lane == 0)
+#pragma unroll
+      for (int e = 0; e < 3; ++e) sm.half[0].red[warp][e] = s[e];
+    __syncthreads();
+    if (t < 3) {
+      float a = 0.f;
+      for (int w = 0; w < kEstThreads / 32; ++w) a += sm.half[0].red[w][t];
+      sm.sums[slot][t] = a;
+    }
+    __syncthreads();
   }
-#pragma unroll
-  for (int e = 0; e < 6; ++e)
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s[e] += __shfl_xor_sync(0xffffffffu, s[e], o);
-  if ((threadIdx.x & 31) == 0)
-#pragma unroll
-    for (int e = 0; e < 6; ++e) red[threadIdx.x >> 5][e] = s[e];
-  __syncthreads();
-  if (threadIdx.x == 0) {
+  if (t < P.G) {
+    const int row = bi * P.hq + kv * P.G + t;
     float th, tl;
-    if (explicit_tau) {
-      th = tau_hi_x;
-      tl = tau_lo_x;
+    if (P.explicit_tau) {
+      th = P.tau_hi;
+      tl = P.tau_lo;
     } else {
-      float S[6];
-      for (int e = 0; e < 6; ++e) {
-        float a = 0.f;
-        for (int w = 0; w < kTauThreads / 32; ++w) a += red[w][e];
-        S[e] = a;
-      }
-      const float n = (float)nb;
-      const float rq_hi = sqrtf(S[0] / (n * d_hi)), rq_lo = sqrtf(S[1] / (n * d_lo));
-      const float rq_f = sqrtf(S[2] / (n * 128.f));
-      const float rk_hi = sqrtf(S[3] / (n * d_hi)), rk_lo = sqrtf(S[4] / (n * d_lo));
-      const float rk_f = sqrtf(S[5] / (n * 128.f));
+      const float n = (float)P.nb;
+      const float* sq = sm.sums[t];
+      const float* sk = sm.sums[P.G];
+      const float rq_hi = sqrtf(sq[0] / (n * P.bl.d_hi)), rq_lo = sqrtf(sq[1] / (n * P.bl.d_lo));
+      const float rq_f = sqrtf(sq[2] / (n * 128.f));
+      const float rk_hi = sqrtf(sk[0] / (n * P.bl.d_hi)), rk_lo = sqrtf(sk[1] / (n * P.bl.d_lo));
+      const float rk_f = sqrtf(sk[2] / (n * 128.f));
       const float den = rq_f * rk_f;
       const float nh = rq_hi * rk_hi, nl = rq_lo * rk_lo;
       th = (den > 0.f && nh > 0.f) ? nh / den : 1.f;
       tl = (den > 0.f && nl > 0.f) ? nl / den : 1.f;
     }
-    tau[row * 4 + 0] = th;
-    tau[row * 4 + 1] = tl;
-    tau[row * 4 + 2] = 1.0f / (th * sqrtf((float)d_hi));
-    tau[row * 4 + 3] = 1.0f / (tl * sqrtf((float)d_lo));
-    if (dbg_tau) {
-      dbg_tau[row * 2 + 0] = th;
-      dbg_tau[row * 2 + 1] = tl;
+    P.tau[row * 4 + 0] = th;
+    P.tau[row * 4 + 1] = tl;
+    P.tau[row * 4 + 2] = 1.0f / (th * sqrtf((float)P.bl.d_hi));
+    P.tau[row * 4 + 3] = 1.0f / (tl * sqrtf((float)P.bl.d_lo));
+    if (P.dbg_tau) {
+      P.dbg_tau[row * 2 + 0] = th;
+      P.dbg_tau[row * 2 + 1] = tl;
+    }
+  }
+}
+
+// One pool item: kPoolTilesPerItem consecutive blocks of one head row of the
+// group (its Q heads, then its KV head), the next tile's loads in flight
+// while the current one is reduced.
+__device__ void pool_item(const EstParams& P, int g, int y, PoolSmem& sm) {
+  const int slot = y / P.pool_item_span;
+  const int blk0 = (y - slot * P.pool_item_span) * kPoolTilesPerItem;
+  const int blk1 = min(blk0 + kPoolTilesPerItem, P.nb);
+  const int bi = g / P.hkv, kv = g - bi * P.hkv;
+  int hr;
+  const __nv_bfloat16* base;
+  if (slot < P.G) {
+    hr = bi * P.hq + kv * P.G + slot;
+    base = P.q + (size_t)hr * P.nb * (128 * 128);
+  } else {
+    hr = P.q_rows + g;
+    base = P.k + (size_t)g * P.nb * (128 * 128);
+  }
+  // half h reduces tiles blk0 + h, blk0 + h + 2, ...; the next tile of the
+  // half is loaded while the current one is reduced
+  const int h = threadIdx.x >> 8;
+  PoolHalf& hs = sm.half[h];
+  uint4 va[8], vb[8];
+  if (blk0 + h < blk1) pool_load(va, base + (size_t)(blk0 + h) * (128 * 128));
+  for (int b = blk0 + h; b < blk1; b += 4) {
+    if (b + 2 < blk1) pool_load(vb, base + (size_t)(b + 2) * (128 * 128));
+    pool_reduce(va, P, hr, b, hs);
+    if (b + 2 < blk1) {
+      if (b + 4 < blk1) pool_load(va, base + (size_t)(b + 4) * (128 * 128));
+      pool_reduce(vb, P, hr, b + 2, hs);
+    }
+  }
+  // publish: count the item; the CTA that completes the group computes tau
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const uint32_t done = atomicAdd(&P.sync[1 + g], 1u);
+    sm.flag = (done == (uint32_t)P.pool_items - 1u);
+    if (sm.flag) __threadfence();
+  }
+  __syncthreads();
+  if (sm.flag) {
+    group_temperatures(P, g, sm);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      st_release_gpu(&P.sync[1 + P.n_groups + g], 1u);
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// (5) band logits: L_z[i][j] = Qbar_z[i] . Kbar_z[j] * scale_z for j <= i.
-// 64 x 64 output tiles over the lower triangle of each (batch, Q head);
-// 256 threads, each a 4 x 4 register tile; the dims are accumulated segment
-// by segment so the two bands share the overlapping dims' products.
-// Output: packed lower-triangular rows, [row][band][i(i+1)/2 + j].
+// step (6): exact Top-P of one band row
 // ---------------------------------------------------------------------------
-constexpr int kScoreTile = 64;
-constexpr int kScoreThreads = 256;
-constexpr int kScoreSmemBytes = 2 * 128 * kScoreTile * 4;
+// Shared-memory scratch of one Top-P warp.
+struct ToppScratch {
+  uint32_t* d;            // [n] logits, then the rank keys d_j (below)
+  float* L2;              // [n] the second band's logits, loaded with the first
+  uint16_t* cand;         // [n] members of the crossing bin
+  unsigned long long* h;  // [256] bin masses
+  uint32_t* kb;           // [W] blocks of bins before the crossing bin
+};
 
-__global__ void __launch_bounds__(kScoreThreads)
-scores_kernel(const float* __restrict__ pool, int q_rows, int hq, int hkv, int nb,
-              const float* __restrict__ tau, int s1, int s2, int s3, float* __restrict__ scores) {
-  extern __shared__ __align__(16) float score_smem[];
-  float(*qT)[kScoreTile] = reinterpret_cast<float(*)[kScoreTile]>(score_smem);
-  float(*kT)[kScoreTile] = reinterpret_cast<float(*)[kScoreTile]>(score_smem + 128 * kScoreTile);
-  const int row = blockIdx.y;  // batch * hq + h
-  const int bi = row / hq;
-  const int h = row - bi * hq;
-  const int kvrow = q_rows + bi * hkv + h / (hq / hkv);
-  // lower-triangle tile index -> (ti, tj), tj <= ti
-  const int tid = blockIdx.x;
-  int ti = (int)((sqrtf(8.f * tid + 1.f) - 1.f) * 0.5f);
-  while ((ti + 1) * (ti + 2) / 2 <= tid) ++ti;
-  while (ti * (ti + 1) / 2 > tid) --ti;
-  const int tj = tid - ti * (ti + 1) / 2;
-  const int i0 = ti * kScoreTile, j0 = tj * kScoreTile;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float* qsrc = pool + (size_t)row * nb * 128;
-  const float* ksrc = pool + (size_t)kvrow * nb * 128;
-  // transposed staging: lane -> row, warp -> 4-dim chunks
+constexpr int kTopPBins = 256;
+constexpr float kFix = 2147483648.0f;  // 2^31: e_j in [0, 2) -> 32-bit fixed point
+
+// e_j (in (0, 2)) -> rank key d_j = 0x40000000 - bits(e_j): an exact,
+// order-reversing map (smaller key = larger e_j; equal keys = equal e_j).
+__device__ __forceinline__ uint32_t rank_key(float e) { return 0x40000000u - __float_as_uint(e); }
+__device__ __forceinline__ float key_value(uint32_t d) { return __uint_as_float(0x40000000u - d); }
+__device__ __forceinline__ uint32_t fixmass(float e) { return __float2uint_rn(e * kFix); }
+
+// Warp-wide inclusive scan of 64-bit values.
+__device__ __forceinline__ unsigned long long warp_scan_u64(unsigned long long v, int lane) {
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const int r = rr * 32 + lane;
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      const int c = warp + 8 * cc;
-      float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-      if (i0 + r < nb) a = *reinterpret_cast<const float4*>(qsrc + (size_t)(i0 + r) * 128 + 4 * c);
-      if (j0 + r < nb) b = *reinterpret_cast<const float4*>(ksrc + (size_t)(j0 + r) * 128 + 4 * c);
-      qT[4 * c + 0][r] = a.x; qT[4 * c + 1][r] = a.y; qT[4 * c + 2][r] = a.z; qT[4 * c + 3][r] = a.w;
-      kT[4 * c + 0][r] = b.x; kT[4 * c + 1][r] = b.y; kT[4 * c + 2][r] = b.z; kT[4 * c + 3][r] = b.w;
-    }
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
   }
-  __syncthreads();
-  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-  float a[4][4], b[4][4];
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-#pragma unroll
-    for (int w = 0; w < 4; ++w) a[u][w] = b[u][w] = 0.f;
-  auto fma_range = [&](float(&acc)[4][4], int d0, int d1) {
-#pragma unroll 4
-    for (int d = d0; d < d1; ++d) {
-      const float4 qa = *reinterpret_cast<const float4*>(&qT[d][4 * ty]);
-      const float4 kb = *reinterpret_cast<const float4*>(&kT[d][4 * tx]);
-      const float qv[4] = {qa.x, qa.y, qa.z, qa.w};
-      const float kv[4] = {kb.x, kb.y, kb.z, kb.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(qv[u], kv[w], acc[u][w]);
-    }
-  };
-  fma_range(a, 0, s1);   // high-only dims
-  fma_range(b, s1, s2);  // dims in both bands
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-#pragma unroll
-    for (int w = 0; w < 4; ++w) a[u][w] += b[u][w];  // a = high band
-  fma_range(b, s2, s3);  // b = low band
-  const float sc_hi = tau[row * 4 + 2], sc_lo = tau[row * 4 + 3];
-  __syncthreads();
-  // stage the two 64 x 64 tiles through shared memory for coalesced row writes
-  float* stage = &qT[0][0];  // 2 * 64 * 65 floats fit in qT + kT (16384 floats)
-  constexpr int LD = kScoreTile + 1;
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      stage[(4 * ty + u) * LD + 4 * tx + w] = a[u][w] * sc_hi;
-      stage[kScoreTile * LD + (4 * ty + u) * LD + 4 * tx + w] = b[u][w] * sc_lo;
-    }
-  __syncthreads();
-  const size_t tri = (size_t)nb * (nb + 1) / 2;
-  float* out_hi = scores + (size_t)row * 2 * tri;
-  float* out_lo = out_hi + tri;
-  for (int r = warp; r < kScoreTile; r += kScoreThreads / 32) {
-    const int i = i0 + r;
-    if (i >= nb) break;
-    const size_t base = (size_t)i * (i + 1) / 2;
-    for (int c = lane; c < kScoreTile; c += 32) {
-      const int j = j0 + c;
-      if (j <= i) {
-        out_hi[base + j] = stage[r * LD + c];
-        out_lo[base + j] = stage[kScoreTile * LD + r * LD + c];
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// (5 softmax)+(6)+(7): one warp per (batch, Q head, query block i).
-// For each band: e_j = exp(L_j - max), Z = sum e_j; rank j by (-e_j, j);
-// the crossing block c is the one with mass(ahead of c) < p Z <= mass(ahead)
-// + e_c; keep every block ranked at or ahead of c.  The crossing block is
-// found by a warp quickselect over candidate lists in shared memory (median
-// of three pivots, stable ballot compaction), so the cost is O(n) per row.
-// All sums run in a fixed order: the result is deterministic.
-// ---------------------------------------------------------------------------
-constexpr int kTopPWarps = 4;
-
-__device__ __forceinline__ bool ranks_before(const float* e, int a, int b) {
-  const float ea = e[a], eb = e[b];
-  return ea > eb || (ea == eb && a < b);
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ int warp_sum_i(int v) {
+
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
-// Returns the crossing block index, or -1 when every block is kept.
-__device__ int topp_crossing(const float* e, uint16_t* bufA, uint16_t* bufB, int n, float target,
-                             int lane) {
-  const uint16_t* cur = nullptr;  // nullptr: candidates are 0..cnt-1
-  uint16_t* nxt = bufA;
-  int cnt = n;
-  float base = 0.f;  // mass of blocks known to rank ahead of every candidate
-#define CAND(x) (cur ? (int)cur[(x)] : (x))
-  while (cnt > 32) {
-    int p1 = CAND(cnt >> 2), p2 = CAND(cnt >> 1), p3 = CAND((3 * cnt) >> 2);
-    // median of three by rank
-    if (ranks_before(e, p2, p1)) { int t = p1; p1 = p2; p2 = t; }
-    if (ranks_before(e, p3, p2)) { int t = p2; p2 = p3; p3 = t; }
-    if (ranks_before(e, p2, p1)) { int t = p1; p1 = p2; p2 = t; }
-    const int piv = p2;
-    const float ep = e[piv];
-    float s = 0.f;
-    int c = 0;
-    for (int x = lane; x < cnt; x += 32) {
-      const int j = CAND(x);
-      if (ranks_before(e, j, piv)) { s += e[j]; ++c; }
-    }
-    s = warp_sum(s);
-    c = warp_sum_i(c);
-    bool take_ahead;
-    if (base + s >= target) {
-      take_ahead = true;
-    } else if (base + s + ep >= target) {
-      return piv;
-    } else {
-      base = base + s + ep;
-      take_ahead = false;
-    }
-    int out = 0;
-    for (int x0 = 0; x0 < cnt; x0 += 32) {
-      const int x = x0 + lane;
-      bool sel = false;
-      int j = 0;
-      if (x < cnt) {
-        j = CAND(x);
-        sel = take_ahead ? ranks_before(e, j, piv) : ranks_before(e, piv, j);
-      }
-      const unsigned m = __ballot_sync(0xffffffffu, sel);
-      if (sel) nxt[out + __popc(m & ((1u << lane) - 1u))] = (uint16_t)j;
-      out += __popc(m);
-    }
-    __syncwarp();
-    cur = nxt;
-    nxt = (nxt == bufA) ? bufB : bufA;
-    cnt = take_ahead ? c : cnt - c - 1;
-  }
-  // at most 32 candidates left: each lane holds one and sums the mass ahead of it
+// Exact crossing among `cnt` members (<= 32) listed in S.cand, all ranked
+// behind mass `base`: returns the member c with ahead(c) < target <=
+// ahead(c) + e_c, or -1 if none reaches the target.
+__device__ __forceinline__ int topp_exact32(const ToppScratch& S, int cnt, unsigned long long base,
+                                            unsigned long long target, int lane) {
   int j = -1;
-  float ej = 0.f;
+  uint32_t dj = 0xffffffffu;
+  uint32_t mj = 0u;
   if (lane < cnt) {
-    j = CAND(lane);
-    ej = e[j];
+    j = S.cand[lane];
+    dj = S.d[j];
+    mj = fixmass(key_value(dj));
   }
-#undef CAND
-  float ahead = 0.f;
+  unsigned long long ahead = 0ull;
   int rank = 0;
-  for (int l = 0; l < cnt; ++l) {
+#pragma unroll
+  for (int l = 0; l < 32; ++l) {
     const int jl = __shfl_sync(0xffffffffu, j, l);
-    const float el = __shfl_sync(0xffffffffu, ej, l);
-    if (lane < cnt && (el > ej || (el == ej && jl < j))) {
-      ahead += el;
+    const uint32_t dl = __shfl_sync(0xffffffffu, dj, l);
+    const uint32_t ml = __shfl_sync(0xffffffffu, mj, l);
+    if (l < cnt && lane < cnt && (dl < dj || (dl == dj && jl < j))) {
+      ahead += ml;
       ++rank;
     }
   }
-  const bool crosses = lane < cnt && (base + ahead + ej >= target);
-  // first crossing in rank order (ranks are distinct integers)
+  const bool crosses = lane < cnt && base + ahead + mj >= target;
   int best = crosses ? rank : 0x7fffffff;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, o));
-  if (best != 0x7fffffff) {
-    const unsigned m = __ballot_sync(0xffffffffu, crosses && rank == best);
-    return __shfl_sync(0xffffffffu, j, __ffs(m) - 1);
-  }
-  // no candidate reaches the target (rounding with p close to 1): keep all of
-  // them -- the lowest-ranked candidate becomes the cut, or everything if none
-  if (cnt == 0) return -1;
-  int worst = lane < cnt ? rank : -1;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) worst = max(worst, __shfl_xor_sync(0xffffffffu, worst, o));
-  const unsigned m = __ballot_sync(0xffffffffu, lane < cnt && rank == worst);
-  return __shfl_sync(0xffffffffu, j, __ffs(m) - 1);
+  if (best == 0x7fffffff) return -1;
+  const unsigned mk = __ballot_sync(0xffffffffu, crosses && rank == best);
+  return __shfl_sync(0xffffffffu, j, __ffs(mk) - 1);
 }
 
-__global__ void __launch_bounds__(kTopPWarps * 32)
-topp_kernel(const float* __restrict__ scores, int rows_total /* b*hq*nb */, int nb, float p,
-            uint32_t* __restrict__ mask) {
-  extern __shared__ __align__(16) unsigned char topp_smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int W = (nb + 31) >> 5;
-  const int nbp = (nb + 3) & ~3;
-  const size_t per_warp = (size_t)nbp * 4 + (size_t)nbp * 2 * 2 + (size_t)W * 4;
-  unsigned char* base = topp_smem + warp * ((per_warp + 15) & ~(size_t)15);
-  float* e = reinterpret_cast<float*>(base);
-  uint16_t* bufA = reinterpret_cast<uint16_t*>(base + (size_t)nbp * 4);
-  uint16_t* bufB = bufA + nbp;
-  uint32_t* bits = reinterpret_cast<uint32_t*>(base + (size_t)nbp * 8);
-  const int gr = blockIdx.x * (blockDim.x >> 5) + warp;  // (batch*hq) * nb + i
-  if (gr >= rows_total) return;
-  const int row = gr / nb;
-  const int i = gr - row * nb;
-  const int n = i + 1;
-  const size_t tri = (size_t)nb * (nb + 1) / 2;
-  for (int w = lane; w < W; w += 32) bits[w] = 0u;
+// 64-bit bin mass kept as two 32-bit words: the low word's atomic add returns
+// the old value, and an add that wraps it carries one into the high word, so
+// the final sum is exact and independent of the order of the adds.
+__device__ __forceinline__ void bin_add(uint32_t* lo, uint32_t* hi, int b, uint32_t x) {
+  const uint32_t old = atomicAdd(&lo[b], x);
+  if (old > ~x) atomicAdd(&hi[b], 1u);
+}
+
+// Softmax (step 5) + Top-P (step 6) of one band row of n scaled logits held
+// in shared memory; ORs the kept blocks into bits[].
+//
+// e_j = 2^((L_j - max) log2 e); blocks ranked by (-e_j, j) == (d_j, j) with
+// the exact order-reversing key d_j.  Radix selection on the keys: bins of 16
+// per octave of e (bin = d >> 19, the last one collecting everything below
+// 2^-14) hold their mass exactly (e_j in 2^-31 fixed point, 64-bit exact
+// sums), so one scan gives Z, the crossing bin and the mass ranked before it
+// as exact integers.  Blocks of earlier bins are kept, of later bins dropped;
+// the crossing bin's members are ranked exactly (pairwise when <= 32, else by
+// refining on the lower key bits the same way).  A block is kept iff the
+// mass ranked strictly ahead of it is < p Z.
+__device__ void topp_band_row(const float* Lsm, int n, int W, float p, const ToppScratch& S, uint32_t* bits,
+                              int lane) {
+  const unsigned lt = (1u << lane) - 1u;
+  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 4
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    if (j < n) mx[(j0 >> 5) & 3] = fmaxf(mx[(j0 >> 5) & 3], Lsm[j]);
+  }
+  const int nw = (n + 31) >> 5;
+  if (p >= 1.0f) {  // every causal block is kept
+    for (int w = lane; w < nw; w += 32) {
+      const int lo = w * 32;
+      bits[w] |= lo + 32 <= n ? 0xffffffffu : ((1u << (n - lo)) - 1u);
+    }
+    __syncwarp();
+    return;
+  }
+  const float m = warp_max(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]))) * kLog2e;
+  uint32_t* hlo = reinterpret_cast<uint32_t*>(S.h);
+  uint32_t* hhi = hlo + kTopPBins;
+  for (int b = lane; b < kTopPBins; b += 32) {
+    hlo[b] = 0u;
+    hhi[b] = 0u;
+  }
   __syncwarp();
-  for (int band = 0; band < 2; ++band) {
-    const float* src = scores + ((size_t)row * 2 + band) * tri + (size_t)i * (i + 1) / 2;
-    float m = -INFINITY;
-    for (int j = lane; j < n; j += 32) {
-      const float x = src[j];
-      e[j] = x;
-      m = fmaxf(m, x);
+  // e_j, keys, exact bin masses
+#pragma unroll 4
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    if (j < n) {
+      const float e = fast_exp2(fmaf(Lsm[j], kLog2e, -m));
+      const uint32_t d = rank_key(e);
+      S.d[j] = d;
+      bin_add(hlo, hhi, (int)min(d >> 19, (uint32_t)(kTopPBins - 1)), fixmass(e));
     }
-    m = warp_max(m);
-    float z = 0.f;
-    for (int j = lane; j < n; j += 32) {
-      const float x = expf(e[j] - m);
-      e[j] = x;
-      z += x;
+  }
+  __syncwarp();
+  unsigned long long hv[8], tot = 0ull;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    hv[u] = ((unsigned long long)hhi[lane * 8 + u] << 32) | hlo[lane * 8 + u];
+    tot += hv[u];
+  }
+  unsigned long long incl = warp_scan_u64(tot, lane);
+  const unsigned long long Z = __shfl_sync(0xffffffffu, incl, 31);
+  const unsigned long long target = (unsigned long long)((double)p * (double)Z);
+  // crossing bin: the first with (mass before it + its mass) >= target
+  int xb;
+  unsigned long long base;
+  {
+    unsigned long long run = incl - tot;
+    int bin = -1;
+    unsigned long long bb = 0ull;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (bin < 0 && run + hv[u] >= target && hv[u] > 0ull) {
+        bin = lane * 8 + u;
+        bb = run;
+      }
+      run += hv[u];
     }
-    z = warp_sum(z);
-    __syncwarp();
-    int cross = -1;
-    if (p < 1.0f) cross = topp_crossing(e, bufA, bufB, n, p * z, lane);
-    __syncwarp();
+    const unsigned found = __ballot_sync(0xffffffffu, bin >= 0);
+    const int sl = found ? __ffs(found) - 1 : 31;
+    xb = found ? __shfl_sync(0xffffffffu, bin, sl) : kTopPBins - 1;
+    base = found ? __shfl_sync(0xffffffffu, bb, sl) : Z;
+  }
+  // one pass: keep the earlier bins, list the crossing bin's members
+  int cnt = 0;
+#pragma unroll 2
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    bool before = false, in = false;
+    if (j < n) {
+      const int b = (int)min(S.d[j] >> 19, (uint32_t)(kTopPBins - 1));
+      before = b < xb;
+      in = b == xb;
+    }
+    const unsigned mb = __ballot_sync(0xffffffffu, before), mi = __ballot_sync(0xffffffffu, in);
+    if (in) S.cand[cnt + __popc(mi & lt)] = (uint16_t)j;
+    cnt += __popc(mi);
+    if (lane == 0) bits[j0 >> 5] |= mb;
+  }
+  __syncwarp();
+  // rank the crossing bin's members
+  int cross = -1;
+  bool refined = false;
+  if (cnt <= 32) {
+    cross = topp_exact32(S, cnt, base, target, lane);
+  } else {
+    // refine on lower key bits, 8-bit digits: a regular bin spans 2^19 keys
+    // (digits at shifts 11, 3, 0), the catch-all bin up to 2^30 (22, 14, 6, 0)
+    refined = true;
+    uint32_t lo_key = (uint32_t)xb << 19;
+    const bool wide = xb == kTopPBins - 1;
+    for (int level = 0;; ++level) {
+      const int sh = wide ? (level == 0 ? 22 : level == 1 ? 14 : level == 2 ? 6 : 0)
+                          : (level == 0 ? 11 : level == 1 ? 3 : 0);
+      for (int b = lane; b < kTopPBins; b += 32) {
+        hlo[b] = 0u;
+        hhi[b] = 0u;
+      }
+      __syncwarp();
+      for (int x0 = 0; x0 < cnt; x0 += 32) {
+        const int x = x0 + lane;
+        if (x < cnt) {
+          const uint32_t d = S.d[S.cand[x]];
+          bin_add(hlo, hhi, (int)min((d - lo_key) >> sh, (uint32_t)(kTopPBins - 1)), fixmass(key_value(d)));
+        }
+      }
+      __syncwarp();
+      unsigned long long h2[8], t2 = 0ull;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        h2[u] = ((unsigned long long)hhi[lane * 8 + u] << 32) | hlo[lane * 8 + u];
+        t2 += h2[u];
+      }
+      const unsigned long long inc2 = warp_scan_u64(t2, lane);
+      unsigned long long run = inc2 - t2;
+      int bin2 = -1;
+      unsigned long long bb = 0ull;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (bin2 < 0 && base + run + h2[u] >= target && h2[u] > 0ull) {
+          bin2 = lane * 8 + u;
+          bb = base + run;
+        }
+        run += h2[u];
+      }
+      const unsigned f2 = __ballot_sync(0xffffffffu, bin2 >= 0);
+      if (f2 == 0u) {
+        // (exact sums make this unreachable) the members' mass stays below
+        // the target: all of them are kept -- the cut is the last member
+        uint32_t bd = 0u;
+        int bj = -1;
+        for (int x = lane; x < cnt; x += 32) {
+          const int jj = S.cand[x];
+          const uint32_t dd = S.d[jj];
+          if (bj < 0 || dd > bd || (dd == bd && jj > bj)) {
+            bd = dd;
+            bj = jj;
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const uint32_t od = __shfl_xor_sync(0xffffffffu, bd, o);
+          const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+          if (bj < 0 || (oj >= 0 && (od > bd || (od == bd && oj > bj)))) {
+            bd = od;
+            bj = oj;
+          }
+        }
+        cross = bj;
+        break;
+      }
+      const int sl = __ffs(f2) - 1;
+      const int xb2 = __shfl_sync(0xffffffffu, bin2, sl);
+      base = __shfl_sync(0xffffffffu, bb, sl);
+      const uint32_t blo = lo_key + ((uint32_t)xb2 << sh);
+      const uint32_t bhi = sh == 0 ? blo : blo + ((1u << sh) - 1u);
+      int c2 = 0;
+      for (int x0 = 0; x0 < cnt; x0 += 32) {
+        const int x = x0 + lane;
+        int jj = 0;
+        bool in = false;
+        if (x < cnt) {
+          jj = S.cand[x];
+          const uint32_t d = S.d[jj];
+          in = d >= blo && d <= bhi;
+        }
+        const unsigned mk = __ballot_sync(0xffffffffu, in);
+        __syncwarp();
+        if (in) S.cand[c2 + __popc(mk & lt)] = (uint16_t)jj;
+        c2 += __popc(mk);
+      }
+      __syncwarp();
+      cnt = c2;
+      lo_key = blo;
+      if (cnt <= 32) {
+        cross = topp_exact32(S, cnt, base, target, lane);
+        break;
+      }
+      if (sh == 0) {
+        // equal keys: the first member (by index) whose cumulative mass
+        // reaches the target
+        const unsigned long long me = (unsigned long long)fixmass(key_value(blo));
+        unsigned long long acc = base;
+        for (int x0 = 0; x0 < cnt && cross < 0; x0 += 32) {
+          const int x = x0 + lane;
+          const bool ok = x < cnt;
+          const unsigned mk = __ballot_sync(0xffffffffu, ok);
+          const int pos = __popc(mk & lt);
+          const bool hit = ok && acc + me * (unsigned long long)(pos + 1) >= target;
+          const unsigned hm = __ballot_sync(0xffffffffu, hit);
+          if (hm) cross = __shfl_sync(0xffffffffu, ok ? (int)S.cand[x] : 0, __ffs(hm) - 1);
+          acc += me * (unsigned long long)__popc(mk);
+        }
+        break;
+      }
+    }
+  }
+  __syncwarp();
+  if (!refined) {
+    // the crossing bin's members ranked at or ahead of the crossing
+    const uint32_t dc = cross >= 0 ? S.d[cross] : 0u;
+    if (lane < cnt) {
+      const int j = S.cand[lane];
+      const uint32_t d = S.d[j];
+      if (cross < 0 || d < dc || (d == dc && j <= cross)) atomicOr(&bits[j >> 5], 1u << (j & 31));
+    }
+  } else {
+    // general case: every block ranked at or ahead of the crossing
+    const uint32_t dc = cross >= 0 ? S.d[cross] : 0xffffffffu;
     for (int j0 = 0; j0 < n; j0 += 32) {
       const int j = j0 + lane;
       bool keep = false;
-      if (j < n) keep = (cross < 0) || j == cross || ranks_before(e, j, cross);
+      if (j < n) {
+        const uint32_t d = S.d[j];
+        keep = cross < 0 || d < dc || (d == dc && j <= cross);
+      }
       const unsigned word = __ballot_sync(0xffffffffu, keep);
       if (lane == 0) bits[j0 >> 5] |= word;
     }
-    __syncwarp();
   }
-  uint32_t* dst = mask + (size_t)gr * W;
-  for (int w = lane; w < W; w += 32) dst[w] = bits[w];
+  __syncwarp();
+}
+
+// ---------------------------------------------------------------------------
+// score item: kScoreRows (head, query block) rows of one group, enumerated
+// from the last query block down and over the group's heads; the rows share
+// the group's pooled K.  Step (5) logits for j <= i with an fp32 4x4
+// register tile per thread (the dims accumulate segment by segment so the
+// two bands share the products of their common dims), then steps (5)-(7)
+// per row.
+// ---------------------------------------------------------------------------
+__device__ void score_item(const EstParams& P, int g, int y, unsigned char* smem) {
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int bi = g / P.hkv, kv = g - bi * P.hkv;
+  const int rows_total = P.G * P.nb;
+  const int idx0 = y * kScoreRows;
+  float* qT = reinterpret_cast<float*>(smem);      // [128 dims][64 rows]
+  float* kT = qT + 128 * kScoreRows;               // [128 dims][128 cols]
+  float* stage = kT + 128 * kColTile;              // [2][64][129]
+  float* scl = stage + 2 * kScoreRows * kStageLD;  // [64][2]
+  const size_t tri = (size_t)P.nb * (P.nb + 1) / 2;
+  const float* kbase = P.pool + (size_t)(P.q_rows + g) * P.nb * 128;
+  const int max_i = P.nb - 1 - idx0 / P.G;
+
+  // rows of this item: r -> (head h, block i); false past the group's end
+  auto row_of = [&](int r, int& bh, int& i) -> bool {
+    const int idx = idx0 + r;
+    if (idx >= rows_total) return false;
+    bh = bi * P.hq + kv * P.G + idx % P.G;
+    i = P.nb - 1 - idx / P.G;
+    return true;
+  };
+
+  if (t < kScoreRows) {
+    int bh, i;
+    if (row_of(t, bh, i)) {
+      scl[2 * t] = P.tau[bh * 4 + 2];
+      scl[2 * t + 1] = P.tau[bh * 4 + 3];
+    } else {
+      scl[2 * t] = scl[2 * t + 1] = 0.f;
+    }
+  }
+  // Qbar rows, transposed: lane -> row, warp -> 4-dim chunks
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    const int r = rr * 32 + lane;
+    int bh = 0, i = 0;
+    const bool ok = row_of(r, bh, i);
+    const float* src = P.pool + ((size_t)bh * P.nb + i) * 128;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const int c = warp + 16 * cc;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (ok) a = *reinterpret_cast<const float4*>(src + 4 * c);
+      qT[(4 * c + 0) * kScoreRows + r] = a.x;
+      qT[(4 * c + 1) * kScoreRows + r] = a.y;
+      qT[(4 * c + 2) * kScoreRows + r] = a.z;
+      qT[(4 * c + 3) * kScoreRows + r] = a.w;
+    }
+  }
+  const int ty = t >> 5, tx = t & 31;  // 16 x 32 threads, 4 x 4 outputs each
+  for (int j0 = 0; j0 <= max_i; j0 += kColTile) {
+    __syncthreads();  // the previous tile's kT and stage reads are done
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+      const int r = rr * 32 + lane;
+      const bool ok = j0 + r <= max_i;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = warp + 16 * cc;
+        float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (ok) b = *reinterpret_cast<const float4*>(kbase + (size_t)(j0 + r) * 128 + 4 * c);
+        kT[(4 * c + 0) * kColTile + r] = b.x;
+        kT[(4 * c + 1) * kColTile + r] = b.y;
+        kT[(4 * c + 2) * kColTile + r] = b.z;
+        kT[(4 * c + 3) * kColTile + r] = b.w;
+      }
+    }
+    __syncthreads();
+    float a[4][4], b[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) a[u][w] = b[u][w] = 0.f;
+    auto fma_range = [&](float(&acc)[4][4], int d0, int d1) {
+#pragma unroll 4
+      for (int d = d0; d < d1; ++d) {
+        const float4 qa = *reinterpret_cast<const float4*>(&qT[d * kScoreRows + 4 * ty]);
+        const float4 kb = *reinterpret_cast<const float4*>(&kT[d * kColTile + 4 * tx]);
+        const float qv[4] = {qa.x, qa.y, qa.z, qa.w};
+        const float kvv[4] = {kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(qv[u], kvv[w], acc[u][w]);
+      }
+    };
+    fma_range(a, 0, P.bl.s1);        // high-only dims
+    fma_range(b, P.bl.s1, P.bl.s2);  // dims of both bands
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) a[u][w] += b[u][w];  // a = high band
+    fma_range(b, P.bl.s2, P.bl.s3);  // b = low band
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int row = 4 * ty + u;
+      const float sh = scl[2 * row], sl = scl[2 * row + 1];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        stage[row * kStageLD + 4 * tx + w] = a[u][w] * sh;
+        stage[kScoreRows * kStageLD + row * kStageLD + 4 * tx + w] = b[u][w] * sl;
+      }
+    }
+    __syncthreads();
+    for (int r = warp; r < kScoreRows; r += kEstThreads / 32) {
+      int bh, i;
+      if (!row_of(r, bh, i)) continue;
+      float* out_hi = P.scores + (size_t)bh * 2 * tri + (size_t)i * (i + 1) / 2;
+      float* out_lo = out_hi + tri;
+      for (int c = lane; c < kColTile; c += 32) {
+        const int jj = j0 + c;
+        if (jj <= i) {
+          out_hi[jj] = stage[r * kStageLD + c];
+          out_lo[jj] = stage[kScoreRows * kStageLD + r * kStageLD + c];
+        }
+      }
+    }
+  }
+  __syncthreads();  // this CTA's score rows are visible to all its threads
+
+  // steps (5)-(7): one warp per row, both bands, union, whole mask row
+  if (warp < P.topp_warps) {
+    unsigned char* wb = smem + (size_t)warp * P.topp_stride;
+    const int nbp = (P.nb + 7) & ~7;
+    ToppScratch S;
+    S.d = reinterpret_cast<uint32_t*>(wb);
+    S.L2 = reinterpret_cast<float*>(wb + (size_t)nbp * 4);
+    S.cand = reinterpret_cast<uint16_t*>(wb + (size_t)nbp * 8);
+    S.h = reinterpret_cast<unsigned long long*>(wb + (size_t)nbp * 10);
+    S.kb = reinterpret_cast<uint32_t*>(wb + (size_t)nbp * 10 + kTopPBins * 8);
+    uint32_t* bits = S.kb + P.W;
+    for (int r = warp; r < kScoreRows; r += P.topp_warps) {
+      int bh, i;
+      if (!row_of(r, bh, i)) continue;
+      for (int w = lane; w < P.W; w += 32) bits[w] = 0u;
+      __syncwarp();
+      // both bands' rows -> shared memory in one round trip (32 loads in flight per lane)
+      const float* row_hi = P.scores + (size_t)bh * 2 * tri + (size_t)i * (i + 1) / 2;
+      const float* row_lo = row_hi + tri;
+      const int n = i + 1;
+      float* Lhi = reinterpret_cast<float*>(S.d);
+      for (int j0 = 0; j0 < n; j0 += 512) {
+        float xh[16], xl[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int j = j0 + u * 32 + lane;
+          xh[u] = j < n ? row_hi[j] : 0.f;
+          xl[u] = j < n ? row_lo[j] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int j = j0 + u * 32 + lane;
+          if (j < n) {
+            Lhi[j] = xh[u];
+            S.L2[j] = xl[u];
+          }
+        }
+      }
+      __syncwarp();
+      topp_band_row(Lhi, n, P.W, P.p, S, bits, lane);
+      topp_band_row(S.L2, n, P.W, P.p, S, bits, lane);
+      uint32_t* dst = P.mask + ((size_t)bh * P.nb + i) * P.W;
+      for (int w = lane; w < P.W; w += 32) dst[w] = bits[w];
+      __syncwarp();
+    }
+  }
+  __syncthreads();  // shared memory is reused by the next item
+}
+
+// ---------------------------------------------------------------------------
+// the persistent kernel
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kEstThreads)
+estimator_kernel(const __grid_constant__ EstParams P) {
+  extern __shared__ __align__(16) unsigned char est_smem[];
+  __shared__ PoolSmem psm;
+  __shared__ int s_item;
+  __shared__ int s_ok;
+  const int per_pair = P.pool_items + P.score_items;
+  const int total = P.n_groups * per_pair;
+  for (;;) {
+    if (threadIdx.x == 0) s_item = (int)atomicAdd(&P.sync[0], 1u);
+    __syncthreads();
+    const int x = s_item;
+    __syncthreads();
+    if (x >= total) return;
+    // queue order: pool(0), then pairs (pool(g+1), score(g)), last pair score(n-1) only
+    int g, y;
+    bool is_pool;
+    if (x < P.pool_items) {
+      is_pool = true;
+      g = 0;
+      y = x;
+    } else {
+      const int x2 = x - P.pool_items;
+      const int pair = x2 / per_pair;
+      const int rem = x2 - pair * per_pair;
+      if (pair < P.n_groups - 1 && rem < P.pool_items) {
+        is_pool = true;
+        g = pair + 1;
+        y = rem;
+      } else {
+        is_pool = false;
+        g = pair;
+        y = pair < P.n_groups - 1 ? rem - P.pool_items : rem;
+      }
+    }
+    if (is_pool) {
+      pool_item(P, g, y, psm);
+      continue;
+    }
+    // wait until the group's pooling and temperatures are published
+    if (threadIdx.x == 0) {
+      const uint32_t* ready = &P.sync[1 + P.n_groups + g];
+      int ok = 1;
+      if (ld_acquire_gpu(ready) == 0u) {
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_gpu(ready) == 0u) {
+          if (globaltimer_ns() - t0 > 2000000000ull) {
+            set_device_error(kDevErrTimeout);
+            ok = 0;
+            break;
+          }
+        }
+      }
+      s_ok = ok;
+    }
+    __syncthreads();
+    if (s_ok) score_item(P, g, y, est_smem);
+    __syncthreads();
+  }
 }
 
 }  // namespace prism

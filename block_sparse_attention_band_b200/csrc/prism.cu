@@ -32,7 +32,7 @@ struct Plan {
   int explicit_tau;
   float tau_hi, tau_lo;
   float scale;
-  size_t off_pool, off_part, off_tau, off_scores, off_mask, total;
+  size_t off_pool, off_part, off_tau, off_scores, off_mask, off_sync, sync_bytes, total;
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -42,6 +42,7 @@ int validate(const prism_config* cfg, Plan* pl) {
   if (cfg->batch <= 0 || cfg->hq <= 0 || cfg->hkv <= 0 || cfg->seqlen <= 0) return PRISM_ERR_SHAPE;
   if (cfg->head_dim != 128 || cfg->block != 128 || cfg->causal != 1) return PRISM_ERR_UNSUPPORTED;
   if (cfg->hq % cfg->hkv != 0) return PRISM_ERR_SHAPE;
+  if (cfg->hq / cfg->hkv > kMaxGroupHeads) return PRISM_ERR_UNSUPPORTED;
   if (cfg->seqlen % cfg->block != 0) return PRISM_ERR_SHAPE;
   const long long nb = cfg->seqlen / cfg->block;
   // TMA row coordinates are 32-bit; Top-P indices are 16-bit
@@ -109,6 +110,9 @@ int validate(const prism_config* cfg, Plan* pl) {
   off = align_up(off + (size_t)P.q_rows * 2 * tri * sizeof(float), 256);
   P.off_mask = off;
   off = align_up(off + (size_t)P.q_rows * P.nb * P.W * sizeof(uint32_t), 256);
+  P.off_sync = off;
+  P.sync_bytes = (1 + 2 * (size_t)P.kv_rows) * sizeof(uint32_t);
+  off = align_up(off + P.sync_bytes, 256);
   P.total = off;
   return PRISM_OK;
 }
@@ -122,15 +126,29 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 int g_dev_state[kMaxDevices];  // 0 unknown, 1 ready, <0 error code
 
-int topp_warps(int nb, size_t* smem) {
+// Shared memory of the persistent estimator: the score items' product tiles,
+// reused by the Top-P warps (each needs 8 bytes per key block + the bitset).
+struct EstLaunch {
+  int topp_warps, topp_stride;
+  size_t smem;
+};
+EstLaunch est_launch_shape(int nb) {
   const int W = (nb + 31) / 32;
-  const int nbp = (nb + 3) & ~3;
-  const size_t per = align_up((size_t)nbp * 8 + (size_t)W * 4, 16);
-  int warps = 4;
-  while (warps > 1 && per * warps > 200 * 1024) --warps;
-  *smem = per * warps;
-  return warps;
+  const int nbp = (nb + 7) & ~7;
+  EstLaunch L;
+  // two bands' logits (the first reused for keys) + one u16 member list + 256
+  // 64-bit bins + two bit rows per warp
+  L.topp_stride = (int)align_up((size_t)nbp * 10 + 256 * 8 + (size_t)W * 8, 16);
+  // dynamic shared memory: the product tiles, or as many Top-P warps as fit
+  // next to the static pool scratch (227 KB per CTA in all)
+  const size_t max_dyn = 232448 - sizeof(PoolSmem) - 256;
+  const size_t want = std::min<size_t>((size_t)(kEstThreads / 32) * L.topp_stride, max_dyn);
+  L.smem = std::max<size_t>(kGemmSmemBytes, want);
+  L.topp_warps = (int)std::max<size_t>(1, std::min<size_t>(kEstThreads / 32, L.smem / L.topp_stride));
+  return L;
 }
+
+int g_num_sms[kMaxDevices];
 
 int ensure_device() {
   int dev = 0;
@@ -157,10 +175,9 @@ int ensure_device() {
   }
   if (cudaFuncSetAttribute(attn::sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)attn::kSmemBytes) != cudaSuccess ||
-      cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kScoreSmemBytes) != cudaSuccess ||
-      cudaFuncSetAttribute(topp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
-          cudaSuccess)
+      cudaFuncSetAttribute(estimator_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)(232448 - sizeof(PoolSmem) - 256)) != cudaSuccess ||
+      cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return PRISM_ERR_CUDA;
   g_dev_state[dev] = 1;
   return PRISM_OK;
@@ -208,27 +225,44 @@ int launched() { return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR
 // ---------------------------------------------------------------------------
 int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, unsigned char* ws,
                  cudaStream_t st, float* dbg_scores, float* dbg_tau) {
-  float* pool = reinterpret_cast<float*>(ws + P.off_pool);
-  float* part = reinterpret_cast<float*>(ws + P.off_part);
-  float* tau = reinterpret_cast<float*>(ws + P.off_tau);
-  float* scores = dbg_scores ? dbg_scores : reinterpret_cast<float*>(ws + P.off_scores);
-  const int units = (P.q_rows + P.kv_rows) * P.nb;
-  pool_kernel<<<units, kPoolThreads, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(q),
-                                              reinterpret_cast<const __nv_bfloat16*>(k), P.q_rows,
-                                              P.nb, pool, part, P.bl);
-  if (launched() != PRISM_OK) return PRISM_ERR_CUDA;
-  tau_kernel<<<P.q_rows, kTauThreads, 0, st>>>(part, P.q_rows, P.hq, P.hkv, P.nb, P.bl.d_hi, P.bl.d_lo,
-                                               P.explicit_tau, P.tau_hi, P.tau_lo, tau, dbg_tau);
-  if (launched() != PRISM_OK) return PRISM_ERR_CUDA;
-  const int T = (P.nb + kScoreTile - 1) / kScoreTile;
-  dim3 sgrid(T * (T + 1) / 2, P.q_rows);
-  scores_kernel<<<sgrid, kScoreThreads, kScoreSmemBytes, st>>>(pool, P.q_rows, P.hq, P.hkv, P.nb, tau,
-                                                              P.bl.s1, P.bl.s2, P.bl.s3, scores);
-  if (launched() != PRISM_OK) return PRISM_ERR_CUDA;
-  size_t smem = 0;
-  const int warps = topp_warps(P.nb, &smem);
-  const int rows = P.q_rows * P.nb;
-  topp_kernel<<<(rows + warps - 1) / warps, warps * 32, smem, st>>>(scores, rows, P.nb, P.p_eff, mask);
+  EstParams E;
+  E.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  E.k = reinterpret_cast<const __nv_bfloat16*>(k);
+  E.pool = reinterpret_cast<float*>(ws + P.off_pool);
+  E.part = reinterpret_cast<float*>(ws + P.off_part);
+  E.tau = reinterpret_cast<float*>(ws + P.off_tau);
+  E.scores = dbg_scores ? dbg_scores : reinterpret_cast<float*>(ws + P.off_scores);
+  E.mask = mask;
+  E.dbg_tau = dbg_tau;
+  E.sync = reinterpret_cast<uint32_t*>(ws + P.off_sync);
+  E.hq = P.hq;
+  E.hkv = P.hkv;
+  E.G = P.hq / P.hkv;
+  E.nb = P.nb;
+  E.W = P.W;
+  E.q_rows = P.q_rows;
+  E.n_groups = P.kv_rows;
+  E.pool_item_span = (P.nb + kPoolTilesPerItem - 1) / kPoolTilesPerItem;
+  E.pool_items = (E.G + 1) * E.pool_item_span;
+  E.score_items = (E.G * P.nb + kScoreRows - 1) / kScoreRows;
+  const EstLaunch L = est_launch_shape(P.nb);
+  E.topp_warps = L.topp_warps;
+  E.topp_stride = L.topp_stride;
+  E.p = P.p_eff;
+  E.explicit_tau = P.explicit_tau;
+  E.tau_hi = P.tau_hi;
+  E.tau_lo = P.tau_lo;
+  E.bl = P.bl;
+  int dev = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, estimator_kernel, kEstThreads, L.smem) !=
+          cudaSuccess)
+    return PRISM_ERR_CUDA;
+  const long long items = (long long)E.n_groups * (E.pool_items + E.score_items);
+  const long long grid = std::min<long long>(items, (long long)g_num_sms[dev] * std::max(per_sm, 1));
+  // the queue head and the per-group counters start at zero on every call
+  if (cudaMemsetAsync(E.sync, 0, P.sync_bytes, st) != cudaSuccess) return PRISM_ERR_CUDA;
+  estimator_kernel<<<(unsigned)grid, kEstThreads, L.smem, st>>>(E);
   return launched();
 }
 
@@ -356,8 +390,10 @@ int prism_prefill(const prism_config* cfg, const void* q, const void* k, const v
 }
 
 // Same estimator as prism_estimate, with the library's built-in scratch array in
-// place of a caller-provided workspace.  Nothing in the scratch has to start
-// at zero: every word a kernel reads was written earlier in the same call.
+// place of a caller-provided workspace.  The work-queue counters, the only
+// words that must start at zero, are cleared on the stream at the start of
+// every call (as for prism_estimate); every other word a kernel reads is
+// written earlier in the same call.
 int prism_estimate_noalloc(const prism_config* cfg, const void* q, const void* k, uint32_t* mask,
                            prism_stream_t stream) {
   Plan P;

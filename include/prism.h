@@ -112,8 +112,10 @@ typedef struct prism_config {
  * Device workspace, in bytes, that prism_estimate / prism_prefill need for
  * `cfg` (prism_sparse_attn needs none).  Host-only; enqueues nothing.
  * Writes the size to *bytes.  The workspace holds the pooled Q/K means (fp32),
- * per-block energy partials, the temperatures and the fp32 band scores
- * (b * hq * 2 * nb(nb+1)/2 floats); its contents on return are unspecified.
+ * per-block energy partials, the temperatures, the fp32 band scores
+ * (b * hq * 2 * nb(nb+1)/2 floats) and the estimator's work-queue counters,
+ * which each call clears with a memset on its stream; its contents on return
+ * are unspecified.
  */
 int prism_workspace_size(const prism_config* cfg, size_t* bytes);
 
@@ -174,9 +176,11 @@ int prism_prefill(const prism_config* cfg, const void* q, const void* k, const v
  *     before any stream capture.
  *   - Calls no cudaMalloc, cudaFree or other allocating routine.
  *   - Every call on a device shares the one array, which keeps the previous
- *     call's contents: calls whose work overlaps on the GPU (different streams,
- *     or host threads, without ordering between them) race on it.  Order them
- *     on one stream, or synchronise between them.
+ *     call's contents; the few counters that must start at zero are cleared
+ *     on `stream` at the start of each call.  Calls whose work overlaps on
+ *     the GPU (different streams, or host threads, without ordering between
+ *     them) race on the array.  Order them on one stream, or synchronise
+ *     between them.
  */
 int prism_estimate_noalloc(const prism_config* cfg, const void* q, const void* k, uint32_t* mask,
                            prism_stream_t stream);

@@ -67,8 +67,9 @@ def test_workspace_size_formula():
 
     def up(x):
         return (x + 255) // 256 * 256
+    kv_rows = rows - q_rows
     expect = up(rows * nb * 128 * 4) + up(rows * nb * 4 * 4) + up(q_rows * 16) + up(q_rows * 2 * tri * 4) \
-        + up(q_rows * nb * 1 * 4)
+        + up(q_rows * nb * 1 * 4) + up((1 + 2 * kv_rows) * 4)
     assert n == expect
 
 
