@@ -10,7 +10,8 @@
 //
 //   pool(0), pool(1), score(0), pool(2), score(1), ..., pool(n-1), score(n-2), score(n-1)
 //
-// pool items (HBM-bound) stream 128x128 bf16 tiles of Q and K once and write
+// pool items (HBM-bound) stream 128x128 bf16 tiles of Q and K once (bulk
+// copies into a ring of shared-memory stages, several tiles in flight) and write
 // the fp32 block means (steps 1-2) and per-block energy partials (step 3);
 // the CTA that finishes the last pool item of a group also computes the
 // group's temperatures (steps 3-4) and publishes "group ready".  score items
@@ -36,8 +37,9 @@ struct BandLayout {
 };
 
 constexpr int kEstThreads = 512;      // 16 warps, one CTA per SM
-constexpr int kHalfThreads = 256;     // a pool item is reduced by two halves, one tile each
 constexpr int kPoolTilesPerItem = 8;  // 8 x 32 KB of Q or K per pool item
+constexpr uint32_t kTileBytes = 128 * 128 * 2;
+constexpr int kMaxPoolStages = 6;     // bulk-copy ring depth (32 KB stages)
 constexpr int kScoreRows = 64;        // (head, query block) rows per score item
 constexpr int kColTile = 128;         // key blocks per product column tile
 constexpr int kStageLD = kColTile + 1;
@@ -61,6 +63,7 @@ struct EstParams {
   int pool_item_span;  // pool items per head row
   int topp_warps;
   int topp_stride;  // bytes of shared memory per Top-P warp
+  int pool_stages;  // bulk-copy ring depth (<= kMaxPoolStages)
   float p;
   int explicit_tau;
   float tau_hi, tau_lo;
@@ -97,47 +100,42 @@ __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
 // energy partials.  Thread t holds 16-byte vectors of rows t/16 + 16 r at
 // dims 8 (t % 16) .. +7: each warp reads two full 256-byte rows.
 // ---------------------------------------------------------------------------
-struct PoolHalf {
+struct PoolSmem {
   float red[16][128];
   float mean[128];
   float wsum[4][3];
-};
-struct PoolSmem {
-  PoolHalf half[2];
   float sums[kMaxGroupHeads + 1][3];
+  uint64_t bars[kMaxPoolStages];
   int flag;
 };
 
-__device__ __forceinline__ void pool_load(uint4 (&v)[8], const __nv_bfloat16* tile) {
-  const int t = threadIdx.x & (kHalfThreads - 1);
+// Reduces one tile held in shared memory (128 rows x 256 bytes): thread t
+// sums the 16 rows 8k + t/64 of the bf16 pair in 32-bit word t % 64
+// (conflict-free), the 8 row groups are combined in a fixed order.  `refill`
+// runs once every thread has read the stage (it may overwrite it).
+template <class Refill>
+__device__ __forceinline__ void pool_tile(const uint32_t* tile, const EstParams& P, int hr, int blk, PoolSmem& sm,
+                                          Refill refill) {
+  const int t = threadIdx.x;
+  const int pw = t & 63, rg = t >> 6;
+  float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-  for (int r = 0; r < 8; ++r) v[r] = ldg_nc_v4(tile + (size_t)((t >> 4) + 16 * r) * 128 + (t & 15) * 8);
-}
-
-__device__ __forceinline__ void pool_reduce(const uint4 (&v)[8], const EstParams& P, int hr, int blk,
-                                            PoolHalf& sm) {
-  const int t = threadIdx.x & (kHalfThreads - 1);
-  const int bar_id = 1 + (threadIdx.x >> 8);
-  float acc[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    acc[0] += bf16lo(v[r].x); acc[1] += bf16hi(v[r].x);
-    acc[2] += bf16lo(v[r].y); acc[3] += bf16hi(v[r].y);
-    acc[4] += bf16lo(v[r].z); acc[5] += bf16hi(v[r].z);
-    acc[6] += bf16lo(v[r].w); acc[7] += bf16hi(v[r].w);
+  for (int k = 0; k < 16; ++k) {
+    const uint32_t w = tile[(rg + 8 * k) * 64 + pw];
+    a0 += bf16lo(w);
+    a1 += bf16hi(w);
   }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) sm.red[t >> 4][(t & 15) * 8 + e] = acc[e];
-  named_barrier(bar_id, kHalfThreads);
+  sm.red[rg][2 * pw] = a0;
+  sm.red[rg][2 * pw + 1] = a1;
+  __syncthreads();
+  refill();
   if (t < 128) {
     float s = 0.f;
 #pragma unroll
-    for (int g = 0; g < 16; ++g) s += sm.red[g][t];
+    for (int g = 0; g < 8; ++g) s += sm.red[g][t];
     sm.mean[t] = s * (1.0f / 128.0f);
   }
-  named_barrier(bar_id, kHalfThreads);
+  __syncthreads();
   if (t < 128) {
     const float m = sm.mean[P.bl.perm[t]];
     P.pool[((size_t)hr * P.nb + blk) * 128 + t] = m;
@@ -157,7 +155,7 @@ __device__ __forceinline__ void pool_reduce(const uint4 (&v)[8], const EstParams
       sm.wsum[t >> 5][2] = all;
     }
   }
-  named_barrier(bar_id, kHalfThreads);
+  __syncthreads();
   if (t < 3)
     P.part[((size_t)hr * P.nb + blk) * 4 + t] =
         (sm.wsum[0][t] + sm.wsum[1][t]) + (sm.wsum[2][t] + sm.wsum[3][t]);
@@ -182,11 +180,11 @@ __device__ void group_temperatures(const EstParams& P, int g, PoolSmem& sm) {
     for (int e = 0; e < 3; ++e) s[e] = warp_sum(s[e]);
     if (lane == 0)
 #pragma unroll
-      for (int e = 0; e < 3; ++e) sm.half[0].red[warp][e] = s[e];
+      for (int e = 0; e < 3; ++e) sm.red[warp][e] = s[e];
     __syncthreads();
     if (t < 3) {
       float a = 0.f;
-      for (int w = 0; w < kEstThreads / 32; ++w) a += sm.half[0].red[w][t];
+      for (int w = 0; w < kEstThreads / 32; ++w) a += sm.red[w][t];
       sm.sums[slot][t] = a;
     }
     __syncthreads();
@@ -224,7 +222,8 @@ __device__ void group_temperatures(const EstParams& P, int g, PoolSmem& sm) {
 // One pool item: kPoolTilesPerItem consecutive blocks of one head row of the
 // group (its Q heads, then its KV head), the next tile's loads in flight
 // while the current one is reduced.
-__device__ void pool_item(const EstParams& P, int g, int y, PoolSmem& sm) {
+__device__ void pool_item(const EstParams& P, int g, int y, PoolSmem& sm, unsigned char* ring, int stages,
+                          uint32_t& phases) {
   const int slot = y / P.pool_item_span;
   const int blk0 = (y - slot * P.pool_item_span) * kPoolTilesPerItem;
   const int blk1 = min(blk0 + kPoolTilesPerItem, P.nb);
@@ -238,19 +237,28 @@ __device__ void pool_item(const EstParams& P, int g, int y, PoolSmem& sm) {
     hr = P.q_rows + g;
     base = P.k + (size_t)g * P.nb * (128 * 128);
   }
-  // half h reduces tiles blk0 + h, blk0 + h + 2, ...; the next tile of the
-  // half is loaded while the current one is reduced
-  const int h = threadIdx.x >> 8;
-  PoolHalf& hs = sm.half[h];
-  uint4 va[8], vb[8];
-  if (blk0 + h < blk1) pool_load(va, base + (size_t)(blk0 + h) * (128 * 128));
-  for (int b = blk0 + h; b < blk1; b += 4) {
-    if (b + 2 < blk1) pool_load(vb, base + (size_t)(b + 2) * (128 * 128));
-    pool_reduce(va, P, hr, b, hs);
-    if (b + 2 < blk1) {
-      if (b + 4 < blk1) pool_load(va, base + (size_t)(b + 4) * (128 * 128));
-      pool_reduce(vb, P, hr, b + 2, hs);
-    }
+  // bulk-copy ring: up to `stages` tiles in flight, each stage refilled with
+  // the tile `stages` ahead as soon as every thread has read it
+  const int nt = blk1 - blk0;
+  const uint32_t ring0 = smem_u32(ring);
+  auto issue = [&](int tt) {
+    const int slot = tt % stages;
+    const uint32_t bar = smem_u32(&sm.bars[slot]);
+    mbar_arrive_expect_tx(bar, kTileBytes);
+    bulk_load(ring0 + slot * kTileBytes, base + (size_t)(blk0 + tt) * (128 * 128), kTileBytes, bar);
+  };
+  if (threadIdx.x == 0)
+    for (int tt = 0; tt < min(stages, nt); ++tt) issue(tt);
+  for (int tt = 0; tt < nt; ++tt) {
+    const int slot = tt % stages;
+    mbar_wait(smem_u32(&sm.bars[slot]), (phases >> slot) & 1u);  // a timeout is recorded on the device
+    phases ^= 1u << slot;
+    pool_tile(reinterpret_cast<const uint32_t*>(ring + (size_t)slot * kTileBytes), P, hr, blk0 + tt, sm, [&] {
+      if (threadIdx.x == 0 && tt + stages < nt) {
+        fence_proxy_async_smem();
+        issue(tt + stages);
+      }
+    });
   }
   // publish: count the item; the CTA that completes the group computes tau
   __syncthreads();
@@ -310,36 +318,31 @@ __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v)
 
 // Exact crossing among `cnt` members (<= 32) listed in S.cand, all ranked
 // behind mass `base`: returns the member c with ahead(c) < target <=
-// ahead(c) + e_c, or -1 if none reaches the target.
+// ahead(c) + e_c, or -1 if none reaches the target.  The members are sorted
+// across the warp by (d, j) with a bitonic network, then an inclusive scan of
+// their masses in that order finds the crossing.
 __device__ __forceinline__ int topp_exact32(const ToppScratch& S, int cnt, unsigned long long base,
                                             unsigned long long target, int lane) {
-  int j = -1;
-  uint32_t dj = 0xffffffffu;
-  uint32_t mj = 0u;
+  unsigned long long key = ~0ull;  // (d << 32) | j; absent members sort last
   if (lane < cnt) {
-    j = S.cand[lane];
-    dj = S.d[j];
-    mj = fixmass(key_value(dj));
+    const int j = S.cand[lane];
+    key = ((unsigned long long)S.d[j] << 32) | (uint32_t)j;
   }
-  unsigned long long ahead = 0ull;
-  int rank = 0;
 #pragma unroll
-  for (int l = 0; l < 32; ++l) {
-    const int jl = __shfl_sync(0xffffffffu, j, l);
-    const uint32_t dl = __shfl_sync(0xffffffffu, dj, l);
-    const uint32_t ml = __shfl_sync(0xffffffffu, mj, l);
-    if (l < cnt && lane < cnt && (dl < dj || (dl == dj && jl < j))) {
-      ahead += ml;
-      ++rank;
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, jj);
+      const bool take_min = ((lane & jj) == 0) == ((lane & k) == 0);
+      key = take_min ? (other < key ? other : key) : (other > key ? other : key);
     }
   }
-  const bool crosses = lane < cnt && base + ahead + mj >= target;
-  int best = crosses ? rank : 0x7fffffff;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, o));
-  if (best == 0x7fffffff) return -1;
-  const unsigned mk = __ballot_sync(0xffffffffu, crosses && rank == best);
-  return __shfl_sync(0xffffffffu, j, __ffs(mk) - 1);
+  const bool valid = lane < cnt;
+  const unsigned long long m = valid ? (unsigned long long)fixmass(key_value((uint32_t)(key >> 32))) : 0ull;
+  const unsigned long long incl = warp_scan_u64(m, lane);
+  const unsigned hit = __ballot_sync(0xffffffffu, valid && base + incl >= target);
+  if (hit == 0u) return -1;
+  return (int)(uint32_t)__shfl_sync(0xffffffffu, key, __ffs(hit) - 1);
 }
 
 // 64-bit bin mass kept as two 32-bit words: the low word's atomic add returns
@@ -776,6 +779,13 @@ estimator_kernel(const __grid_constant__ EstParams P) {
   __shared__ int s_item;
   __shared__ int s_ok;
   const int per_pair = P.pool_items + P.score_items;
+  const int stages = P.pool_stages;
+  uint32_t phases = 0u;  // parity to wait for next, one bit per ring stage
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < stages; ++st) mbar_init(smem_u32(&psm.bars[st]), 1u);
+    fence_mbar_init();
+  }
+  __syncthreads();
   const int total = P.n_groups * per_pair;
   for (;;) {
     if (threadIdx.x == 0) s_item = (int)atomicAdd(&P.sync[0], 1u);
@@ -805,7 +815,7 @@ estimator_kernel(const __grid_constant__ EstParams P) {
       }
     }
     if (is_pool) {
-      pool_item(P, g, y, psm);
+      pool_item(P, g, y, psm, est_smem, stages, phases);
       continue;
     }
     // wait until the group's pooling and temperatures are published

@@ -248,6 +248,7 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   const EstLaunch L = est_launch_shape(P.nb);
   E.topp_warps = L.topp_warps;
   E.topp_stride = L.topp_stride;
+  E.pool_stages = (int)std::min<size_t>(kMaxPoolStages, L.smem / kTileBytes);
   E.p = P.p_eff;
   E.explicit_tau = P.explicit_tau;
   E.tau_hi = P.tau_hi;
