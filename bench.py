@@ -143,6 +143,25 @@ def cpu_oracle_sample(q, k, v, mask_words, w, n_heads=1, n_rows=2, seed=0):
     return (t_est + t_attn) * 1e3, t_est * 1e3, t_attn * 1e3, sample
 
 
+def layer_workload(w, rank: int):
+    """Rank r times its own independent layer: the workload with seed + r."""
+    return gen.Workload(**{**w.__dict__, "seed": w.seed + rank})
+
+
+def reduce_max(values, dist, device):
+    """Max over ranks of each value (the slowest rank sets the job time)."""
+    if dist is None:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_value(ms_step_max: float, world: int) -> float:
+    """Job-wide ms per layer: every rank finishes one layer per step."""
+    return ms_step_max / world
+
+
 def blas_threads():
     try:
         import threadpoolctl
@@ -215,7 +234,7 @@ def main():
     torch.cuda.set_device(dev)
 
     # inputs: rank r runs the layer seeded seed + r (independent layers)
-    wr = gen.Workload(**{**w.__dict__, "seed": w.seed + rank})
+    wr = layer_workload(w, rank)
     q, k, v = gen.make_inputs(wr)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     hi, lo = gen.default_bands()
@@ -249,11 +268,7 @@ def main():
         torch.cuda.synchronize()
         barrier()
     clocks = clk.summary()
-    ms_step = ev0.elapsed_time(ev1) / args.steps
-    if dist is not None:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = reduce_max([ev0.elapsed_time(ev1) / args.steps], dist, dev)[0]
     assert pb.prism_get_last_device_error() == 0
 
     # ---------------- stage breakdown (same launches, events in between) ----
@@ -302,11 +317,7 @@ def main():
         torch.cuda.synchronize()
         if it > 0:
             e2e.append(ea.elapsed_time(eb))
-    e2e_ms = statistics.median(e2e)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = reduce_max([statistics.median(e2e)], dist, dev)[0]
     h2d = qh.nbytes + kh.nbytes + vh.nbytes
     d2h = oh.nbytes
 
@@ -320,7 +331,7 @@ def main():
         dist.destroy_process_group()
     if rank != 0:
         return
-    value = ms_step / world
+    value = job_value(ms_step, world)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
@@ -340,7 +351,7 @@ def main():
                      "traffic": None, "peak_source": f"{peak_src} bf16 sustained"},
         "estimator_roofline": {"bound": "hbm", "achieved": est_gbs, "peak": peak_hbm, "unit": "GB/s",
                                "frac": est_gbs / peak_hbm, "bytes": est_bytes, "peak_source": peak_src},
-        "e2e": {"value": e2e_ms / world, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": job_value(e2e_ms, world), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 5 * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
