@@ -15,45 +15,66 @@
 // the fp32 block means (steps 1-2) and per-block energy partials (step 3);
 // the CTA that finishes the last pool item of a group also computes the
 // group's temperatures (steps 3-4) and publishes "group ready".  score items
-// (ALU-bound) wait for their group, compute both bands' pooled logits with an
-// fp32 register-tiled product (step 5) and run softmax + Top-P + union per
-// row (steps 5-7).  Scoring of group g overlaps pooling of group g+1.  An
+// wait for their group, compute both bands' pooled logits on the tensor cores
+// (step 5; tcgen05 on a three-term bf16 split, fp32 accuracy) and run
+// softmax + Top-P + union per row (steps 5-7).  Scoring of
+// group g overlaps pooling of group g+1.  An
 // item only ever waits for items earlier in the queue, which running CTAs
 // hold and which never wait, so the schedule cannot deadlock; the wait is
 // bounded all the same.
 //
-// Band slicing is folded into the pooled layout: the pool items write the 128
-// pooled dims in a permuted order [high-only | both | low-only | neither], so
-// each band is a contiguous column range: high = [0, s2), low = [s1, s3).
+// Band slicing is folded into the pooled layout: the pool items write each
+// pooled row as [high-only | both | low-only] dims, every segment padded with
+// zeros to a multiple of 16 (one MMA K step), so each band is a contiguous,
+// aligned column range: high = [0, s2), low = [s1, s3).  Dims in neither band
+// are not stored.  The values are stored as three bf16 terms h + m + l (each
+// the rounding error of the ones before, 24 significant bits in all); the
+// products sum the six cross terms of order >= 2^-24 (hh, hm, mh, hl, lh,
+// mm), which matches an fp32 dot product.
 #pragma once
 #include "ptx.cuh"
 
 namespace prism {
 
 struct BandLayout {
-  uint8_t perm[128];  // pooled column c holds original dim perm[c]
-  int s1, s2, s3;     // segment boundaries (see above)
-  int d_hi, d_lo;     // band sizes
+  uint8_t src[192];  // pooled column c holds original dim src[c]; 255 = zero padding
+  int s1, s2, s3;    // 16-aligned segment boundaries (see above)
+  int dp;            // stored row length: a multiple of 64 (64, 128 or 192)
+  int d_hi, d_lo;    // band sizes
 };
 
 constexpr int kEstThreads = 512;      // 16 warps, one CTA per SM
 constexpr int kPoolTilesPerItem = 8;  // 8 x 32 KB of Q or K per pool item
 constexpr uint32_t kTileBytes = 128 * 128 * 2;
 constexpr int kMaxPoolStages = 6;     // bulk-copy ring depth (32 KB stages)
-constexpr int kScoreRows = 64;        // (head, query block) rows per score item
-constexpr int kColTile = 128;         // key blocks per product column tile
-constexpr int kStageLD = kColTile + 1;
-constexpr int kGemmSmemBytes = (128 * kScoreRows + 128 * kColTile + 2 * kScoreRows * kStageLD + 2 * kScoreRows) * 4;
+constexpr int kScoreRows = 128;       // query blocks (of one head) per score item = MMA M
+constexpr uint32_t kOpChunk = 128 * 64 * 2;  // one 64-dim x 128-row bf16 operand chunk (SW128)
+constexpr int kTerms = 3;             // bf16 terms per pooled value
+// product operands: A (3 terms x dp/64 chunks of 128 rows) once, B one term at
+// a time in kBSlots slots (dp/64 chunks of N rows; N = 128, or 64 when dp = 192)
+constexpr int kBSlots = 3;
+__host__ __device__ constexpr int score_cols(int dp) { return dp <= 128 ? 128 : 64; }
+__host__ __device__ constexpr int gemm_smem_bytes(int dp) {
+  return kTerms * (dp / 64) * (int)kOpChunk + kBSlots * (dp / 64) * score_cols(dp) * 128 + 1024;
+}
+constexpr int kGemmSmemBytes = gemm_smem_bytes(192);  // the largest layout: 144 + 3 x 24 KB + alignment
 constexpr int kMaxGroupHeads = 64;    // Q heads per KV head supported by the tau step
 constexpr float kLog2e = 1.4426950408889634f;
+
+// TMA descriptors of the three pooled bf16 terms [rows, dp]: boxes of 64 dims
+// x 128 rows (m[0..2]) and 64 dims x 64 rows (m[3..5])
+struct TermMaps {
+  CUtensorMap m[6];
+};
 
 struct EstParams {
   const __nv_bfloat16* q;
   const __nv_bfloat16* k;
-  float* pool;    // [q_rows + kv_rows, nb, 128] band-ordered means
+  __nv_bfloat16* pool_t[kTerms];  // [q_rows + kv_rows, nb, dp] band-segment means, bf16 terms h, m, l
   float* part;    // [q_rows + kv_rows, nb, 4] sum(mean^2): hi, lo, all
   float* tau;     // [q_rows, 4]: tau_hi, tau_lo, 1/(tau_hi sqrt d_hi), 1/(tau_lo sqrt d_lo)
-  float* scores;  // [q_rows, 2, nb(nb+1)/2] scaled band logits, packed rows
+  float* scores;      // scaled band logits in 128 x 128 tiles: [q_rows][tile (cr, cc), cc <= cr][band][128][128]
+  float* dbg_scores;  // optional copy in packed lower-triangular rows [q_rows, 2, nb(nb+1)/2]
   uint32_t* mask;
   float* dbg_tau;
   uint32_t* sync;  // [0] queue head, [1 + g] pool items done, [1 + n_groups + g] group ready
@@ -64,11 +85,20 @@ struct EstParams {
   int topp_warps;
   int topp_stride;  // bytes of shared memory per Top-P warp
   int pool_stages;  // bulk-copy ring depth (<= kMaxPoolStages)
+  int smem_bytes;   // dynamic shared memory of the launch
   float p;
   int explicit_tau;
   float tau_hi, tau_lo;
   BandLayout bl;
 };
+
+// The 128 x 128 score tile (row chunk cr, column chunk cc <= cr) of one
+// (batch, Q head): rows = query blocks 128 cr + r, columns = key blocks 128 cc + c.
+__device__ __forceinline__ float* score_tile(const EstParams& P, int bh, int cr, int cc) {
+  const int nch = (P.nb + 127) / 128;
+  const size_t pairs = (size_t)nch * (nch + 1) / 2;
+  return P.scores + ((size_t)bh * pairs + (size_t)cr * (cr + 1) / 2 + cc) * (2 * 128 * 128);
+}
 
 // ---------------------------------------------------------------------------
 // warp / ordering helpers
@@ -103,9 +133,11 @@ __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
 struct PoolSmem {
   float red[16][128];
   float mean[128];
-  float wsum[4][3];
+  float wsum[6][3];
   float sums[kMaxGroupHeads + 1][3];
   uint64_t bars[kMaxPoolStages];
+  uint64_t bar_a, bar_b[kBSlots], bar_free[kBSlots], bar_mma[2];  // score item: operands, slots, products
+  uint32_t tmem;
   int flag;
 };
 
@@ -136,13 +168,24 @@ __device__ __forceinline__ void pool_tile(const uint32_t* tile, const EstParams&
     sm.mean[t] = s * (1.0f / 128.0f);
   }
   __syncthreads();
-  if (t < 128) {
-    const float m = sm.mean[P.bl.perm[t]];
-    P.pool[((size_t)hr * P.nb + blk) * 128 + t] = m;
-    const float sq = m * m;
-    float hi = t < P.bl.s2 ? sq : 0.f;
-    float lo = (t >= P.bl.s1 && t < P.bl.s3) ? sq : 0.f;
-    float all = sq;
+  if (t < 192) {
+    float hi = 0.f, lo = 0.f, all = 0.f;
+    if (t < P.bl.dp) {
+      const int src = P.bl.src[t];
+      const float m = src < 128 ? sm.mean[src] : 0.f;
+      const __nv_bfloat16 th = __float2bfloat16_rn(m);
+      const float r1 = m - __bfloat162float(th);
+      const __nv_bfloat16 tm = __float2bfloat16_rn(r1);
+      const __nv_bfloat16 tl = __float2bfloat16_rn(r1 - __bfloat162float(tm));
+      const size_t o = ((size_t)hr * P.nb + blk) * P.bl.dp + t;
+      P.pool_t[0][o] = th;
+      P.pool_t[1][o] = tm;
+      P.pool_t[2][o] = tl;
+      const float sq = m * m;
+      hi = t < P.bl.s2 ? sq : 0.f;
+      lo = (t >= P.bl.s1 && t < P.bl.s3) ? sq : 0.f;
+    }
+    if (t < 128) all = sm.mean[t] * sm.mean[t];  // every dim, in or out of the bands
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       hi += __shfl_xor_sync(0xffffffffu, hi, o);
@@ -158,7 +201,7 @@ __device__ __forceinline__ void pool_tile(const uint32_t* tile, const EstParams&
   __syncthreads();
   if (t < 3)
     P.part[((size_t)hr * P.nb + blk) * 4 + t] =
-        (sm.wsum[0][t] + sm.wsum[1][t]) + (sm.wsum[2][t] + sm.wsum[3][t]);
+        ((sm.wsum[0][t] + sm.wsum[1][t]) + (sm.wsum[2][t] + sm.wsum[3][t])) + (sm.wsum[4][t] + sm.wsum[5][t]);
 }
 
 // steps (3b)-(4): RMS of every pooled band of the group's heads over all
@@ -593,129 +636,160 @@ __device__ void topp_band_row(const float* Lsm, int n, int W, float p, const Top
 }
 
 // ---------------------------------------------------------------------------
-// score item: kScoreRows (head, query block) rows of one group, enumerated
-// from the last query block down and over the group's heads; the rows share
-// the group's pooled K.  Step (5) logits for j <= i with an fp32 4x4
-// register tile per thread (the dims accumulate segment by segment so the
-// two bands share the products of their common dims), then steps (5)-(7)
-// per row.
+// score item: up to 128 consecutive query blocks i of one Q head (the rows of
+// one MMA, M = 128) against every key block j <= i of its KV head, in column
+// chunks of 128 (N = 128).  Step (5): logits of both bands on the tensor
+// cores, accumulators in tensor memory (two chunks in flight: the products
+// of chunk c+1 run while chunk c is scaled and written out).  Steps (5)-(7)
+// per row follow on the CUDA cores.
 // ---------------------------------------------------------------------------
-__device__ void score_item(const EstParams& P, int g, int y, unsigned char* smem) {
+struct ScoreState {  // mbarrier parities, carried across items
+  uint32_t a, b, free, mma;
+};
+
+// The B operand is streamed one term at a time ("units": chunk c, term t,
+// u = 3c + t) through kBSlots shared-memory slots, kBSlots - 1 units ahead.  Unit u's products pair its B
+// term with every A term whose cross term matters: t = h with A = h, m, l;
+// t = m with A = h, m; t = l with A = h.  High band K steps accumulate into
+// d, low band K steps into d + N.
+__device__ __forceinline__ void score_mma_unit(const EstParams& P, uint32_t d, uint32_t a0, uint32_t b, int term,
+                                               int n_cols, uint32_t idesc) {
+  const uint32_t nch = (uint32_t)P.bl.dp / 64;
+  const uint32_t b_bytes = (uint32_t)n_cols * 128;  // one 64-dim chunk of N rows
+  const int na = term == 0 ? 3 : (term == 1 ? 2 : 1);
+  for (int ta = 0; ta < na; ++ta) {
+    const uint32_t a = a0 + (uint32_t)ta * nch * kOpChunk;
+    const bool first = term == 0 && ta == 0;
+    for (int k = 0; k < P.bl.s2 / 16; ++k) {
+      const uint32_t ka = (uint32_t)(k >> 2) * kOpChunk + (uint32_t)(k & 3) * 32;
+      const uint32_t kb = (uint32_t)(k >> 2) * b_bytes + (uint32_t)(k & 3) * 32;
+      mma_bf16_ss(d, smem_desc_sw128(a + ka, 16, 1024), smem_desc_sw128(b + kb, 16, 1024), idesc,
+                  (first && k == 0) ? 0u : 1u);
+    }
+    for (int k = P.bl.s1 / 16; k < P.bl.s3 / 16; ++k) {
+      const uint32_t ka = (uint32_t)(k >> 2) * kOpChunk + (uint32_t)(k & 3) * 32;
+      const uint32_t kb = (uint32_t)(k >> 2) * b_bytes + (uint32_t)(k & 3) * 32;
+      mma_bf16_ss(d + (uint32_t)n_cols, smem_desc_sw128(a + ka, 16, 1024), smem_desc_sw128(b + kb, 16, 1024),
+                  idesc, (first && k == P.bl.s1 / 16) ? 0u : 1u);
+    }
+  }
+}
+
+__device__ void score_item(const EstParams& P, const CUtensorMap* tm, int g, int y, unsigned char* smem,
+                           PoolSmem& sm, ScoreState& ps) {
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int bi = g / P.hkv, kv = g - bi * P.hkv;
-  const int rows_total = P.G * P.nb;
-  const int idx0 = y * kScoreRows;
-  float* qT = reinterpret_cast<float*>(smem);      // [128 dims][64 rows]
-  float* kT = qT + 128 * kScoreRows;               // [128 dims][128 cols]
-  float* stage = kT + 128 * kColTile;              // [2][64][129]
-  float* scl = stage + 2 * kScoreRows * kStageLD;  // [64][2]
+  const int nchunk = (P.nb + kScoreRows - 1) / kScoreRows;
+  const int chunk = nchunk - 1 - y / P.G;  // longest rows first
+  const int bh = bi * P.hq + kv * P.G + y % P.G;
+  const int i0 = chunk * kScoreRows;
+  const int max_i = min(P.nb, i0 + kScoreRows) - 1;
+  const uint32_t nch = (uint32_t)P.bl.dp / 64;
+  const int ncolw = score_cols(P.bl.dp);  // N: key blocks per column chunk
+  const int ncol = max_i / ncolw + 1;
+  const int units = 3 * ncol;
   const size_t tri = (size_t)P.nb * (P.nb + 1) / 2;
-  const float* kbase = P.pool + (size_t)(P.q_rows + g) * P.nb * 128;
-  const int max_i = P.nb - 1 - idx0 / P.G;
-
-  // rows of this item: r -> (head h, block i); false past the group's end
-  auto row_of = [&](int r, int& bh, int& i) -> bool {
-    const int idx = idx0 + r;
-    if (idx >= rows_total) return false;
-    bh = bi * P.hq + kv * P.G + idx % P.G;
-    i = P.nb - 1 - idx / P.G;
-    return true;
+  const float sc_hi = P.tau[bh * 4 + 2], sc_lo = P.tau[bh * 4 + 3];
+  const uint32_t idesc = ncolw == 128 ? idesc_bf16_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 64, 0, 0);
+  const uint32_t sbase = (smem_u32(smem) + 1023u) & ~1023u;
+  if (sbase - smem_u32(smem) + (uint32_t)gemm_smem_bytes(P.bl.dp) - 1024u > (uint32_t)P.smem_bytes) {
+    if (t == 0) set_device_error(-6);  // PRISM_ERR_UNSUPPORTED (host sizing makes this unreachable)
+    return;
+  }
+  const uint32_t a0 = sbase;                                   // 3 terms x nch chunks x 16 KB
+  const uint32_t slot_bytes = nch * (uint32_t)ncolw * 128;    // one B term of N rows
+  const uint32_t b_base = sbase + kTerms * nch * kOpChunk;
+  auto slot_addr = [&](int u) { return b_base + (uint32_t)(u % kBSlots) * slot_bytes; };
+  const int arow = bh * P.nb + i0;          // pooled rows of the Q head
+  const int brow0 = (P.q_rows + g) * P.nb;  // pooled rows of the KV head
+  const uint32_t bar_a = smem_u32(&sm.bar_a);
+  auto bar_b = [&](int u) { return smem_u32(&sm.bar_b[u % kBSlots]); };
+  auto bar_f = [&](int u) { return smem_u32(&sm.bar_free[u % kBSlots]); };
+  auto bar_m = [&](int c) { return smem_u32(&sm.bar_mma[c & 1]); };
+  auto dacc = [&](int c) { return sm.tmem + 256u * (uint32_t)(c & 1); };
+  auto load_b = [&](int u) {
+    const int c = u / 3, term = u - 3 * c;
+    mbar_arrive_expect_tx(bar_b(u), slot_bytes);
+    for (uint32_t k = 0; k < nch; ++k)
+      tma_load_2d(slot_addr(u) + k * (uint32_t)ncolw * 128, &tm[term + (ncolw == 128 ? 0 : 3)], (int)(64 * k),
+                  brow0 + c * ncolw, bar_b(u));
+  };
+  // issue units [u0, u1): each waits for its B term, runs its products and
+  // releases its slot; unit u + kBSlots - 1's term goes into the slot of unit
+  // u - 1 as soon as that unit's products are done
+  auto issue = [&](int u0, int u1) {
+    for (int u = u0; u < u1; ++u) {
+      const int sl = u % kBSlots;
+      mbar_wait(bar_b(u), (ps.b >> sl) & 1u);
+      ps.b ^= 1u << sl;
+      tc_fence_after();
+      const int c = u / 3;
+      score_mma_unit(P, dacc(c), a0, slot_addr(u), u - 3 * c, ncolw, idesc);
+      mma_commit(bar_f(u));
+      if (u - 3 * c == 2) mma_commit(bar_m(c));
+      if (u + kBSlots - 1 < units) {
+        if (u >= 1) {
+          const int sp = (u - 1) % kBSlots;
+          mbar_wait(bar_f(u - 1), (ps.free >> sp) & 1u);
+          ps.free ^= 1u << sp;
+        }
+        load_b(u + kBSlots - 1);
+      }
+    }
   };
 
-  if (t < kScoreRows) {
-    int bh, i;
-    if (row_of(t, bh, i)) {
-      scl[2 * t] = P.tau[bh * 4 + 2];
-      scl[2 * t + 1] = P.tau[bh * 4 + 3];
-    } else {
-      scl[2 * t] = scl[2 * t + 1] = 0.f;
-    }
+  if (t == 0) {
+    mbar_arrive_expect_tx(bar_a, kTerms * nch * kOpChunk);
+    for (int term = 0; term < kTerms; ++term)
+      for (uint32_t k = 0; k < nch; ++k)
+        tma_load_2d(a0 + ((uint32_t)term * nch + k) * kOpChunk, &tm[term], (int)(64 * k), arow, bar_a);
+    for (int u = 0; u < kBSlots - 1 && u < units; ++u) load_b(u);
+    mbar_wait(bar_a, ps.a & 1u);
+    issue(0, 3);  // chunk 0
   }
-  // Qbar rows, transposed: lane -> row, warp -> 4-dim chunks
+  ps.a ^= 1u;
+  for (int c = 0; c < ncol; ++c) {
+    // chunk c+1's products go in (accumulators of chunk c-1 are read out)
+    if (t == 0 && c + 1 < ncol) issue(3 * (c + 1), 3 * (c + 2));
+    mbar_wait(bar_m(c), (ps.mma >> (c & 1)) & 1u);
+    ps.mma ^= 1u << (c & 1);
+    tc_fence_after();
+    // epilogue of chunk c: warp w reads TMEM lane quarter w % 4 and column
+    // quarter w / 4; thread = query block i writes its N / 4 key blocks of
+    // both bands into the score tile with 16-byte stores
+    {
+      const int q = warp & 3, cq = warp >> 2;
+      const int r = q * 32 + lane;
+      const int qw = ncolw / 4;
+      const int cbase = c * ncolw;                // first key block of this column chunk
+      float* tile = score_tile(P, bh, chunk, cbase >> 7);
+      float* row_hi = tile + r * 128 + (cbase & 127) + cq * qw;
+      float* row_lo = row_hi + 128 * 128;
+      for (int part = 0; part < qw; part += 16) {
+        const uint32_t taddr = dacc(c) + ((uint32_t)(q * 32) << 16) + (uint32_t)(cq * qw + part);
+        uint32_t vh[16], vl[16];
+        tmem_ld16(taddr, vh);
+        tmem_ld16(taddr + (uint32_t)ncolw, vl);
+        tmem_wait_ld_dep16(vh);
+        tmem_wait_ld_dep16(vl);
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const int r = rr * 32 + lane;
-    int bh = 0, i = 0;
-    const bool ok = row_of(r, bh, i);
-    const float* src = P.pool + ((size_t)bh * P.nb + i) * 128;
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      const int c = warp + 16 * cc;
-      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (ok) a = *reinterpret_cast<const float4*>(src + 4 * c);
-      qT[(4 * c + 0) * kScoreRows + r] = a.x;
-      qT[(4 * c + 1) * kScoreRows + r] = a.y;
-      qT[(4 * c + 2) * kScoreRows + r] = a.z;
-      qT[(4 * c + 3) * kScoreRows + r] = a.w;
-    }
-  }
-  const int ty = t >> 5, tx = t & 31;  // 16 x 32 threads, 4 x 4 outputs each
-  for (int j0 = 0; j0 <= max_i; j0 += kColTile) {
-    __syncthreads();  // the previous tile's kT and stage reads are done
-#pragma unroll
-    for (int rr = 0; rr < 4; ++rr) {
-      const int r = rr * 32 + lane;
-      const bool ok = j0 + r <= max_i;
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = warp + 16 * cc;
-        float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (ok) b = *reinterpret_cast<const float4*>(kbase + (size_t)(j0 + r) * 128 + 4 * c);
-        kT[(4 * c + 0) * kColTile + r] = b.x;
-        kT[(4 * c + 1) * kColTile + r] = b.y;
-        kT[(4 * c + 2) * kColTile + r] = b.z;
-        kT[(4 * c + 3) * kColTile + r] = b.w;
-      }
-    }
-    __syncthreads();
-    float a[4][4], b[4][4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int w = 0; w < 4; ++w) a[u][w] = b[u][w] = 0.f;
-    auto fma_range = [&](float(&acc)[4][4], int d0, int d1) {
-#pragma unroll 4
-      for (int d = d0; d < d1; ++d) {
-        const float4 qa = *reinterpret_cast<const float4*>(&qT[d * kScoreRows + 4 * ty]);
-        const float4 kb = *reinterpret_cast<const float4*>(&kT[d * kColTile + 4 * tx]);
-        const float qv[4] = {qa.x, qa.y, qa.z, qa.w};
-        const float kvv[4] = {kb.x, kb.y, kb.z, kb.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-          for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(qv[u], kvv[w], acc[u][w]);
-      }
-    };
-    fma_range(a, 0, P.bl.s1);        // high-only dims
-    fma_range(b, P.bl.s1, P.bl.s2);  // dims of both bands
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int w = 0; w < 4; ++w) a[u][w] += b[u][w];  // a = high band
-    fma_range(b, P.bl.s2, P.bl.s3);  // b = low band
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int row = 4 * ty + u;
-      const float sh = scl[2 * row], sl = scl[2 * row + 1];
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        stage[row * kStageLD + 4 * tx + w] = a[u][w] * sh;
-        stage[kScoreRows * kStageLD + row * kStageLD + 4 * tx + w] = b[u][w] * sl;
-      }
-    }
-    __syncthreads();
-    for (int r = warp; r < kScoreRows; r += kEstThreads / 32) {
-      int bh, i;
-      if (!row_of(r, bh, i)) continue;
-      float* out_hi = P.scores + (size_t)bh * 2 * tri + (size_t)i * (i + 1) / 2;
-      float* out_lo = out_hi + tri;
-      for (int c = lane; c < kColTile; c += 32) {
-        const int jj = j0 + c;
-        if (jj <= i) {
-          out_hi[jj] = stage[r * kStageLD + c];
-          out_lo[jj] = stage[kScoreRows * kStageLD + r * kStageLD + c];
+        for (int e = 0; e < 16; e += 4) {
+          *reinterpret_cast<float4*>(row_hi + part + e) =
+              make_float4(__uint_as_float(vh[e]) * sc_hi, __uint_as_float(vh[e + 1]) * sc_hi,
+                          __uint_as_float(vh[e + 2]) * sc_hi, __uint_as_float(vh[e + 3]) * sc_hi);
+          *reinterpret_cast<float4*>(row_lo + part + e) =
+              make_float4(__uint_as_float(vl[e]) * sc_lo, __uint_as_float(vl[e + 1]) * sc_lo,
+                          __uint_as_float(vl[e + 2]) * sc_lo, __uint_as_float(vl[e + 3]) * sc_lo);
         }
       }
+    }
+    tc_fence_before();
+    __syncthreads();  // chunk c's accumulators are read
+  }
+  if (t == 0) {  // the releases of the last kBSlots units were not waited for yet
+    for (int u = max(units - kBSlots, 0); u < units; ++u) {
+      mbar_wait(bar_f(u), (ps.free >> (u % kBSlots)) & 1u);
+      ps.free ^= 1u << (u % kBSlots);
     }
   }
   __syncthreads();  // this CTA's score rows are visible to all its threads
@@ -731,23 +805,27 @@ __device__ void score_item(const EstParams& P, int g, int y, unsigned char* smem
     S.h = reinterpret_cast<unsigned long long*>(wb + (size_t)nbp * 10);
     S.kb = reinterpret_cast<uint32_t*>(wb + (size_t)nbp * 10 + kTopPBins * 8);
     uint32_t* bits = S.kb + P.W;
-    for (int r = warp; r < kScoreRows; r += P.topp_warps) {
-      int bh, i;
-      if (!row_of(r, bh, i)) continue;
+    for (int i = i0 + warp; i <= max_i; i += P.topp_warps) {
       for (int w = lane; w < P.W; w += 32) bits[w] = 0u;
       __syncwarp();
-      // both bands' rows -> shared memory in one round trip (32 loads in flight per lane)
-      const float* row_hi = P.scores + (size_t)bh * 2 * tri + (size_t)i * (i + 1) / 2;
-      const float* row_lo = row_hi + tri;
+      // both bands' rows -> shared memory in one round trip (32 loads in flight
+      // per lane); the row is spread over the tiles (i / 128, cc), cc <= i / 128
       const int n = i + 1;
+      const int cr = i >> 7, r = i & 127;
       float* Lhi = reinterpret_cast<float*>(S.d);
+      float* dbg_hi = P.dbg_scores ? P.dbg_scores + (size_t)bh * 2 * tri + (size_t)i * (i + 1) / 2 : nullptr;
       for (int j0 = 0; j0 < n; j0 += 512) {
         float xh[16], xl[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const int j = j0 + u * 32 + lane;
-          xh[u] = j < n ? row_hi[j] : 0.f;
-          xl[u] = j < n ? row_lo[j] : 0.f;
+          xh[u] = 0.f;
+          xl[u] = 0.f;
+          if (j < n) {
+            const float* src = score_tile(P, bh, cr, j >> 7) + r * 128 + (j & 127);
+            xh[u] = src[0];
+            xl[u] = src[128 * 128];
+          }
         }
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
@@ -755,6 +833,10 @@ __device__ void score_item(const EstParams& P, int g, int y, unsigned char* smem
           if (j < n) {
             Lhi[j] = xh[u];
             S.L2[j] = xl[u];
+            if (dbg_hi) {
+              dbg_hi[j] = xh[u];
+              dbg_hi[tri + j] = xl[u];
+            }
           }
         }
       }
@@ -772,8 +854,8 @@ __device__ void score_item(const EstParams& P, int g, int y, unsigned char* smem
 // ---------------------------------------------------------------------------
 // the persistent kernel
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kEstThreads)
-estimator_kernel(const __grid_constant__ EstParams P) {
+__global__ void __launch_bounds__(kEstThreads, 1)
+estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ TermMaps tms) {
   extern __shared__ __align__(16) unsigned char est_smem[];
   __shared__ PoolSmem psm;
   __shared__ int s_item;
@@ -781,18 +863,33 @@ estimator_kernel(const __grid_constant__ EstParams P) {
   const int per_pair = P.pool_items + P.score_items;
   const int stages = P.pool_stages;
   uint32_t phases = 0u;  // parity to wait for next, one bit per ring stage
+  ScoreState ss = {0u, 0u, 0u, 0u};
   if (threadIdx.x == 0) {
     for (int st = 0; st < stages; ++st) mbar_init(smem_u32(&psm.bars[st]), 1u);
+    mbar_init(smem_u32(&psm.bar_a), 1u);
+    for (int sl = 0; sl < kBSlots; ++sl) {
+      mbar_init(smem_u32(&psm.bar_b[sl]), 1u);
+      mbar_init(smem_u32(&psm.bar_free[sl]), 1u);
+    }
+    mbar_init(smem_u32(&psm.bar_mma[0]), 1u);
+    mbar_init(smem_u32(&psm.bar_mma[1]), 1u);
     fence_mbar_init();
+    for (int m = 0; m < 6; ++m) tma_prefetch_desc(&tms.m[m]);
   }
+  if ((threadIdx.x >> 5) == 0) {  // the score items' accumulators: 2 chunks x (hi, lo) x 128 columns
+    tmem_alloc(smem_u32(&psm.tmem), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
   const int total = P.n_groups * per_pair;
   for (;;) {
     if (threadIdx.x == 0) s_item = (int)atomicAdd(&P.sync[0], 1u);
     __syncthreads();
     const int x = s_item;
     __syncthreads();
-    if (x >= total) return;
+    if (x >= total) break;
     // queue order: pool(0), then pairs (pool(g+1), score(g)), last pair score(n-1) only
     int g, y;
     bool is_pool;
@@ -835,8 +932,14 @@ estimator_kernel(const __grid_constant__ EstParams P) {
       s_ok = ok;
     }
     __syncthreads();
-    if (s_ok) score_item(P, g, y, est_smem);
+    if (s_ok) score_item(P, tms.m, g, y, est_smem, psm, ss);
     __syncthreads();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if ((threadIdx.x >> 5) == 0) {
+    tc_fence_after();
+    tmem_dealloc(psm.tmem, 512);
   }
 }
 

@@ -32,7 +32,7 @@ struct Plan {
   int explicit_tau;
   float tau_hi, tau_lo;
   float scale;
-  size_t off_pool, off_part, off_tau, off_scores, off_mask, off_sync, sync_bytes, total;
+  size_t off_pool[kTerms], off_part, off_tau, off_scores, off_mask, off_sync, sync_bytes, total;
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -77,19 +77,22 @@ int validate(const prism_config* cfg, Plan* pl) {
   P.W = (P.nb + 31) / 32;
   P.q_rows = P.b * P.hq;
   P.kv_rows = P.b * P.hkv;
-  // pooled column order: [high only | both | low only | neither]
+  // pooled row layout: [high only | both | low only], each segment zero-padded
+  // to a multiple of 16 columns (one MMA K step), total padded to 64
+  std::memset(P.bl.src, 0xff, sizeof(P.bl.src));
   int c = 0;
-  for (int d = 0; d < 128; ++d)
-    if (in_hi[d] && !in_lo[d]) P.bl.perm[c++] = (uint8_t)d;
+  auto segment = [&](bool want_hi, bool want_lo) {
+    for (int d = 0; d < 128; ++d)
+      if (in_hi[d] == want_hi && in_lo[d] == want_lo) P.bl.src[c++] = (uint8_t)d;
+    c = (c + 15) & ~15;
+  };
+  segment(true, false);
   P.bl.s1 = c;
-  for (int d = 0; d < 128; ++d)
-    if (in_hi[d] && in_lo[d]) P.bl.perm[c++] = (uint8_t)d;
+  segment(true, true);
   P.bl.s2 = c;
-  for (int d = 0; d < 128; ++d)
-    if (!in_hi[d] && in_lo[d]) P.bl.perm[c++] = (uint8_t)d;
+  segment(false, true);
   P.bl.s3 = c;
-  for (int d = 0; d < 128; ++d)
-    if (!in_hi[d] && !in_lo[d]) P.bl.perm[c++] = (uint8_t)d;
+  P.bl.dp = (c + 63) & ~63;
   P.bl.d_hi = cfg->n_hi;
   P.bl.d_lo = cfg->n_lo;
   P.p_eff = cfg->p >= 1.f ? 1.f : cfg->p;
@@ -100,14 +103,17 @@ int validate(const prism_config* cfg, Plan* pl) {
   const size_t rows = (size_t)P.q_rows + P.kv_rows;
   const size_t tri = (size_t)P.nb * (P.nb + 1) / 2;
   size_t off = 0;
-  P.off_pool = off;
-  off = align_up(off + rows * P.nb * 128 * sizeof(float), 256);
+  for (int term = 0; term < kTerms; ++term) {
+    P.off_pool[term] = off;
+    off = align_up(off + rows * P.nb * P.bl.dp * sizeof(__nv_bfloat16), 256);
+  }
   P.off_part = off;
   off = align_up(off + rows * P.nb * 4 * sizeof(float), 256);
   P.off_tau = off;
   off = align_up(off + (size_t)P.q_rows * 4 * sizeof(float), 256);
   P.off_scores = off;
-  off = align_up(off + (size_t)P.q_rows * 2 * tri * sizeof(float), 256);
+  const size_t nch = ((size_t)P.nb + 127) / 128;
+  off = align_up(off + (size_t)P.q_rows * (nch * (nch + 1) / 2) * 2 * 128 * 128 * sizeof(float), 256);
   P.off_mask = off;
   off = align_up(off + (size_t)P.q_rows * P.nb * P.W * sizeof(uint32_t), 256);
   P.off_sync = off;
@@ -205,12 +211,12 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-int make_map(CUtensorMap* map, const void* base, size_t rows) {
+int make_map(CUtensorMap* map, const void* base, size_t rows, int cols = 128, int box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return PRISM_ERR_CUDA;
-  cuuint64_t dims[2] = {128, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {128 * sizeof(__nv_bfloat16)};
-  cuuint32_t box[2] = {64, 128};
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * sizeof(__nv_bfloat16)};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -228,10 +234,12 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   EstParams E;
   E.q = reinterpret_cast<const __nv_bfloat16*>(q);
   E.k = reinterpret_cast<const __nv_bfloat16*>(k);
-  E.pool = reinterpret_cast<float*>(ws + P.off_pool);
+  for (int term = 0; term < kTerms; ++term)
+    E.pool_t[term] = reinterpret_cast<__nv_bfloat16*>(ws + P.off_pool[term]);
   E.part = reinterpret_cast<float*>(ws + P.off_part);
   E.tau = reinterpret_cast<float*>(ws + P.off_tau);
-  E.scores = dbg_scores ? dbg_scores : reinterpret_cast<float*>(ws + P.off_scores);
+  E.scores = reinterpret_cast<float*>(ws + P.off_scores);
+  E.dbg_scores = dbg_scores;
   E.mask = mask;
   E.dbg_tau = dbg_tau;
   E.sync = reinterpret_cast<uint32_t*>(ws + P.off_sync);
@@ -244,11 +252,12 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   E.n_groups = P.kv_rows;
   E.pool_item_span = (P.nb + kPoolTilesPerItem - 1) / kPoolTilesPerItem;
   E.pool_items = (E.G + 1) * E.pool_item_span;
-  E.score_items = (E.G * P.nb + kScoreRows - 1) / kScoreRows;
+  E.score_items = E.G * ((P.nb + kScoreRows - 1) / kScoreRows);
   const EstLaunch L = est_launch_shape(P.nb);
   E.topp_warps = L.topp_warps;
   E.topp_stride = L.topp_stride;
   E.pool_stages = (int)std::min<size_t>(kMaxPoolStages, L.smem / kTileBytes);
+  E.smem_bytes = (int)L.smem;
   E.p = P.p_eff;
   E.explicit_tau = P.explicit_tau;
   E.tau_hi = P.tau_hi;
@@ -261,9 +270,17 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
     return PRISM_ERR_CUDA;
   const long long items = (long long)E.n_groups * (E.pool_items + E.score_items);
   const long long grid = std::min<long long>(items, (long long)g_num_sms[dev] * std::max(per_sm, 1));
+  // the score items' operands: pooled rows as bf16 [rows, dp], boxes of 64
+  // dims x 128 rows (A, and B when dp <= 128) or x 64 rows (B when dp = 192)
+  TermMaps tms;
+  const size_t prow = ((size_t)P.q_rows + P.kv_rows) * P.nb;
+  for (int term = 0; term < kTerms; ++term)
+    if (make_map(&tms.m[term], E.pool_t[term], prow, P.bl.dp, 128) != PRISM_OK ||
+        make_map(&tms.m[3 + term], E.pool_t[term], prow, P.bl.dp, 64) != PRISM_OK)
+      return PRISM_ERR_CUDA;
   // the queue head and the per-group counters start at zero on every call
   if (cudaMemsetAsync(E.sync, 0, P.sync_bytes, st) != cudaSuccess) return PRISM_ERR_CUDA;
-  estimator_kernel<<<(unsigned)grid, kEstThreads, L.smem, st>>>(E);
+  estimator_kernel<<<(unsigned)grid, kEstThreads, L.smem, st>>>(E, tms);
   return launched();
 }
 

@@ -111,7 +111,8 @@ typedef struct prism_config {
 /*
  * Device workspace, in bytes, that prism_estimate / prism_prefill need for
  * `cfg` (prism_sparse_attn needs none).  Host-only; enqueues nothing.
- * Writes the size to *bytes.  The workspace holds the pooled Q/K means (fp32),
+ * Writes the size to *bytes.  The workspace holds the pooled Q/K means (three
+ * bf16 terms per value),
  * per-block energy partials, the temperatures, the fp32 band scores
  * (b * hq * 2 * nb(nb+1)/2 floats) and the estimator's work-queue counters,
  * which each call clears with a memset on its stream; its contents on return
@@ -169,8 +170,8 @@ int prism_prefill(const prism_config* cfg, const void* q, const void* k, const v
  * (device pointers, layouts as above); no dbg outputs.
  *   - Problems whose workspace (prism_workspace_size) exceeds 32 MiB are
  *     rejected with PRISM_ERR_SCRATCH_LIMIT before anything is enqueued
- *     (the Llama-3-8B shape, 32 Q / 8 KV heads, batch 1, fits up to 54,912
- *     tokens = 429 blocks).
+ *     (the Llama-3-8B shape, 32 Q / 8 KV heads, batch 1, fits up to 32,896
+ *     tokens = 257 blocks).
  *   - The first call on a device looks up the array's device address with
  *     cudaGetSymbolAddress while that device is current; make that first call
  *     before any stream capture.

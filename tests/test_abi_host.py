@@ -63,13 +63,14 @@ def test_workspace_size_formula():
     s, n = _ws_size(_cfg())
     assert s == 0
     nb, rows, q_rows = 8, 6, 4
-    tri = nb * (nb + 1) // 2
+    # scores: one 128 x 128 tile pair (row chunk 0, column chunk 0) per Q row
 
     def up(x):
         return (x + 255) // 256 * 256
     kv_rows = rows - q_rows
-    expect = up(rows * nb * 128 * 4) + up(rows * nb * 4 * 4) + up(q_rows * 16) + up(q_rows * 2 * tri * 4) \
-        + up(q_rows * nb * 1 * 4) + up((1 + 2 * kv_rows) * 4)
+    dp = 128  # default bands: 32 high-only + 32 shared + 64 low-only padded columns
+    expect = 3 * up(rows * nb * dp * 2) + up(rows * nb * 4 * 4) + up(q_rows * 16) \
+        + up(q_rows * 1 * 2 * 128 * 128 * 4) + up(q_rows * nb * 1 * 4) + up((1 + 2 * kv_rows) * 4)
     assert n == expect
 
 

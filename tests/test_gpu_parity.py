@@ -114,6 +114,23 @@ def test_explicit_tau_and_custom_bands(cuda_device):
     P.check_mask(mask, ref, w.p)
 
 
+@pytest.mark.parametrize("seed,n_hi,n_lo", [(41, 17, 50), (42, 60, 90), (43, 5, 3), (44, 100, 100)])
+def test_irregular_bands(seed, n_hi, n_lo, cuda_device):
+    """Arbitrary band index sets (any sizes, overlaps, dims in neither band):
+    exercises the zero-padded segment layout of the pooled rows."""
+    w = gen.small_workload(f"bands_{seed}", 1, 4, 2, 19 * 128, seed=seed, p=0.9)
+    q, k, v, qd, kd, vd = _inputs(w, cuda_device)
+    rng = np.random.default_rng(seed)
+    hi = sorted(rng.choice(128, n_hi, replace=False).tolist())
+    lo = sorted(rng.choice(128, n_lo, replace=False).tolist())
+    cfg = P.make_cfg(w, bands=(hi, lo))
+    mask, sc, tau, _ = P.run_estimate(cfg, qd, kd)
+    ref = oracle.estimate(q, k, hi, lo, w.p)
+    P.check_tau(tau, ref)
+    P.check_scores(sc, ref)
+    P.check_mask(mask, ref, w.p)
+
+
 def test_small_p_sparse_rows(cuda_device):
     w = gen.small_workload("sparse_nb48", 1, 2, 1, 48 * 128, seed=35, p=0.3)
     q, k, v, qd, kd, vd = _inputs(w, cuda_device)
