@@ -131,12 +131,16 @@ __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
 // dims 8 (t % 16) .. +7: each warp reads two full 256-byte rows.
 // ---------------------------------------------------------------------------
 struct PoolSmem {
-  float red[16][128];
+  union {                   // pool and score items never overlap in a CTA
+    float red[16][128];     // pool item: row-group partial sums; temperatures: warp partials
+    float rmax[2][2][128];  // score item: row maxima per column half and band
+  };
   float mean[128];
   float wsum[6][3];
   float sums[kMaxGroupHeads + 1][3];
   uint64_t bars[kMaxPoolStages];
-  uint64_t bar_a, bar_b[kBSlots], bar_free[kBSlots], bar_mma[2];  // score item: operands, slots, products
+  uint64_t bar_a, bar_b[kBSlots], bar_free[kBSlots], bar_mma[2], bar_acc[2];  // score item: operands, slots,
+                                                                            // products, accumulators read
   uint32_t tmem;
   int flag;
 };
@@ -207,7 +211,7 @@ __device__ __forceinline__ void pool_tile(const uint32_t* tile, const EstParams&
 // steps (3b)-(4): RMS of every pooled band of the group's heads over all
 // blocks and the temperatures of its Q heads (reading R1 of the pages: the
 // band's pooled Q x K energy relative to the full spectrum's).
-__device__ void group_temperatures(const EstParams& P, int g, PoolSmem& sm) {
+__device__ __forceinline__ void group_temperatures(const EstParams& P, int g, PoolSmem& sm) {
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int bi = g / P.hkv, kv = g - bi * P.hkv;
   for (int slot = 0; slot <= P.G; ++slot) {  // slots 0..G-1: Q heads, G: the KV head
@@ -265,7 +269,7 @@ __device__ void group_temperatures(const EstParams& P, int g, PoolSmem& sm) {
 // One pool item: kPoolTilesPerItem consecutive blocks of one head row of the
 // group (its Q heads, then its KV head), the next tile's loads in flight
 // while the current one is reduced.
-__device__ void pool_item(const EstParams& P, int g, int y, PoolSmem& sm, unsigned char* ring, int stages,
+__device__ __forceinline__ void pool_item(const EstParams& P, int g, int y, PoolSmem& sm, unsigned char* ring, int stages,
                           uint32_t& phases) {
   const int slot = y / P.pool_item_span;
   const int blk0 = (y - slot * P.pool_item_span) * kPoolTilesPerItem;
@@ -327,11 +331,9 @@ __device__ void pool_item(const EstParams& P, int g, int y, PoolSmem& sm, unsign
 // ---------------------------------------------------------------------------
 // Shared-memory scratch of one Top-P warp.
 struct ToppScratch {
-  uint32_t* d;            // [n] logits, then the rank keys d_j (below)
-  float* L2;              // [n] the second band's logits, loaded with the first
+  uint32_t* d;            // [n] the rank keys d_j (below)
   uint16_t* cand;         // [n] members of the crossing bin
   unsigned long long* h;  // [256] bin masses
-  uint32_t* kb;           // [W] blocks of bins before the crossing bin
 };
 
 constexpr int kTopPBins = 256;
@@ -396,27 +398,29 @@ __device__ __forceinline__ void bin_add(uint32_t* lo, uint32_t* hi, int b, uint3
   if (old > ~x) atomicAdd(&hi[b], 1u);
 }
 
-// Softmax (step 5) + Top-P (step 6) of one band row of n scaled logits held
-// in shared memory; ORs the kept blocks into bits[].
+// Softmax (step 5) + Top-P (step 6) of one band row of n scaled logits; ORs
+// the kept blocks into bits[].  The row lives in the item's score tiles: key
+// block j at row[(j / 128) * kTilePair + j % 128]; rmax is its maximum.
 //
 // e_j = 2^((L_j - max) log2 e); blocks ranked by (-e_j, j) == (d_j, j) with
 // the exact order-reversing key d_j.  Radix selection on the keys: bins of 16
 // per octave of e (bin = d >> 19, the last one collecting everything below
 // 2^-14) hold their mass exactly (e_j in 2^-31 fixed point, 64-bit exact
 // sums), so one scan gives Z, the crossing bin and the mass ranked before it
-// as exact integers.  Blocks of earlier bins are kept, of later bins dropped;
-// the crossing bin's members are ranked exactly (pairwise when <= 32, else by
-// refining on the lower key bits the same way).  A block is kept iff the
-// mass ranked strictly ahead of it is < p Z.
-__device__ void topp_band_row(const float* Lsm, int n, int W, float p, const ToppScratch& S, uint32_t* bits,
-                              int lane) {
+// as exact integers.  Blocks of earlier bins are kept, of later bins dropped.
+// A member x of the crossing bin is kept iff the mass ranked strictly ahead
+// of it is below the target p Z (the top block always): with <= 32 members
+// every member sums the masses of the members ahead of it directly, else the
+// bin is refined on the lower key bits the same way.
+constexpr size_t kTilePair = 2 * 128 * 128;  // floats per score tile pair (both bands)
+constexpr int kSegPerLane = 16;              // logits per lane per pass (512 per warp)
+
+__device__ __forceinline__ void topp_band_row(const float* row, float rmax, int n, float p, const ToppScratch& S,
+                                              uint32_t* bits, float* dbg, int lane) {
   const unsigned lt = (1u << lane) - 1u;
-  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 4
-  for (int j0 = 0; j0 < n; j0 += 32) {
-    const int j = j0 + lane;
-    if (j < n) mx[(j0 >> 5) & 3] = fmaxf(mx[(j0 >> 5) & 3], Lsm[j]);
-  }
+  constexpr int kSeg = 32 * kSegPerLane;
+  if (dbg)
+    for (int j = lane; j < n; j += 32) dbg[j] = row[(size_t)(j >> 7) * kTilePair + (j & 127)];
   const int nw = (n + 31) >> 5;
   if (p >= 1.0f) {  // every causal block is kept
     for (int w = lane; w < nw; w += 32) {
@@ -426,7 +430,7 @@ __device__ void topp_band_row(const float* Lsm, int n, int W, float p, const Top
     __syncwarp();
     return;
   }
-  const float m = warp_max(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]))) * kLog2e;
+  const float m = rmax * kLog2e;
   uint32_t* hlo = reinterpret_cast<uint32_t*>(S.h);
   uint32_t* hhi = hlo + kTopPBins;
   for (int b = lane; b < kTopPBins; b += 32) {
@@ -434,15 +438,23 @@ __device__ void topp_band_row(const float* Lsm, int n, int W, float p, const Top
     hhi[b] = 0u;
   }
   __syncwarp();
-  // e_j, keys, exact bin masses
-#pragma unroll 4
-  for (int j0 = 0; j0 < n; j0 += 32) {
-    const int j = j0 + lane;
-    if (j < n) {
-      const float e = fast_exp2(fmaf(Lsm[j], kLog2e, -m));
-      const uint32_t d = rank_key(e);
-      S.d[j] = d;
-      bin_add(hlo, hhi, (int)min(d >> 19, (uint32_t)(kTopPBins - 1)), fixmass(e));
+  // e_j, keys, exact bin masses: a batch of loads, then their arithmetic
+  for (int j0 = 0; j0 < n; j0 += kSeg) {
+    float x[kSegPerLane];
+#pragma unroll
+    for (int u = 0; u < kSegPerLane; ++u) {
+      const int j = j0 + u * 32 + lane;
+      x[u] = j < n ? row[(size_t)(j >> 7) * kTilePair + (j & 127)] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kSegPerLane; ++u) {
+      const int j = j0 + u * 32 + lane;
+      if (j < n) {
+        const float e = fast_exp2(fmaf(x[u], kLog2e, -m));
+        const uint32_t d = rank_key(e);
+        S.d[j] = d;
+        bin_add(hlo, hhi, (int)min(d >> 19, (uint32_t)(kTopPBins - 1)), fixmass(e));
+      }
     }
   }
   __syncwarp();
@@ -475,162 +487,176 @@ __device__ void topp_band_row(const float* Lsm, int n, int W, float p, const Top
     xb = found ? __shfl_sync(0xffffffffu, bin, sl) : kTopPBins - 1;
     base = found ? __shfl_sync(0xffffffffu, bb, sl) : Z;
   }
-  // one pass: keep the earlier bins, list the crossing bin's members
+  // one pass: keep the earlier bins, list the crossing bin's members; lane u
+  // collects mask word u of each batch
   int cnt = 0;
-#pragma unroll 2
+  for (int j0 = 0; j0 < n; j0 += kSeg) {
+    uint32_t dv[kSegPerLane];
+#pragma unroll
+    for (int u = 0; u < kSegPerLane; ++u) {
+      const int j = j0 + u * 32 + lane;
+      dv[u] = j < n ? S.d[j] : 0u;
+    }
+    uint32_t myw = 0u;
+#pragma unroll
+    for (int u = 0; u < kSegPerLane; ++u) {
+      const int j = j0 + u * 32 + lane;
+      const int b = (int)min(dv[u] >> 19, (uint32_t)(kTopPBins - 1));
+      const bool valid = j < n;
+      const unsigned mb = __ballot_sync(0xffffffffu, valid && b < xb);
+      const bool in = valid && b == xb;
+      const unsigned mi = __ballot_sync(0xffffffffu, in);
+      if (in) S.cand[cnt + __popc(mi & lt)] = (uint16_t)j;
+      cnt += __popc(mi);
+      if (lane == u) myw = mb;
+    }
+    const int w = (j0 >> 5) + lane;
+    if (lane < kSegPerLane && w < nw) bits[w] |= myw;
+  }
+  __syncwarp();
+  const unsigned long long lim = target > 0ull ? target : 1ull;
+  if (cnt <= 32) {
+    // member x is kept iff base + (mass of the members ranked ahead of it) < lim
+    uint32_t dx = 0xffffffffu, mx = 0u;
+    int jx = 0x7fffffff;
+    if (lane < cnt) {
+      jx = S.cand[lane];
+      dx = S.d[jx];
+      mx = fixmass(key_value(dx));
+    }
+    unsigned long long ahead = base;
+    for (int y = 0; y < cnt; ++y) {
+      const uint32_t dy = __shfl_sync(0xffffffffu, dx, y);
+      const int jy = __shfl_sync(0xffffffffu, jx, y);
+      const uint32_t my = __shfl_sync(0xffffffffu, mx, y);
+      if (dy < dx || (dy == dx && jy < jx)) ahead += my;
+    }
+    if (lane < cnt && ahead < lim) atomicOr(&bits[jx >> 5], 1u << (jx & 31));
+    __syncwarp();
+    return;
+  }
+  // refine on lower key bits, 8-bit digits: a regular bin spans 2^19 keys
+  // (digits at shifts 11, 3, 0), the catch-all bin up to 2^30 (22, 14, 6, 0)
+  int cross = -1;
+  uint32_t lo_key = (uint32_t)xb << 19;
+  const bool wide = xb == kTopPBins - 1;
+  for (int level = 0;; ++level) {
+    const int sh = wide ? (level == 0 ? 22 : level == 1 ? 14 : level == 2 ? 6 : 0)
+                        : (level == 0 ? 11 : level == 1 ? 3 : 0);
+    for (int b = lane; b < kTopPBins; b += 32) {
+      hlo[b] = 0u;
+      hhi[b] = 0u;
+    }
+    __syncwarp();
+    for (int x0 = 0; x0 < cnt; x0 += 32) {
+      const int x = x0 + lane;
+      if (x < cnt) {
+        const uint32_t d = S.d[S.cand[x]];
+        bin_add(hlo, hhi, (int)min((d - lo_key) >> sh, (uint32_t)(kTopPBins - 1)), fixmass(key_value(d)));
+      }
+    }
+    __syncwarp();
+    unsigned long long h2[8], t2 = 0ull;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      h2[u] = ((unsigned long long)hhi[lane * 8 + u] << 32) | hlo[lane * 8 + u];
+      t2 += h2[u];
+    }
+    const unsigned long long inc2 = warp_scan_u64(t2, lane);
+    unsigned long long run = inc2 - t2;
+    int bin2 = -1;
+    unsigned long long bb = 0ull;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (bin2 < 0 && base + run + h2[u] >= target && h2[u] > 0ull) {
+        bin2 = lane * 8 + u;
+        bb = base + run;
+      }
+      run += h2[u];
+    }
+    const unsigned f2 = __ballot_sync(0xffffffffu, bin2 >= 0);
+    if (f2 == 0u) {
+      // (exact sums make this unreachable) the members' mass stays below
+      // the target: all of them are kept -- the cut is the last member
+      uint32_t bd = 0u;
+      int bj = -1;
+      for (int x = lane; x < cnt; x += 32) {
+        const int jj = S.cand[x];
+        const uint32_t dd = S.d[jj];
+        if (bj < 0 || dd > bd || (dd == bd && jj > bj)) {
+          bd = dd;
+          bj = jj;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const uint32_t od = __shfl_xor_sync(0xffffffffu, bd, o);
+        const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+        if (bj < 0 || (oj >= 0 && (od > bd || (od == bd && oj > bj)))) {
+          bd = od;
+          bj = oj;
+        }
+      }
+      cross = bj;
+      break;
+    }
+    const int sl = __ffs(f2) - 1;
+    const int xb2 = __shfl_sync(0xffffffffu, bin2, sl);
+    base = __shfl_sync(0xffffffffu, bb, sl);
+    const uint32_t blo = lo_key + ((uint32_t)xb2 << sh);
+    const uint32_t bhi = sh == 0 ? blo : blo + ((1u << sh) - 1u);
+    int c2 = 0;
+    for (int x0 = 0; x0 < cnt; x0 += 32) {
+      const int x = x0 + lane;
+      int jj = 0;
+      bool in = false;
+      if (x < cnt) {
+        jj = S.cand[x];
+        const uint32_t d = S.d[jj];
+        in = d >= blo && d <= bhi;
+      }
+      const unsigned mk = __ballot_sync(0xffffffffu, in);
+      __syncwarp();
+      if (in) S.cand[c2 + __popc(mk & lt)] = (uint16_t)jj;
+      c2 += __popc(mk);
+    }
+    __syncwarp();
+    cnt = c2;
+    lo_key = blo;
+    if (cnt <= 32) {
+      cross = topp_exact32(S, cnt, base, target, lane);
+      break;
+    }
+    if (sh == 0) {
+      // equal keys: the first member (by index) whose cumulative mass
+      // reaches the target
+      const unsigned long long me = (unsigned long long)fixmass(key_value(blo));
+      unsigned long long acc = base;
+      for (int x0 = 0; x0 < cnt && cross < 0; x0 += 32) {
+        const int x = x0 + lane;
+        const bool ok = x < cnt;
+        const unsigned mk = __ballot_sync(0xffffffffu, ok);
+        const int pos = __popc(mk & lt);
+        const bool hit = ok && acc + me * (unsigned long long)(pos + 1) >= target;
+        const unsigned hm = __ballot_sync(0xffffffffu, hit);
+        if (hm) cross = __shfl_sync(0xffffffffu, ok ? (int)S.cand[x] : 0, __ffs(hm) - 1);
+        acc += me * (unsigned long long)__popc(mk);
+      }
+      break;
+    }
+  }
+  __syncwarp();
+  // every block ranked at or ahead of the crossing
+  const uint32_t dc = cross >= 0 ? S.d[cross] : 0xffffffffu;
   for (int j0 = 0; j0 < n; j0 += 32) {
     const int j = j0 + lane;
-    bool before = false, in = false;
+    bool keep = false;
     if (j < n) {
-      const int b = (int)min(S.d[j] >> 19, (uint32_t)(kTopPBins - 1));
-      before = b < xb;
-      in = b == xb;
-    }
-    const unsigned mb = __ballot_sync(0xffffffffu, before), mi = __ballot_sync(0xffffffffu, in);
-    if (in) S.cand[cnt + __popc(mi & lt)] = (uint16_t)j;
-    cnt += __popc(mi);
-    if (lane == 0) bits[j0 >> 5] |= mb;
-  }
-  __syncwarp();
-  // rank the crossing bin's members
-  int cross = -1;
-  bool refined = false;
-  if (cnt <= 32) {
-    cross = topp_exact32(S, cnt, base, target, lane);
-  } else {
-    // refine on lower key bits, 8-bit digits: a regular bin spans 2^19 keys
-    // (digits at shifts 11, 3, 0), the catch-all bin up to 2^30 (22, 14, 6, 0)
-    refined = true;
-    uint32_t lo_key = (uint32_t)xb << 19;
-    const bool wide = xb == kTopPBins - 1;
-    for (int level = 0;; ++level) {
-      const int sh = wide ? (level == 0 ? 22 : level == 1 ? 14 : level == 2 ? 6 : 0)
-                          : (level == 0 ? 11 : level == 1 ? 3 : 0);
-      for (int b = lane; b < kTopPBins; b += 32) {
-        hlo[b] = 0u;
-        hhi[b] = 0u;
-      }
-      __syncwarp();
-      for (int x0 = 0; x0 < cnt; x0 += 32) {
-        const int x = x0 + lane;
-        if (x < cnt) {
-          const uint32_t d = S.d[S.cand[x]];
-          bin_add(hlo, hhi, (int)min((d - lo_key) >> sh, (uint32_t)(kTopPBins - 1)), fixmass(key_value(d)));
-        }
-      }
-      __syncwarp();
-      unsigned long long h2[8], t2 = 0ull;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        h2[u] = ((unsigned long long)hhi[lane * 8 + u] << 32) | hlo[lane * 8 + u];
-        t2 += h2[u];
-      }
-      const unsigned long long inc2 = warp_scan_u64(t2, lane);
-      unsigned long long run = inc2 - t2;
-      int bin2 = -1;
-      unsigned long long bb = 0ull;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (bin2 < 0 && base + run + h2[u] >= target && h2[u] > 0ull) {
-          bin2 = lane * 8 + u;
-          bb = base + run;
-        }
-        run += h2[u];
-      }
-      const unsigned f2 = __ballot_sync(0xffffffffu, bin2 >= 0);
-      if (f2 == 0u) {
-        // (exact sums make this unreachable) the members' mass stays below
-        // the target: all of them are kept -- the cut is the last member
-        uint32_t bd = 0u;
-        int bj = -1;
-        for (int x = lane; x < cnt; x += 32) {
-          const int jj = S.cand[x];
-          const uint32_t dd = S.d[jj];
-          if (bj < 0 || dd > bd || (dd == bd && jj > bj)) {
-            bd = dd;
-            bj = jj;
-          }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const uint32_t od = __shfl_xor_sync(0xffffffffu, bd, o);
-          const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
-          if (bj < 0 || (oj >= 0 && (od > bd || (od == bd && oj > bj)))) {
-            bd = od;
-            bj = oj;
-          }
-        }
-        cross = bj;
-        break;
-      }
-      const int sl = __ffs(f2) - 1;
-      const int xb2 = __shfl_sync(0xffffffffu, bin2, sl);
-      base = __shfl_sync(0xffffffffu, bb, sl);
-      const uint32_t blo = lo_key + ((uint32_t)xb2 << sh);
-      const uint32_t bhi = sh == 0 ? blo : blo + ((1u << sh) - 1u);
-      int c2 = 0;
-      for (int x0 = 0; x0 < cnt; x0 += 32) {
-        const int x = x0 + lane;
-        int jj = 0;
-        bool in = false;
-        if (x < cnt) {
-          jj = S.cand[x];
-          const uint32_t d = S.d[jj];
-          in = d >= blo && d <= bhi;
-        }
-        const unsigned mk = __ballot_sync(0xffffffffu, in);
-        __syncwarp();
-        if (in) S.cand[c2 + __popc(mk & lt)] = (uint16_t)jj;
-        c2 += __popc(mk);
-      }
-      __syncwarp();
-      cnt = c2;
-      lo_key = blo;
-      if (cnt <= 32) {
-        cross = topp_exact32(S, cnt, base, target, lane);
-        break;
-      }
-      if (sh == 0) {
-        // equal keys: the first member (by index) whose cumulative mass
-        // reaches the target
-        const unsigned long long me = (unsigned long long)fixmass(key_value(blo));
-        unsigned long long acc = base;
-        for (int x0 = 0; x0 < cnt && cross < 0; x0 += 32) {
-          const int x = x0 + lane;
-          const bool ok = x < cnt;
-          const unsigned mk = __ballot_sync(0xffffffffu, ok);
-          const int pos = __popc(mk & lt);
-          const bool hit = ok && acc + me * (unsigned long long)(pos + 1) >= target;
-          const unsigned hm = __ballot_sync(0xffffffffu, hit);
-          if (hm) cross = __shfl_sync(0xffffffffu, ok ? (int)S.cand[x] : 0, __ffs(hm) - 1);
-          acc += me * (unsigned long long)__popc(mk);
-        }
-        break;
-      }
-    }
-  }
-  __syncwarp();
-  if (!refined) {
-    // the crossing bin's members ranked at or ahead of the crossing
-    const uint32_t dc = cross >= 0 ? S.d[cross] : 0u;
-    if (lane < cnt) {
-      const int j = S.cand[lane];
       const uint32_t d = S.d[j];
-      if (cross < 0 || d < dc || (d == dc && j <= cross)) atomicOr(&bits[j >> 5], 1u << (j & 31));
+      keep = cross < 0 || d < dc || (d == dc && j <= cross);
     }
-  } else {
-    // general case: every block ranked at or ahead of the crossing
-    const uint32_t dc = cross >= 0 ? S.d[cross] : 0xffffffffu;
-    for (int j0 = 0; j0 < n; j0 += 32) {
-      const int j = j0 + lane;
-      bool keep = false;
-      if (j < n) {
-        const uint32_t d = S.d[j];
-        keep = cross < 0 || d < dc || (d == dc && j <= cross);
-      }
-      const unsigned word = __ballot_sync(0xffffffffu, keep);
-      if (lane == 0) bits[j0 >> 5] |= word;
-    }
+    const unsigned word = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) bits[j0 >> 5] |= word;
   }
   __syncwarp();
 }
@@ -638,45 +664,49 @@ __device__ void topp_band_row(const float* Lsm, int n, int W, float p, const Top
 // ---------------------------------------------------------------------------
 // score item: up to 128 consecutive query blocks i of one Q head (the rows of
 // one MMA, M = 128) against every key block j <= i of its KV head, in column
-// chunks of 128 (N = 128).  Step (5): logits of both bands on the tensor
-// cores, accumulators in tensor memory (two chunks in flight: the products
-// of chunk c+1 run while chunk c is scaled and written out).  Steps (5)-(7)
-// per row follow on the CUDA cores.
+// chunks of N = 128 (64 for the widest band layout).  Step (5): logits of
+// both bands on the tensor cores, accumulators in tensor memory, double
+// buffered; warp roles: warp 0 lane 0 streams the operands (TMA), warp 1
+// lane 0 issues the products, warps 4-11 read the accumulators of a finished
+// chunk, scale them, write the score tiles and keep the row maxima.  Steps
+// (5)-(7) per row follow on all 16 warps.
 // ---------------------------------------------------------------------------
-struct ScoreState {  // mbarrier parities, carried across items
-  uint32_t a, b, free, mma;
+struct ScoreState {  // mbarrier parities, carried across items (each role keeps its own)
+  uint32_t a, b, free, mma, acc;
 };
 
 // The B operand is streamed one term at a time ("units": chunk c, term t,
-// u = 3c + t) through kBSlots shared-memory slots, kBSlots - 1 units ahead.  Unit u's products pair its B
-// term with every A term whose cross term matters: t = h with A = h, m, l;
-// t = m with A = h, m; t = l with A = h.  High band K steps accumulate into
-// d, low band K steps into d + N.
+// u = 3c + t) through kBSlots shared-memory slots.  Unit u's products pair
+// its B term with every A term whose cross term matters: t = h with A = h, m,
+// l; t = m with A = h, m; t = l with A = h.  High band K steps accumulate
+// into d, low band K steps into d + N.
 __device__ __forceinline__ void score_mma_unit(const EstParams& P, uint32_t d, uint32_t a0, uint32_t b, int term,
                                                int n_cols, uint32_t idesc) {
   const uint32_t nch = (uint32_t)P.bl.dp / 64;
   const uint32_t b_bytes = (uint32_t)n_cols * 128;  // one 64-dim chunk of N rows
   const int na = term == 0 ? 3 : (term == 1 ? 2 : 1);
+  const int k_hi = P.bl.s2 / 16, k_lo0 = P.bl.s1 / 16, k_lo1 = P.bl.s3 / 16;
+  // a descriptor's start address field is the byte address / 16, so an
+  // operand offset is added to the descriptor directly
+  const uint64_t bdesc = smem_desc_sw128(b, 16, 1024);
   for (int ta = 0; ta < na; ++ta) {
-    const uint32_t a = a0 + (uint32_t)ta * nch * kOpChunk;
+    const uint64_t adesc = smem_desc_sw128(a0 + (uint32_t)ta * nch * kOpChunk, 16, 1024);
     const bool first = term == 0 && ta == 0;
-    for (int k = 0; k < P.bl.s2 / 16; ++k) {
-      const uint32_t ka = (uint32_t)(k >> 2) * kOpChunk + (uint32_t)(k & 3) * 32;
-      const uint32_t kb = (uint32_t)(k >> 2) * b_bytes + (uint32_t)(k & 3) * 32;
-      mma_bf16_ss(d, smem_desc_sw128(a + ka, 16, 1024), smem_desc_sw128(b + kb, 16, 1024), idesc,
-                  (first && k == 0) ? 0u : 1u);
+    for (int k = 0; k < k_hi; ++k) {
+      const uint32_t ka = ((uint32_t)(k >> 2) * kOpChunk + (uint32_t)(k & 3) * 32) >> 4;
+      const uint32_t kb = ((uint32_t)(k >> 2) * b_bytes + (uint32_t)(k & 3) * 32) >> 4;
+      mma_bf16_ss(d, adesc + ka, bdesc + kb, idesc, (first && k == 0) ? 0u : 1u);
     }
-    for (int k = P.bl.s1 / 16; k < P.bl.s3 / 16; ++k) {
-      const uint32_t ka = (uint32_t)(k >> 2) * kOpChunk + (uint32_t)(k & 3) * 32;
-      const uint32_t kb = (uint32_t)(k >> 2) * b_bytes + (uint32_t)(k & 3) * 32;
-      mma_bf16_ss(d + (uint32_t)n_cols, smem_desc_sw128(a + ka, 16, 1024), smem_desc_sw128(b + kb, 16, 1024),
-                  idesc, (first && k == P.bl.s1 / 16) ? 0u : 1u);
+    for (int k = k_lo0; k < k_lo1; ++k) {
+      const uint32_t ka = ((uint32_t)(k >> 2) * kOpChunk + (uint32_t)(k & 3) * 32) >> 4;
+      const uint32_t kb = ((uint32_t)(k >> 2) * b_bytes + (uint32_t)(k & 3) * 32) >> 4;
+      mma_bf16_ss(d + (uint32_t)n_cols, adesc + ka, bdesc + kb, idesc, (first && k == k_lo0) ? 0u : 1u);
     }
   }
 }
 
-__device__ void score_item(const EstParams& P, const CUtensorMap* tm, int g, int y, unsigned char* smem,
-                           PoolSmem& sm, ScoreState& ps) {
+__device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap* tm, int g, int y,
+                                           unsigned char* smem, PoolSmem& sm, ScoreState& ps) {
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int bi = g / P.hkv, kv = g - bi * P.hkv;
   const int nchunk = (P.nb + kScoreRows - 1) / kScoreRows;
@@ -689,110 +719,148 @@ __device__ void score_item(const EstParams& P, const CUtensorMap* tm, int g, int
   const int ncol = max_i / ncolw + 1;
   const int units = 3 * ncol;
   const size_t tri = (size_t)P.nb * (P.nb + 1) / 2;
-  const float sc_hi = P.tau[bh * 4 + 2], sc_lo = P.tau[bh * 4 + 3];
   const uint32_t idesc = ncolw == 128 ? idesc_bf16_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 64, 0, 0);
   const uint32_t sbase = (smem_u32(smem) + 1023u) & ~1023u;
   if (sbase - smem_u32(smem) + (uint32_t)gemm_smem_bytes(P.bl.dp) - 1024u > (uint32_t)P.smem_bytes) {
     if (t == 0) set_device_error(-6);  // PRISM_ERR_UNSUPPORTED (host sizing makes this unreachable)
     return;
   }
-  const uint32_t a0 = sbase;                                   // 3 terms x nch chunks x 16 KB
-  const uint32_t slot_bytes = nch * (uint32_t)ncolw * 128;    // one B term of N rows
+  const uint32_t a0 = sbase;                                 // 3 terms x nch chunks x 16 KB
+  const uint32_t slot_bytes = nch * (uint32_t)ncolw * 128;  // one B term of N rows
   const uint32_t b_base = sbase + kTerms * nch * kOpChunk;
   auto slot_addr = [&](int u) { return b_base + (uint32_t)(u % kBSlots) * slot_bytes; };
-  const int arow = bh * P.nb + i0;          // pooled rows of the Q head
-  const int brow0 = (P.q_rows + g) * P.nb;  // pooled rows of the KV head
-  const uint32_t bar_a = smem_u32(&sm.bar_a);
   auto bar_b = [&](int u) { return smem_u32(&sm.bar_b[u % kBSlots]); };
   auto bar_f = [&](int u) { return smem_u32(&sm.bar_free[u % kBSlots]); };
   auto bar_m = [&](int c) { return smem_u32(&sm.bar_mma[c & 1]); };
+  auto bar_e = [&](int c) { return smem_u32(&sm.bar_acc[c & 1]); };
   auto dacc = [&](int c) { return sm.tmem + 256u * (uint32_t)(c & 1); };
-  auto load_b = [&](int u) {
-    const int c = u / 3, term = u - 3 * c;
-    mbar_arrive_expect_tx(bar_b(u), slot_bytes);
-    for (uint32_t k = 0; k < nch; ++k)
-      tma_load_2d(slot_addr(u) + k * (uint32_t)ncolw * 128, &tm[term + (ncolw == 128 ? 0 : 3)], (int)(64 * k),
-                  brow0 + c * ncolw, bar_b(u));
-  };
-  // issue units [u0, u1): each waits for its B term, runs its products and
-  // releases its slot; unit u + kBSlots - 1's term goes into the slot of unit
-  // u - 1 as soon as that unit's products are done
-  auto issue = [&](int u0, int u1) {
-    for (int u = u0; u < u1; ++u) {
-      const int sl = u % kBSlots;
-      mbar_wait(bar_b(u), (ps.b >> sl) & 1u);
-      ps.b ^= 1u << sl;
-      tc_fence_after();
-      const int c = u / 3;
-      score_mma_unit(P, dacc(c), a0, slot_addr(u), u - 3 * c, ncolw, idesc);
-      mma_commit(bar_f(u));
-      if (u - 3 * c == 2) mma_commit(bar_m(c));
-      if (u + kBSlots - 1 < units) {
-        if (u >= 1) {
-          const int sp = (u - 1) % kBSlots;
-          mbar_wait(bar_f(u - 1), (ps.free >> sp) & 1u);
-          ps.free ^= 1u << sp;
-        }
-        load_b(u + kBSlots - 1);
-      }
-    }
-  };
 
-  if (t == 0) {
-    mbar_arrive_expect_tx(bar_a, kTerms * nch * kOpChunk);
-    for (int term = 0; term < kTerms; ++term)
-      for (uint32_t k = 0; k < nch; ++k)
-        tma_load_2d(a0 + ((uint32_t)term * nch + k) * kOpChunk, &tm[term], (int)(64 * k), arow, bar_a);
-    for (int u = 0; u < kBSlots - 1 && u < units; ++u) load_b(u);
-    mbar_wait(bar_a, ps.a & 1u);
-    issue(0, 3);  // chunk 0
-  }
-  ps.a ^= 1u;
-  for (int c = 0; c < ncol; ++c) {
-    // chunk c+1's products go in (accumulators of chunk c-1 are read out)
-    if (t == 0 && c + 1 < ncol) issue(3 * (c + 1), 3 * (c + 2));
-    mbar_wait(bar_m(c), (ps.mma >> (c & 1)) & 1u);
-    ps.mma ^= 1u << (c & 1);
-    tc_fence_after();
-    // epilogue of chunk c: warp w reads TMEM lane quarter w % 4 and column
-    // quarter w / 4; thread = query block i writes its N / 4 key blocks of
-    // both bands into the score tile with 16-byte stores
-    {
-      const int q = warp & 3, cq = warp >> 2;
-      const int r = q * 32 + lane;
-      const int qw = ncolw / 4;
-      const int cbase = c * ncolw;                // first key block of this column chunk
-      float* tile = score_tile(P, bh, chunk, cbase >> 7);
-      float* row_hi = tile + r * 128 + (cbase & 127) + cq * qw;
-      float* row_lo = row_hi + 128 * 128;
-      for (int part = 0; part < qw; part += 16) {
-        const uint32_t taddr = dacc(c) + ((uint32_t)(q * 32) << 16) + (uint32_t)(cq * qw + part);
-        uint32_t vh[16], vl[16];
-        tmem_ld16(taddr, vh);
-        tmem_ld16(taddr + (uint32_t)ncolw, vl);
-        tmem_wait_ld_dep16(vh);
-        tmem_wait_ld_dep16(vl);
-#pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-          *reinterpret_cast<float4*>(row_hi + part + e) =
-              make_float4(__uint_as_float(vh[e]) * sc_hi, __uint_as_float(vh[e + 1]) * sc_hi,
-                          __uint_as_float(vh[e + 2]) * sc_hi, __uint_as_float(vh[e + 3]) * sc_hi);
-          *reinterpret_cast<float4*>(row_lo + part + e) =
-              make_float4(__uint_as_float(vl[e]) * sc_lo, __uint_as_float(vl[e + 1]) * sc_lo,
-                          __uint_as_float(vl[e + 2]) * sc_lo, __uint_as_float(vl[e + 3]) * sc_lo);
+  if (warp == 0) {
+    if (lane == 0) {  // operand producer
+      const int arow = bh * P.nb + i0;          // pooled rows of the Q head
+      const int brow0 = (P.q_rows + g) * P.nb;  // pooled rows of the KV head
+      fence_proxy_async_smem();                 // generic writes of the last item before async ones
+      const uint32_t bar_a = smem_u32(&sm.bar_a);
+      mbar_arrive_expect_tx(bar_a, kTerms * nch * kOpChunk);
+      for (int term = 0; term < kTerms; ++term)
+        for (uint32_t k = 0; k < nch; ++k)
+          tma_load_2d(a0 + ((uint32_t)term * nch + k) * kOpChunk, &tm[term], (int)(64 * k), arow, bar_a);
+      for (int u = 0; u < units; ++u) {
+        const int sl = u % kBSlots;
+        if (u >= kBSlots) {  // the slot's previous unit has been multiplied
+          mbar_wait(bar_f(u), (ps.free >> sl) & 1u);
+          ps.free ^= 1u << sl;
         }
+        const int c = u / 3, term = u - 3 * c;
+        mbar_arrive_expect_tx(bar_b(u), slot_bytes);
+        for (uint32_t k = 0; k < nch; ++k)
+          tma_load_2d(slot_addr(u) + k * (uint32_t)ncolw * 128, &tm[term + (ncolw == 128 ? 0 : 3)],
+                      (int)(64 * k), brow0 + c * ncolw, bar_b(u));
+      }
+      for (int u = max(units - kBSlots, 0); u < units; ++u) {  // the last releases
+        mbar_wait(bar_f(u), (ps.free >> (u % kBSlots)) & 1u);
+        ps.free ^= 1u << (u % kBSlots);
       }
     }
-    tc_fence_before();
-    __syncthreads();  // chunk c's accumulators are read
-  }
-  if (t == 0) {  // the releases of the last kBSlots units were not waited for yet
-    for (int u = max(units - kBSlots, 0); u < units; ++u) {
-      mbar_wait(bar_f(u), (ps.free >> (u % kBSlots)) & 1u);
-      ps.free ^= 1u << (u % kBSlots);
+  } else if (warp == 1) {
+    if (lane == 0) {  // product issuer
+      mbar_wait(smem_u32(&sm.bar_a), ps.a & 1u);
+      ps.a ^= 1u;
+      for (int c = 0; c < ncol; ++c) {
+        if (c >= 2) {  // the accumulators of chunk c - 2 have been read out
+          mbar_wait(bar_e(c), (ps.acc >> (c & 1)) & 1u);
+          ps.acc ^= 1u << (c & 1);
+        }
+        for (int tt = 0; tt < 3; ++tt) {
+          const int u = 3 * c + tt, sl = u % kBSlots;
+          mbar_wait(bar_b(u), (ps.b >> sl) & 1u);
+          ps.b ^= 1u << sl;
+          tc_fence_after();
+          score_mma_unit(P, dacc(c), a0, slot_addr(u), tt, ncolw, idesc);
+          mma_commit(bar_f(u));
+        }
+        mma_commit(bar_m(c));
+      }
+      for (int c = max(ncol - 2, 0); c < ncol; ++c) {  // the last read-outs
+        mbar_wait(bar_e(c), (ps.acc >> (c & 1)) & 1u);
+        ps.acc ^= 1u << (c & 1);
+      }
+    }
+  } else if (warp >= 4 && warp < 12) {
+    // warp w reads TMEM lane quarter w % 4 and column half (w - 4) / 4 in the
+    // 16 x 256-bit shape: four threads share a row, each holding two adjacent
+    // key blocks, so every store instruction writes eight whole 32-byte
+    // sectors of the score tiles.  The row maxima over j <= i are kept too.
+    const float sc_hi = P.tau[bh * 4 + 2], sc_lo = P.tau[bh * 4 + 3];
+    const int q4 = warp & 3, h = (warp - 4) >> 2;
+    const int gr = lane >> 2, cq = (lane & 3) * 2;
+    const int hw = ncolw / 2;
+    float mx[2][2][2];  // [lane half][row of the pair][band]
+#pragma unroll
+    for (int a = 0; a < 8; ++a) (&mx[0][0][0])[a] = -INFINITY;
+    for (int c = 0; c < ncol; ++c) {
+      mbar_wait(bar_m(c), (ps.mma >> (c & 1)) & 1u);
+      ps.mma ^= 1u << (c & 1);
+      tc_fence_after();
+#pragma unroll
+      for (int lh = 0; lh < 2; ++lh) {
+        for (int grp = 0; grp < hw; grp += 32) {
+          const int col0 = h * hw + grp;  // column in the chunk
+          const uint32_t taddr = dacc(c) + ((uint32_t)(q4 * 32 + lh * 16) << 16) + (uint32_t)col0;
+          uint32_t vh[16], vl[16];
+          tmem_ld_16x256b_x4(taddr, vh);
+          tmem_ld_16x256b_x4(taddr + (uint32_t)ncolw, vl);
+          tmem_wait_ld_dep16(vh);
+          tmem_wait_ld_dep16(vl);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int j = c * ncolw + col0 + 8 * k + cq;  // key block of the first value
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+              const int rl = q4 * 32 + lh * 16 + gr + 8 * rr;  // row in the item
+              const float h0 = __uint_as_float(vh[4 * k + 2 * rr]) * sc_hi;
+              const float h1 = __uint_as_float(vh[4 * k + 2 * rr + 1]) * sc_hi;
+              const float l0 = __uint_as_float(vl[4 * k + 2 * rr]) * sc_lo;
+              const float l1 = __uint_as_float(vl[4 * k + 2 * rr + 1]) * sc_lo;
+              float* dst = score_tile(P, bh, chunk, j >> 7) + rl * 128 + (j & 127);
+              *reinterpret_cast<float2*>(dst) = make_float2(h0, h1);
+              *reinterpret_cast<float2*>(dst + 128 * 128) = make_float2(l0, l1);
+              const int i = i0 + rl;
+              if (j <= i) {
+                mx[lh][rr][0] = fmaxf(mx[lh][rr][0], h0);
+                mx[lh][rr][1] = fmaxf(mx[lh][rr][1], l0);
+              }
+              if (j + 1 <= i) {
+                mx[lh][rr][0] = fmaxf(mx[lh][rr][0], h1);
+                mx[lh][rr][1] = fmaxf(mx[lh][rr][1], l1);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_e(c));
+    }
+    // the four threads of a row combine their maxima
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
+      float& v = (&mx[0][0][0])[a];
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+    }
+    if ((lane & 3) == 0) {
+#pragma unroll
+      for (int lh = 0; lh < 2; ++lh)
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const int rl = q4 * 32 + lh * 16 + gr + 8 * rr;
+          sm.rmax[h][0][rl] = mx[lh][rr][0];
+          sm.rmax[h][1][rl] = mx[lh][rr][1];
+        }
     }
   }
-  __syncthreads();  // this CTA's score rows are visible to all its threads
+  __syncthreads();  // score tiles and row maxima are visible to all threads
 
   // steps (5)-(7): one warp per row, both bands, union, whole mask row
   if (warp < P.topp_warps) {
@@ -800,49 +868,19 @@ __device__ void score_item(const EstParams& P, const CUtensorMap* tm, int g, int
     const int nbp = (P.nb + 7) & ~7;
     ToppScratch S;
     S.d = reinterpret_cast<uint32_t*>(wb);
-    S.L2 = reinterpret_cast<float*>(wb + (size_t)nbp * 4);
-    S.cand = reinterpret_cast<uint16_t*>(wb + (size_t)nbp * 8);
-    S.h = reinterpret_cast<unsigned long long*>(wb + (size_t)nbp * 10);
-    S.kb = reinterpret_cast<uint32_t*>(wb + (size_t)nbp * 10 + kTopPBins * 8);
-    uint32_t* bits = S.kb + P.W;
+    S.cand = reinterpret_cast<uint16_t*>(wb + (size_t)nbp * 4);
+    S.h = reinterpret_cast<unsigned long long*>(wb + (size_t)nbp * 6);
+    uint32_t* bits = reinterpret_cast<uint32_t*>(wb + (size_t)nbp * 6 + kTopPBins * 8);
     for (int i = i0 + warp; i <= max_i; i += P.topp_warps) {
       for (int w = lane; w < P.W; w += 32) bits[w] = 0u;
       __syncwarp();
-      // both bands' rows -> shared memory in one round trip (32 loads in flight
-      // per lane); the row is spread over the tiles (i / 128, cc), cc <= i / 128
-      const int n = i + 1;
-      const int cr = i >> 7, r = i & 127;
-      float* Lhi = reinterpret_cast<float*>(S.d);
-      float* dbg_hi = P.dbg_scores ? P.dbg_scores + (size_t)bh * 2 * tri + (size_t)i * (i + 1) / 2 : nullptr;
-      for (int j0 = 0; j0 < n; j0 += 512) {
-        float xh[16], xl[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int j = j0 + u * 32 + lane;
-          xh[u] = 0.f;
-          xl[u] = 0.f;
-          if (j < n) {
-            const float* src = score_tile(P, bh, cr, j >> 7) + r * 128 + (j & 127);
-            xh[u] = src[0];
-            xl[u] = src[128 * 128];
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int j = j0 + u * 32 + lane;
-          if (j < n) {
-            Lhi[j] = xh[u];
-            S.L2[j] = xl[u];
-            if (dbg_hi) {
-              dbg_hi[j] = xh[u];
-              dbg_hi[tri + j] = xl[u];
-            }
-          }
-        }
-      }
-      __syncwarp();
-      topp_band_row(Lhi, n, P.W, P.p, S, bits, lane);
-      topp_band_row(S.L2, n, P.W, P.p, S, bits, lane);
+      const int n = i + 1, r = i - i0;
+      const float* row = score_tile(P, bh, chunk, 0) + r * 128;
+      float* dbg = P.dbg_scores ? P.dbg_scores + (size_t)bh * 2 * tri + (size_t)i * (i + 1) / 2 : nullptr;
+#pragma unroll 1
+      for (int band = 0; band < 2; ++band)
+        topp_band_row(row + band * 128 * 128, fmaxf(sm.rmax[0][band][r], sm.rmax[1][band][r]), n, P.p, S, bits,
+                      dbg ? dbg + band * tri : nullptr, lane);
       uint32_t* dst = P.mask + ((size_t)bh * P.nb + i) * P.W;
       for (int w = lane; w < P.W; w += 32) dst[w] = bits[w];
       __syncwarp();
@@ -863,7 +901,7 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
   const int per_pair = P.pool_items + P.score_items;
   const int stages = P.pool_stages;
   uint32_t phases = 0u;  // parity to wait for next, one bit per ring stage
-  ScoreState ss = {0u, 0u, 0u, 0u};
+  ScoreState ss = {0u, 0u, 0u, 0u, 0u};
   if (threadIdx.x == 0) {
     for (int st = 0; st < stages; ++st) mbar_init(smem_u32(&psm.bars[st]), 1u);
     mbar_init(smem_u32(&psm.bar_a), 1u);
@@ -873,6 +911,8 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
     }
     mbar_init(smem_u32(&psm.bar_mma[0]), 1u);
     mbar_init(smem_u32(&psm.bar_mma[1]), 1u);
+    mbar_init(smem_u32(&psm.bar_acc[0]), 8u);  // one arrival per read-out warp
+    mbar_init(smem_u32(&psm.bar_acc[1]), 8u);
     fence_mbar_init();
     for (int m = 0; m < 6; ++m) tma_prefetch_desc(&tms.m[m]);
   }

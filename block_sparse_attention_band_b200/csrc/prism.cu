@@ -101,7 +101,6 @@ int validate(const prism_config* cfg, Plan* pl) {
   P.tau_lo = cfg->tau_lo;
   P.scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.0f / std::sqrt(128.0f);
   const size_t rows = (size_t)P.q_rows + P.kv_rows;
-  const size_t tri = (size_t)P.nb * (P.nb + 1) / 2;
   size_t off = 0;
   for (int term = 0; term < kTerms; ++term) {
     P.off_pool[term] = off;
@@ -134,6 +133,9 @@ int g_dev_state[kMaxDevices];  // 0 unknown, 1 ready, <0 error code
 
 // Shared memory of the persistent estimator: the score items' product tiles,
 // reused by the Top-P warps (each needs 8 bytes per key block + the bitset).
+// the widest product layout and the static scratch share one CTA's 227 KB
+static_assert(kGemmSmemBytes + sizeof(PoolSmem) + 256 <= 232448, "estimator shared memory over the per-CTA limit");
+
 struct EstLaunch {
   int topp_warps, topp_stride;
   size_t smem;
@@ -142,9 +144,8 @@ EstLaunch est_launch_shape(int nb) {
   const int W = (nb + 31) / 32;
   const int nbp = (nb + 7) & ~7;
   EstLaunch L;
-  // two bands' logits (the first reused for keys) + one u16 member list + 256
-  // 64-bit bins + two bit rows per warp
-  L.topp_stride = (int)align_up((size_t)nbp * 10 + 256 * 8 + (size_t)W * 8, 16);
+  // the rank keys + one u16 member list + 256 64-bit bins + one bit row per warp
+  L.topp_stride = (int)align_up((size_t)nbp * 6 + 256 * 8 + (size_t)W * 4, 16);
   // dynamic shared memory: the product tiles, or as many Top-P warps as fit
   // next to the static pool scratch (227 KB per CTA in all)
   const size_t max_dyn = 232448 - sizeof(PoolSmem) - 256;
