@@ -10,9 +10,12 @@
 //
 //   pool(0), pool(1), score(0), pool(2), score(1), ..., pool(n-1), score(n-2), score(n-1)
 //
-// pool items (HBM-bound) stream 128x128 bf16 tiles of Q and K once (bulk
-// copies into a ring of shared-memory stages, several tiles in flight) and write
-// the fp32 block means (steps 1-2) and per-block energy partials (step 3);
+// pool items (HBM-bound) stream 128x128 bf16 tiles of Q and K once (TMA into
+// a ring of shared-memory stages, several tiles in flight); the block sums are
+// products on the tensor cores (the tile, read transposed, times a column of
+// ones: D[dim] += sum over the block's tokens), so the CUDA cores only turn
+// the sums into the fp32 block means (steps 1-2) and per-block energy partials
+// (step 3);
 // the CTA that finishes the last pool item of a group also computes the
 // group's temperatures (steps 3-4) and publishes "group ready".  score items
 // wait for their group, compute both bands' pooled logits on the tensor cores
@@ -38,15 +41,17 @@ namespace prism {
 
 struct BandLayout {
   uint8_t src[192];  // pooled column c holds original dim src[c]; 255 = zero padding
+  uint8_t col[128];  // inverse: the pooled column of dim d; 255 = in neither band
   int s1, s2, s3;    // 16-aligned segment boundaries (see above)
   int dp;            // stored row length: a multiple of 64 (64, 128 or 192)
   int d_hi, d_lo;    // band sizes
 };
 
 constexpr int kEstThreads = 512;      // 16 warps, one CTA per SM
-constexpr int kPoolTilesPerItem = 8;  // 8 x 32 KB of Q or K per pool item
+constexpr int kPoolTilesPerItem = 16;  // 16 x 32 KB of Q or K per pool item
 constexpr uint32_t kTileBytes = 128 * 128 * 2;
-constexpr int kMaxPoolStages = 6;     // bulk-copy ring depth (32 KB stages)
+constexpr int kMaxPoolStages = 6;      // TMA ring depth (32 KB stages)
+constexpr int kPoolN = 16;             // N of a pooling product: block b sums into TMEM columns [16 b, 16 b + 16)
 constexpr int kScoreRows = 128;       // query blocks (of one head) per score item = MMA M
 constexpr uint32_t kOpChunk = 128 * 64 * 2;  // one 64-dim x 128-row bf16 operand chunk (SW128)
 constexpr int kTerms = 3;             // bf16 terms per pooled value
@@ -62,9 +67,10 @@ constexpr int kMaxGroupHeads = 64;    // Q heads per KV head supported by the ta
 constexpr float kLog2e = 1.4426950408889634f;
 
 // TMA descriptors of the three pooled bf16 terms [rows, dp]: boxes of 64 dims
-// x 128 rows (m[0..2]) and 64 dims x 64 rows (m[3..5])
+// x 128 rows (m[0..2]) and 64 dims x 64 rows (m[3..5]); Q and K as
+// [rows x tokens, 128] with boxes of 64 dims x 128 tokens (m[6], m[7])
 struct TermMaps {
-  CUtensorMap m[6];
+  CUtensorMap m[8];
 };
 
 struct EstParams {
@@ -84,7 +90,7 @@ struct EstParams {
   int pool_item_span;  // pool items per head row
   int topp_warps;
   int topp_stride;  // bytes of shared memory per Top-P warp
-  int pool_stages;  // bulk-copy ring depth (<= kMaxPoolStages)
+  int pool_stages;  // TMA ring depth (<= kMaxPoolStages)
   int smem_bytes;   // dynamic shared memory of the launch
   float p;
   int explicit_tau;
@@ -126,86 +132,45 @@ __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
 }
 
 // ---------------------------------------------------------------------------
-// steps (1)-(3a): mean of one 128 x 128 bf16 tile, band-ordered fp32 write,
-// energy partials.  Thread t holds 16-byte vectors of rows t/16 + 16 r at
-// dims 8 (t % 16) .. +7: each warp reads two full 256-byte rows.
+// static shared memory of the kernel
 // ---------------------------------------------------------------------------
 struct PoolSmem {
-  union {                   // pool and score items never overlap in a CTA
-    float red[16][128];     // pool item: row-group partial sums; temperatures: warp partials
-    float rmax[2][2][128];  // score item: row maxima per column half and band
+  // all-ones bf16 B operand of the pooling products: 16 rows x 128 bytes in
+  // the 128-byte-swizzled K-major layout (every element is one, so the
+  // swizzle does not matter)
+  __align__(1024) uint32_t ones[16 * 32];
+  union {                                   // pool and score items never overlap in a CTA
+    float rmax[2][2][128];                  // score item: row maxima per column half and band
+    float wred[16][3];                      // temperatures: per-warp partial sums
+    float bpart[kPoolTilesPerItem][4][3];  // pool item: per block and read-out warp: hi, lo, all
   };
-  float mean[128];
-  float wsum[6][3];
   float sums[kMaxGroupHeads + 1][3];
-  uint64_t bars[kMaxPoolStages];
+  uint64_t bars[kMaxPoolStages];       // pool ring: stage loaded
+  uint64_t bars_free[kMaxPoolStages];  // pool ring: stage multiplied
+  uint64_t bar_pool;                   // pool item: every block sum is in tensor memory
   uint64_t bar_a, bar_b[kBSlots], bar_free[kBSlots], bar_mma[2], bar_acc[2];  // score item: operands, slots,
                                                                             // products, accumulators read
   uint32_t tmem;
   int flag;
 };
 
-// Reduces one tile held in shared memory (128 rows x 256 bytes): thread t
-// sums the 16 rows 8k + t/64 of the bf16 pair in 32-bit word t % 64
-// (conflict-free), the 8 row groups are combined in a fixed order.  `refill`
-// runs once every thread has read the stage (it may overwrite it).
-template <class Refill>
-__device__ __forceinline__ void pool_tile(const uint32_t* tile, const EstParams& P, int hr, int blk, PoolSmem& sm,
-                                          Refill refill) {
-  const int t = threadIdx.x;
-  const int pw = t & 63, rg = t >> 6;
-  float a0 = 0.f, a1 = 0.f;
+// Transpose-reduction across a warp of N (16 or 32) values per lane: lane L
+// ends with the warp's sum of value L % N, in a fixed order (N - 1 shuffles,
+// plus one when N = 16).
+template <int N>
+__device__ __forceinline__ float warp_reduce_n(float (&v)[N], int lane) {
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const uint32_t w = tile[(rg + 8 * k) * 64 + pw];
-    a0 += bf16lo(w);
-    a1 += bf16hi(w);
-  }
-  sm.red[rg][2 * pw] = a0;
-  sm.red[rg][2 * pw + 1] = a1;
-  __syncthreads();
-  refill();
-  if (t < 128) {
-    float s = 0.f;
+  for (int o = N / 2; o > 0; o >>= 1) {
 #pragma unroll
-    for (int g = 0; g < 8; ++g) s += sm.red[g][t];
-    sm.mean[t] = s * (1.0f / 128.0f);
-  }
-  __syncthreads();
-  if (t < 192) {
-    float hi = 0.f, lo = 0.f, all = 0.f;
-    if (t < P.bl.dp) {
-      const int src = P.bl.src[t];
-      const float m = src < 128 ? sm.mean[src] : 0.f;
-      const __nv_bfloat16 th = __float2bfloat16_rn(m);
-      const float r1 = m - __bfloat162float(th);
-      const __nv_bfloat16 tm = __float2bfloat16_rn(r1);
-      const __nv_bfloat16 tl = __float2bfloat16_rn(r1 - __bfloat162float(tm));
-      const size_t o = ((size_t)hr * P.nb + blk) * P.bl.dp + t;
-      P.pool_t[0][o] = th;
-      P.pool_t[1][o] = tm;
-      P.pool_t[2][o] = tl;
-      const float sq = m * m;
-      hi = t < P.bl.s2 ? sq : 0.f;
-      lo = (t >= P.bl.s1 && t < P.bl.s3) ? sq : 0.f;
-    }
-    if (t < 128) all = sm.mean[t] * sm.mean[t];  // every dim, in or out of the bands
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      hi += __shfl_xor_sync(0xffffffffu, hi, o);
-      lo += __shfl_xor_sync(0xffffffffu, lo, o);
-      all += __shfl_xor_sync(0xffffffffu, all, o);
-    }
-    if ((t & 31) == 0) {
-      sm.wsum[t >> 5][0] = hi;
-      sm.wsum[t >> 5][1] = lo;
-      sm.wsum[t >> 5][2] = all;
+    for (int i = 0; i < o; ++i) {
+      const bool up = (lane & o) != 0;
+      const float send = up ? v[i] : v[i + o];
+      const float keep = up ? v[i + o] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
     }
   }
-  __syncthreads();
-  if (t < 3)
-    P.part[((size_t)hr * P.nb + blk) * 4 + t] =
-        ((sm.wsum[0][t] + sm.wsum[1][t]) + (sm.wsum[2][t] + sm.wsum[3][t])) + (sm.wsum[4][t] + sm.wsum[5][t]);
+  if (N == 16) v[0] += __shfl_xor_sync(0xffffffffu, v[0], 16);
+  return v[0];
 }
 
 // steps (3b)-(4): RMS of every pooled band of the group's heads over all
@@ -227,11 +192,11 @@ __device__ __forceinline__ void group_temperatures(const EstParams& P, int g, Po
     for (int e = 0; e < 3; ++e) s[e] = warp_sum(s[e]);
     if (lane == 0)
 #pragma unroll
-      for (int e = 0; e < 3; ++e) sm.red[warp][e] = s[e];
+      for (int e = 0; e < 3; ++e) sm.wred[warp][e] = s[e];
     __syncthreads();
     if (t < 3) {
       float a = 0.f;
-      for (int w = 0; w < kEstThreads / 32; ++w) a += sm.red[w][t];
+      for (int w = 0; w < kEstThreads / 32; ++w) a += sm.wred[w][t];
       sm.sums[slot][t] = a;
     }
     __syncthreads();
@@ -267,49 +232,117 @@ __device__ __forceinline__ void group_temperatures(const EstParams& P, int g, Po
 }
 
 // One pool item: kPoolTilesPerItem consecutive blocks of one head row of the
-// group (its Q heads, then its KV head), the next tile's loads in flight
-// while the current one is reduced.
-__device__ __forceinline__ void pool_item(const EstParams& P, int g, int y, PoolSmem& sm, unsigned char* ring, int stages,
-                          uint32_t& phases) {
+// group (its Q heads, then its KV head).  Warp roles: thread 0 streams the
+// tiles into the ring (TMA, two 64-dim boxes per tile, 128-byte swizzle);
+// thread 32 issues the block sums as tensor-core products: the tile is the A
+// operand read dim-major (M = 128 dims, K = 16 tokens a step), the all-ones
+// matrix the B operand (N = 16), block b accumulating into TMEM columns
+// [16 b, 16 b + 16), each stage released when its products are done; warps
+// 4-7 (thread = dim) read the sums, write the means in the band-segment layout
+// as three bf16 terms and the per-block energy partials.
+struct PoolState {  // per-role counters of ring stages and items, carried across items
+  uint32_t prod, cons, done;
+};
+
+__device__ __forceinline__ void pool_item(const EstParams& P, const CUtensorMap* tm, int g, int y, PoolSmem& sm,
+                                          unsigned char* ring, int stages, PoolState& st) {
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int slot = y / P.pool_item_span;
   const int blk0 = (y - slot * P.pool_item_span) * kPoolTilesPerItem;
-  const int blk1 = min(blk0 + kPoolTilesPerItem, P.nb);
+  const int nt = min(blk0 + kPoolTilesPerItem, P.nb) - blk0;
   const int bi = g / P.hkv, kv = g - bi * P.hkv;
-  int hr;
-  const __nv_bfloat16* base;
-  if (slot < P.G) {
-    hr = bi * P.hq + kv * P.G + slot;
-    base = P.q + (size_t)hr * P.nb * (128 * 128);
-  } else {
-    hr = P.q_rows + g;
-    base = P.k + (size_t)g * P.nb * (128 * 128);
-  }
-  // bulk-copy ring: up to `stages` tiles in flight, each stage refilled with
-  // the tile `stages` ahead as soon as every thread has read it
-  const int nt = blk1 - blk0;
-  const uint32_t ring0 = smem_u32(ring);
-  auto issue = [&](int tt) {
-    const int slot = tt % stages;
-    const uint32_t bar = smem_u32(&sm.bars[slot]);
-    mbar_arrive_expect_tx(bar, kTileBytes);
-    bulk_load(ring0 + slot * kTileBytes, base + (size_t)(blk0 + tt) * (128 * 128), kTileBytes, bar);
-  };
-  if (threadIdx.x == 0)
-    for (int tt = 0; tt < min(stages, nt); ++tt) issue(tt);
-  for (int tt = 0; tt < nt; ++tt) {
-    const int slot = tt % stages;
-    mbar_wait(smem_u32(&sm.bars[slot]), (phases >> slot) & 1u);  // a timeout is recorded on the device
-    phases ^= 1u << slot;
-    pool_tile(reinterpret_cast<const uint32_t*>(ring + (size_t)slot * kTileBytes), P, hr, blk0 + tt, sm, [&] {
-      if (threadIdx.x == 0 && tt + stages < nt) {
-        fence_proxy_async_smem();
-        issue(tt + stages);
+  const bool is_q = slot < P.G;
+  const int hr = is_q ? bi * P.hq + kv * P.G + slot : P.q_rows + g;
+  const uint32_t ring0 = (smem_u32(ring) + 1023u) & ~1023u;
+  if (t == 0) {  // producer
+    const CUtensorMap* map = &tm[is_q ? 6 : 7];
+    const int row0 = (is_q ? hr : g) * P.nb * 128 + blk0 * 128;  // first token row of the item
+    fence_proxy_async_smem();  // generic writes of the last item before the async ones
+    for (int tt = 0; tt < nt; ++tt, ++st.prod) {
+      const uint32_t s = st.prod % (uint32_t)stages;
+      if (st.prod >= (uint32_t)stages)  // the stage's previous tile has been multiplied
+        mbar_wait(smem_u32(&sm.bars_free[s]), (st.prod / (uint32_t)stages - 1u) & 1u);
+      const uint32_t dst = ring0 + s * kTileBytes, bar = smem_u32(&sm.bars[s]);
+      mbar_arrive_expect_tx(bar, kTileBytes);
+      tma_load_2d(dst, map, 0, row0 + tt * 128, bar);
+      tma_load_2d(dst + kTileBytes / 2, map, 64, row0 + tt * 128, bar);
+    }
+  } else if (t == 32) {  // product issuer
+    const uint32_t idesc = idesc_bf16_f32(128, kPoolN, 1, 0);
+    const uint64_t bdesc = smem_desc_sw128(smem_u32(sm.ones), 16, 1024);
+    for (int tt = 0; tt < nt; ++tt, ++st.cons) {
+      const uint32_t s = st.cons % (uint32_t)stages;
+      mbar_wait(smem_u32(&sm.bars[s]), (st.cons / (uint32_t)stages) & 1u);
+      tc_fence_after();
+      // A: 128 tokens x 128 dims, dims contiguous: MN-major, the two 64-dim
+      // halves 16 KB apart, 8-token groups 1 KB apart, 16 tokens = 2 KB a step
+      const uint64_t adesc = smem_desc_sw128(ring0 + s * kTileBytes, kTileBytes / 2, 1024);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        mma_bf16_ss(sm.tmem + (uint32_t)(tt * kPoolN), adesc + (uint64_t)((k * 2048) >> 4), bdesc, idesc,
+                    k > 0 ? 1u : 0u);
+      mma_commit(smem_u32(&sm.bars_free[s]));
+    }
+    mma_commit(smem_u32(&sm.bar_pool));
+  } else if (warp >= 4 && warp < 8) {  // read-out: thread = dim
+    const int q4 = warp & 3, d = q4 * 32 + lane;
+    mbar_wait(smem_u32(&sm.bar_pool), st.done & 1u);
+    ++st.done;
+    tc_fence_after();
+    uint32_t v[kPoolTilesPerItem];
+#pragma unroll
+    for (int b = 0; b < kPoolTilesPerItem; ++b)
+      v[b] = tmem_ld1(sm.tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(b * kPoolN));
+    tmem_wait_ld_dep16(v);
+    tc_fence_before();
+    const int c = P.bl.col[d];
+    const bool ih = c < P.bl.s2, il = c >= P.bl.s1 && c < P.bl.s3;  // c = 255: neither
+    const size_t o0 = ((size_t)hr * P.nb + blk0) * P.bl.dp;
+    float ehl[2 * kPoolTilesPerItem], ea[kPoolTilesPerItem];
+#pragma unroll
+    for (int b = 0; b < kPoolTilesPerItem; ++b) {
+      const float m = __uint_as_float(v[b]) * (1.0f / 128.0f);
+      const bool ok = b < nt;
+      if (ok && c != 255) {
+        const __nv_bfloat16 th = __float2bfloat16_rn(m);
+        const float r1 = m - __bfloat162float(th);
+        const __nv_bfloat16 tmid = __float2bfloat16_rn(r1);
+        const __nv_bfloat16 tl = __float2bfloat16_rn(r1 - __bfloat162float(tmid));
+        const size_t o = o0 + (size_t)b * P.bl.dp + c;
+        P.pool_t[0][o] = th;
+        P.pool_t[1][o] = tmid;
+        P.pool_t[2][o] = tl;
       }
-    });
+      const float x = ok ? m * m : 0.f;
+      ehl[b] = ih ? x : 0.f;
+      ehl[kPoolTilesPerItem + b] = il ? x : 0.f;
+      ea[b] = x;
+    }
+    // zero padding columns of the segment layout
+    for (int cc = d; cc < P.bl.dp; cc += 128)
+      if (P.bl.src[cc] == 255)
+        for (int b = 0; b < nt; ++b) {
+          const size_t o = o0 + (size_t)b * P.bl.dp + cc;
+          P.pool_t[0][o] = __float2bfloat16_rn(0.f);
+          P.pool_t[1][o] = __float2bfloat16_rn(0.f);
+          P.pool_t[2][o] = __float2bfloat16_rn(0.f);
+        }
+    // energy partials: lane L holds the warp's hi (L < 16) or lo sum of
+    // block L % 16, and its all-dims sum; the four warps add in a fixed order
+    const float rhl = warp_reduce_n<2 * kPoolTilesPerItem>(ehl, lane);
+    const float ra = warp_reduce_n<kPoolTilesPerItem>(ea, lane);
+    sm.bpart[lane & 15][q4][lane >> 4] = rhl;
+    if (lane < 16) sm.bpart[lane][q4][2] = ra;
+    named_barrier(1, 128);
+    if (d < nt * 3) {
+      const int b = d / 3, e = d - 3 * b;
+      P.part[((size_t)hr * P.nb + blk0 + b) * 4 + e] =
+          (sm.bpart[b][0][e] + sm.bpart[b][1][e]) + (sm.bpart[b][2][e] + sm.bpart[b][3][e]);
+    }
   }
   // publish: count the item; the CTA that completes the group computes tau
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (t == 0) {
     __threadfence();
     const uint32_t done = atomicAdd(&P.sync[1 + g], 1u);
     sm.flag = (done == (uint32_t)P.pool_items - 1u);
@@ -319,7 +352,7 @@ __device__ __forceinline__ void pool_item(const EstParams& P, int g, int y, Pool
   if (sm.flag) {
     group_temperatures(P, g, sm);
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (t == 0) {
       __threadfence();
       st_release_gpu(&P.sync[1 + P.n_groups + g], 1u);
     }
@@ -331,7 +364,7 @@ __device__ __forceinline__ void pool_item(const EstParams& P, int g, int y, Pool
 // ---------------------------------------------------------------------------
 // Shared-memory scratch of one Top-P warp.
 struct ToppScratch {
-  uint32_t* d;            // [n] the rank keys d_j (below)
+  uint32_t* d;            // [n] the row's logits, replaced by the rank keys d_j (below)
   uint16_t* cand;         // [n] members of the crossing bin
   unsigned long long* h;  // [256] bin masses
 };
@@ -398,9 +431,9 @@ __device__ __forceinline__ void bin_add(uint32_t* lo, uint32_t* hi, int b, uint3
   if (old > ~x) atomicAdd(&hi[b], 1u);
 }
 
-// Softmax (step 5) + Top-P (step 6) of one band row of n scaled logits; ORs
-// the kept blocks into bits[].  The row lives in the item's score tiles: key
-// block j at row[(j / 128) * kTilePair + j % 128]; rmax is its maximum.
+// Softmax (step 5) + Top-P (step 6) of one band row of n scaled logits, held
+// in shared memory at S.d (as floats); ORs the kept blocks into bits[].  rmax
+// is the row's maximum.
 //
 // e_j = 2^((L_j - max) log2 e); blocks ranked by (-e_j, j) == (d_j, j) with
 // the exact order-reversing key d_j.  Radix selection on the keys: bins of 16
@@ -415,12 +448,13 @@ __device__ __forceinline__ void bin_add(uint32_t* lo, uint32_t* hi, int b, uint3
 constexpr size_t kTilePair = 2 * 128 * 128;  // floats per score tile pair (both bands)
 constexpr int kSegPerLane = 16;              // logits per lane per pass (512 per warp)
 
-__device__ __forceinline__ void topp_band_row(const float* row, float rmax, int n, float p, const ToppScratch& S,
-                                              uint32_t* bits, float* dbg, int lane) {
+__device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const ToppScratch& S, uint32_t* bits,
+                                              float* dbg, int lane) {
   const unsigned lt = (1u << lane) - 1u;
   constexpr int kSeg = 32 * kSegPerLane;
+  const float* row = reinterpret_cast<const float*>(S.d);
   if (dbg)
-    for (int j = lane; j < n; j += 32) dbg[j] = row[(size_t)(j >> 7) * kTilePair + (j & 127)];
+    for (int j = lane; j < n; j += 32) dbg[j] = row[j];
   const int nw = (n + 31) >> 5;
   if (p >= 1.0f) {  // every causal block is kept
     for (int w = lane; w < nw; w += 32) {
@@ -438,13 +472,14 @@ __device__ __forceinline__ void topp_band_row(const float* row, float rmax, int 
     hhi[b] = 0u;
   }
   __syncwarp();
-  // e_j, keys, exact bin masses: a batch of loads, then their arithmetic
+  // e_j, keys (in place of the logits), exact bin masses: a batch of loads,
+  // then their arithmetic
   for (int j0 = 0; j0 < n; j0 += kSeg) {
     float x[kSegPerLane];
 #pragma unroll
     for (int u = 0; u < kSegPerLane; ++u) {
       const int j = j0 + u * 32 + lane;
-      x[u] = j < n ? row[(size_t)(j >> 7) * kTilePair + (j & 127)] : 0.f;
+      x[u] = j < n ? row[j] : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < kSegPerLane; ++u) {
@@ -862,29 +897,52 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
   }
   __syncthreads();  // score tiles and row maxima are visible to all threads
 
-  // steps (5)-(7): one warp per row, both bands, union, whole mask row
+  // steps (5)-(7): one warp per row, both bands, union, whole mask row.  A
+  // warp's tasks are (row, band) pairs; the logits of the next task stream
+  // into the other half of a double buffer (cp.async) while the current one
+  // is ranked.
   if (warp < P.topp_warps) {
     unsigned char* wb = smem + (size_t)warp * P.topp_stride;
     const int nbp = (P.nb + 7) & ~7;
     ToppScratch S;
-    S.d = reinterpret_cast<uint32_t*>(wb);
-    S.cand = reinterpret_cast<uint16_t*>(wb + (size_t)nbp * 4);
-    S.h = reinterpret_cast<unsigned long long*>(wb + (size_t)nbp * 6);
-    uint32_t* bits = reinterpret_cast<uint32_t*>(wb + (size_t)nbp * 6 + kTopPBins * 8);
-    for (int i = i0 + warp; i <= max_i; i += P.topp_warps) {
-      for (int w = lane; w < P.W; w += 32) bits[w] = 0u;
+    S.cand = reinterpret_cast<uint16_t*>(wb + (size_t)nbp * 8);
+    S.h = reinterpret_cast<unsigned long long*>(wb + (size_t)nbp * 10);
+    uint32_t* bits = reinterpret_cast<uint32_t*>(wb + (size_t)nbp * 10 + kTopPBins * 8);
+    const int nrows = max_i - i0 - warp >= 0 ? (max_i - i0 - warp) / P.topp_warps + 1 : 0;
+    const int ntasks = 2 * nrows;
+    const float* tiles = score_tile(P, bh, chunk, 0);
+    auto fetch = [&](int task) {  // logits of task -> buffer (task & 1), 16-byte pieces
+      const int i = i0 + warp + (task >> 1) * P.topp_warps;
+      const float* row = tiles + (i - i0) * 128 + (task & 1) * 128 * 128;
+      const uint32_t dst = smem_u32(wb) + (uint32_t)(task & 1) * (uint32_t)nbp * 4u;
+      for (int c = lane; c * 4 <= i; c += 32)
+        cp_async16(dst + (uint32_t)c * 16u, row + (size_t)((c * 4) >> 7) * kTilePair + ((c * 4) & 127));
+      cp_async_commit();
+    };
+    if (ntasks > 0) fetch(0);
+    for (int task = 0; task < ntasks; ++task) {
+      if (task + 1 < ntasks)
+        fetch(task + 1);
+      else
+        cp_async_commit();  // an empty group keeps the count of groups in flight uniform
+      cp_async_wait<1>();   // this task's pieces have landed
       __syncwarp();
-      const int n = i + 1, r = i - i0;
-      const float* row = score_tile(P, bh, chunk, 0) + r * 128;
-      float* dbg = P.dbg_scores ? P.dbg_scores + (size_t)bh * 2 * tri + (size_t)i * (i + 1) / 2 : nullptr;
-#pragma unroll 1
-      for (int band = 0; band < 2; ++band)
-        topp_band_row(row + band * 128 * 128, fmaxf(sm.rmax[0][band][r], sm.rmax[1][band][r]), n, P.p, S, bits,
-                      dbg ? dbg + band * tri : nullptr, lane);
-      uint32_t* dst = P.mask + ((size_t)bh * P.nb + i) * P.W;
-      for (int w = lane; w < P.W; w += 32) dst[w] = bits[w];
-      __syncwarp();
+      const int i = i0 + warp + (task >> 1) * P.topp_warps, band = task & 1, r = i - i0;
+      if (band == 0) {
+        for (int w = lane; w < P.W; w += 32) bits[w] = 0u;
+        __syncwarp();
+      }
+      S.d = reinterpret_cast<uint32_t*>(wb + (size_t)(task & 1) * nbp * 4);
+      float* dbg = P.dbg_scores ? P.dbg_scores + (size_t)bh * 2 * tri + (size_t)band * tri + (size_t)i * (i + 1) / 2
+                                : nullptr;
+      topp_band_row(fmaxf(sm.rmax[0][band][r], sm.rmax[1][band][r]), i + 1, P.p, S, bits, dbg, lane);
+      if (band == 1) {
+        uint32_t* dst = P.mask + ((size_t)bh * P.nb + i) * P.W;
+        for (int w = lane; w < P.W; w += 32) dst[w] = bits[w];
+        __syncwarp();
+      }
     }
+    cp_async_wait<0>();
   }
   __syncthreads();  // shared memory is reused by the next item
 }
@@ -900,10 +958,16 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
   __shared__ int s_ok;
   const int per_pair = P.pool_items + P.score_items;
   const int stages = P.pool_stages;
-  uint32_t phases = 0u;  // parity to wait for next, one bit per ring stage
+  PoolState pst = {0u, 0u, 0u};
   ScoreState ss = {0u, 0u, 0u, 0u, 0u};
+  for (int i = threadIdx.x; i < 16 * 32; i += kEstThreads) psm.ones[i] = 0x3F803F80u;  // bf16 1.0 pairs
+  fence_proxy_async_smem();  // read by the tensor cores
   if (threadIdx.x == 0) {
-    for (int st = 0; st < stages; ++st) mbar_init(smem_u32(&psm.bars[st]), 1u);
+    for (int st = 0; st < stages; ++st) {
+      mbar_init(smem_u32(&psm.bars[st]), 1u);
+      mbar_init(smem_u32(&psm.bars_free[st]), 1u);
+    }
+    mbar_init(smem_u32(&psm.bar_pool), 1u);
     mbar_init(smem_u32(&psm.bar_a), 1u);
     for (int sl = 0; sl < kBSlots; ++sl) {
       mbar_init(smem_u32(&psm.bar_b[sl]), 1u);
@@ -914,9 +978,9 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
     mbar_init(smem_u32(&psm.bar_acc[0]), 8u);  // one arrival per read-out warp
     mbar_init(smem_u32(&psm.bar_acc[1]), 8u);
     fence_mbar_init();
-    for (int m = 0; m < 6; ++m) tma_prefetch_desc(&tms.m[m]);
+    for (int m = 0; m < 8; ++m) tma_prefetch_desc(&tms.m[m]);
   }
-  if ((threadIdx.x >> 5) == 0) {  // the score items' accumulators: 2 chunks x (hi, lo) x 128 columns
+  if ((threadIdx.x >> 5) == 0) {  // score items: 2 chunks x (hi, lo) x 128 columns; pool items: 16 x 16
     tmem_alloc(smem_u32(&psm.tmem), 512);
     tmem_relinquish();
   }
@@ -952,7 +1016,7 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
       }
     }
     if (is_pool) {
-      pool_item(P, g, y, psm, est_smem, stages, phases);
+      pool_item(P, tms.m, g, y, psm, est_smem, stages, pst);
       continue;
     }
     // wait until the group's pooling and temperatures are published

@@ -80,10 +80,14 @@ int validate(const prism_config* cfg, Plan* pl) {
   // pooled row layout: [high only | both | low only], each segment zero-padded
   // to a multiple of 16 columns (one MMA K step), total padded to 64
   std::memset(P.bl.src, 0xff, sizeof(P.bl.src));
+  std::memset(P.bl.col, 0xff, sizeof(P.bl.col));
   int c = 0;
   auto segment = [&](bool want_hi, bool want_lo) {
     for (int d = 0; d < 128; ++d)
-      if (in_hi[d] == want_hi && in_lo[d] == want_lo) P.bl.src[c++] = (uint8_t)d;
+      if (in_hi[d] == want_hi && in_lo[d] == want_lo) {
+        P.bl.col[d] = (uint8_t)c;
+        P.bl.src[c++] = (uint8_t)d;
+      }
     c = (c + 15) & ~15;
   };
   segment(true, false);
@@ -144,8 +148,9 @@ EstLaunch est_launch_shape(int nb) {
   const int W = (nb + 31) / 32;
   const int nbp = (nb + 7) & ~7;
   EstLaunch L;
-  // the rank keys + one u16 member list + 256 64-bit bins + one bit row per warp
-  L.topp_stride = (int)align_up((size_t)nbp * 6 + 256 * 8 + (size_t)W * 4, 16);
+  // two logit rows (double buffer; keys replace the logits in place) + one u16
+  // member list + 256 64-bit bins + one bit row per warp
+  L.topp_stride = (int)align_up((size_t)nbp * 10 + 256 * 8 + (size_t)W * 4, 16);
   // dynamic shared memory: the product tiles, or as many Top-P warps as fit
   // next to the static pool scratch (227 KB per CTA in all)
   const size_t max_dyn = 232448 - sizeof(PoolSmem) - 256;
@@ -257,7 +262,7 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   const EstLaunch L = est_launch_shape(P.nb);
   E.topp_warps = L.topp_warps;
   E.topp_stride = L.topp_stride;
-  E.pool_stages = (int)std::min<size_t>(kMaxPoolStages, L.smem / kTileBytes);
+  E.pool_stages = (int)std::min<size_t>(kMaxPoolStages, (L.smem - 1024) / kTileBytes);  // 1 KB-aligned ring
   E.smem_bytes = (int)L.smem;
   E.p = P.p_eff;
   E.explicit_tau = P.explicit_tau;
@@ -279,6 +284,10 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
     if (make_map(&tms.m[term], E.pool_t[term], prow, P.bl.dp, 128) != PRISM_OK ||
         make_map(&tms.m[3 + term], E.pool_t[term], prow, P.bl.dp, 64) != PRISM_OK)
       return PRISM_ERR_CUDA;
+  // the pool items' tiles: Q and K as [rows x tokens, 128], boxes of 64 dims x 128 tokens
+  if (make_map(&tms.m[6], q, (size_t)P.q_rows * P.n) != PRISM_OK ||
+      make_map(&tms.m[7], k, (size_t)P.kv_rows * P.n) != PRISM_OK)
+    return PRISM_ERR_CUDA;
   // the queue head and the per-group counters start at zero on every call
   if (cudaMemsetAsync(E.sync, 0, P.sync_bytes, st) != cudaSuccess) return PRISM_ERR_CUDA;
   estimator_kernel<<<(unsigned)grid, kEstThreads, L.smem, st>>>(E, tms);
