@@ -5,7 +5,7 @@ in the CUDA kernels of ``libprism_b200.so``; PyTorch provides device memory and
 streams.  The functions carry the C names; each raises ``PrismError`` when the
 library returns a non-zero status.  There is no CPU fallback: importing this
 package fails if the library has not been built
-(``python -m block_sparse_attention_band_b200.build``).
+(``python block_sparse_attention_band_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -40,7 +40,7 @@ def lib_path() -> str:
 if not os.path.exists(_LIB_PATH):
     raise ImportError(
         f"{_LIB_PATH} is missing: build the CUDA library first "
-        "(python -m block_sparse_attention_band_b200.build); there is no CPU fallback")
+        "(python block_sparse_attention_band_b200/build.py); there is no CPU fallback")
 
 lib = ctypes.CDLL(_LIB_PATH)
 

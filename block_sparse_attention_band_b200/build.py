@@ -1,6 +1,7 @@
 """Builds the in-tree CUDA library libprism_b200.so for sm_100a with nvcc.
 
-Usage: python -m block_sparse_attention_band_b200.build [--force]
+Usage: python block_sparse_attention_band_b200/build.py [--force] [-v]
+(run by path: importing the package requires the library this script builds)
 """
 from __future__ import annotations
 

@@ -7,11 +7,7 @@ import subprocess
 
 import pytest
 
-from block_sparse_attention_band_b200 import build as _build
-
-_build.build()
-
-import block_sparse_attention_band_b200 as pb  # noqa: E402
+import block_sparse_attention_band_b200 as pb  # noqa: E402  (built by conftest)
 from tests import gen  # noqa: E402
 
 HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "prism.h")
