@@ -423,12 +423,20 @@ __device__ __forceinline__ int topp_exact32(const ToppScratch& S, int cnt, unsig
   return (int)(uint32_t)__shfl_sync(0xffffffffu, key, __ffs(hit) - 1);
 }
 
-// 64-bit bin mass kept as two 32-bit words: the low word's atomic add returns
-// the old value, and an add that wraps it carries one into the high word, so
-// the final sum is exact and independent of the order of the adds.
+// A bin's 64-bit mass is kept as two 32-bit sums, of the low 16 bits and of
+// the high 16 bits of each added value, so a bin mass is hi * 2^16 + lo.
+// Neither sum can wrap (at most 2^14 values of < 2^16 each), so the adds need
+// no carry and no result: fire-and-forget shared-memory reductions, exact and
+// independent of the order of the adds.
+// (No "memory" clobber: the bins are read only after a __syncwarp, and
+// leaving the compiler free to move other loads across the reductions keeps
+// several blocks' arithmetic in flight.)
 __device__ __forceinline__ void bin_add(uint32_t* lo, uint32_t* hi, int b, uint32_t x) {
-  const uint32_t old = atomicAdd(&lo[b], x);
-  if (old > ~x) atomicAdd(&hi[b], 1u);
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(smem_u32(lo + b)), "r"(x & 0xFFFFu));
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(smem_u32(hi + b)), "r"(x >> 16));
+}
+__device__ __forceinline__ unsigned long long bin_mass(const uint32_t* lo, const uint32_t* hi, int b) {
+  return ((unsigned long long)hi[b] << 16) + lo[b];
 }
 
 // Softmax (step 5) + Top-P (step 6) of one band row of n scaled logits, held
@@ -446,12 +454,10 @@ __device__ __forceinline__ void bin_add(uint32_t* lo, uint32_t* hi, int b, uint3
 // every member sums the masses of the members ahead of it directly, else the
 // bin is refined on the lower key bits the same way.
 constexpr size_t kTilePair = 2 * 128 * 128;  // floats per score tile pair (both bands)
-constexpr int kSegPerLane = 16;              // logits per lane per pass (512 per warp)
 
 __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const ToppScratch& S, uint32_t* bits,
                                               float* dbg, int lane) {
   const unsigned lt = (1u << lane) - 1u;
-  constexpr int kSeg = 32 * kSegPerLane;
   const float* row = reinterpret_cast<const float*>(S.d);
   if (dbg)
     for (int j = lane; j < n; j += 32) dbg[j] = row[j];
@@ -467,25 +473,24 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
   const float m = rmax * kLog2e;
   uint32_t* hlo = reinterpret_cast<uint32_t*>(S.h);
   uint32_t* hhi = hlo + kTopPBins;
-  for (int b = lane; b < kTopPBins; b += 32) {
-    hlo[b] = 0u;
-    hhi[b] = 0u;
-  }
+  // the 2 KB of bins zeroed with 16-byte stores
+  for (int q = lane; q < 2 * kTopPBins / 4; q += 32) reinterpret_cast<uint4*>(hlo)[q] = make_uint4(0u, 0u, 0u, 0u);
   __syncwarp();
-  // e_j, keys (in place of the logits), exact bin masses: a batch of loads,
-  // then their arithmetic
-  for (int j0 = 0; j0 < n; j0 += kSeg) {
-    float x[kSegPerLane];
+  // e_j, keys (in place of the logits), exact bin masses; only the
+  // ceil(n / 32) slots the row has are visited
+  const int ns = (n + 31) >> 5;
+  for (int u0 = 0; u0 < ns; u0 += 4) {  // four slots' loads first, then their arithmetic
+    float x[4];
 #pragma unroll
-    for (int u = 0; u < kSegPerLane; ++u) {
-      const int j = j0 + u * 32 + lane;
-      x[u] = j < n ? row[j] : 0.f;
+    for (int v = 0; v < 4; ++v) {
+      const int j = (u0 + v) * 32 + lane;
+      x[v] = j < n ? row[j] : 0.f;
     }
 #pragma unroll
-    for (int u = 0; u < kSegPerLane; ++u) {
-      const int j = j0 + u * 32 + lane;
+    for (int v = 0; v < 4; ++v) {
+      const int j = (u0 + v) * 32 + lane;
       if (j < n) {
-        const float e = fast_exp2(fmaf(x[u], kLog2e, -m));
+        const float e = fast_exp2(fmaf(x[v], kLog2e, -m));
         const uint32_t d = rank_key(e);
         S.d[j] = d;
         bin_add(hlo, hhi, (int)min(d >> 19, (uint32_t)(kTopPBins - 1)), fixmass(e));
@@ -494,10 +499,16 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
   }
   __syncwarp();
   unsigned long long hv[8], tot = 0ull;
+  {
+    const uint4 l0 = reinterpret_cast<const uint4*>(hlo)[2 * lane], l1 = reinterpret_cast<const uint4*>(hlo)[2 * lane + 1];
+    const uint4 h0 = reinterpret_cast<const uint4*>(hhi)[2 * lane], h1 = reinterpret_cast<const uint4*>(hhi)[2 * lane + 1];
+    const uint32_t lw[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+    const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    hv[u] = ((unsigned long long)hhi[lane * 8 + u] << 32) | hlo[lane * 8 + u];
-    tot += hv[u];
+    for (int u = 0; u < 8; ++u) {
+      hv[u] = ((unsigned long long)hw[u] << 16) + lw[u];
+      tot += hv[u];
+    }
   }
   unsigned long long incl = warp_scan_u64(tot, lane);
   const unsigned long long Z = __shfl_sync(0xffffffffu, incl, 31);
@@ -525,48 +536,44 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
   // one pass: keep the earlier bins, list the crossing bin's members; lane u
   // collects mask word u of each batch
   int cnt = 0;
-  for (int j0 = 0; j0 < n; j0 += kSeg) {
-    uint32_t dv[kSegPerLane];
-#pragma unroll
-    for (int u = 0; u < kSegPerLane; ++u) {
-      const int j = j0 + u * 32 + lane;
-      dv[u] = j < n ? S.d[j] : 0u;
-    }
+  for (int u0 = 0; u0 < ns; u0 += 32) {
+    const int u1 = min(u0 + 32, ns);
     uint32_t myw = 0u;
-#pragma unroll
-    for (int u = 0; u < kSegPerLane; ++u) {
-      const int j = j0 + u * 32 + lane;
-      const int b = (int)min(dv[u] >> 19, (uint32_t)(kTopPBins - 1));
+#pragma unroll 4
+    for (int u = u0; u < u1; ++u) {
+      const int j = u * 32 + lane;
       const bool valid = j < n;
-      const unsigned mb = __ballot_sync(0xffffffffu, valid && b < xb);
-      const bool in = valid && b == xb;
+      const int b = valid ? (int)min(S.d[j] >> 19, (uint32_t)(kTopPBins - 1)) : kTopPBins;
+      const unsigned mb = __ballot_sync(0xffffffffu, b < xb);
+      const bool in = b == xb;
       const unsigned mi = __ballot_sync(0xffffffffu, in);
       if (in) S.cand[cnt + __popc(mi & lt)] = (uint16_t)j;
       cnt += __popc(mi);
-      if (lane == u) myw = mb;
+      if (lane == u - u0) myw = mb;
     }
-    const int w = (j0 >> 5) + lane;
-    if (lane < kSegPerLane && w < nw) bits[w] |= myw;
+    if (lane < u1 - u0) bits[u0 + lane] |= myw;  // slot u holds mask word u
   }
   __syncwarp();
   const unsigned long long lim = target > 0ull ? target : 1ull;
   if (cnt <= 32) {
-    // member x is kept iff base + (mass of the members ranked ahead of it) < lim
-    uint32_t dx = 0xffffffffu, mx = 0u;
-    int jx = 0x7fffffff;
+    // member x is kept iff base + (mass of the members ranked ahead of it) <
+    // lim; the members are listed (key, j, mass) over the no longer needed
+    // bins and read back with broadcast loads
+    uint4* memb = reinterpret_cast<uint4*>(S.h);
+    uint4 me = make_uint4(0xffffffffu, 0x7fffffffu, 0u, 0u);
     if (lane < cnt) {
-      jx = S.cand[lane];
-      dx = S.d[jx];
-      mx = fixmass(key_value(dx));
+      const uint32_t jx = S.cand[lane], dx = S.d[jx];
+      me = make_uint4(dx, jx, fixmass(key_value(dx)), 0u);
+      memb[lane] = me;
     }
+    __syncwarp();
     unsigned long long ahead = base;
+#pragma unroll 4
     for (int y = 0; y < cnt; ++y) {
-      const uint32_t dy = __shfl_sync(0xffffffffu, dx, y);
-      const int jy = __shfl_sync(0xffffffffu, jx, y);
-      const uint32_t my = __shfl_sync(0xffffffffu, mx, y);
-      if (dy < dx || (dy == dx && jy < jx)) ahead += my;
+      const uint4 o = memb[y];
+      if (o.x < me.x || (o.x == me.x && o.y < me.y)) ahead += o.z;
     }
-    if (lane < cnt && ahead < lim) atomicOr(&bits[jx >> 5], 1u << (jx & 31));
+    if (lane < cnt && ahead < lim) atomicOr(&bits[me.y >> 5], 1u << (me.y & 31));
     __syncwarp();
     return;
   }
@@ -594,7 +601,7 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
     unsigned long long h2[8], t2 = 0ull;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      h2[u] = ((unsigned long long)hhi[lane * 8 + u] << 32) | hlo[lane * 8 + u];
+      h2[u] = bin_mass(hlo, hhi, lane * 8 + u);
       t2 += h2[u];
     }
     const unsigned long long inc2 = warp_scan_u64(t2, lane);
@@ -928,16 +935,18 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
       cp_async_wait<1>();   // this task's pieces have landed
       __syncwarp();
       const int i = i0 + warp + (task >> 1) * P.topp_warps, band = task & 1, r = i - i0;
+      const int n = i + 1;
+      const float rmax = fmaxf(sm.rmax[0][band][r], sm.rmax[1][band][r]);
+      S.d = reinterpret_cast<uint32_t*>(wb + (size_t)(task & 1) * nbp * 4);
+      float* dbg = P.dbg_scores ? P.dbg_scores + (size_t)bh * 2 * tri + (size_t)band * tri + (size_t)i * (i + 1) / 2
+                                : nullptr;
+      uint32_t* dst = P.mask + ((size_t)bh * P.nb + i) * P.W;
       if (band == 0) {
         for (int w = lane; w < P.W; w += 32) bits[w] = 0u;
         __syncwarp();
       }
-      S.d = reinterpret_cast<uint32_t*>(wb + (size_t)(task & 1) * nbp * 4);
-      float* dbg = P.dbg_scores ? P.dbg_scores + (size_t)bh * 2 * tri + (size_t)band * tri + (size_t)i * (i + 1) / 2
-                                : nullptr;
-      topp_band_row(fmaxf(sm.rmax[0][band][r], sm.rmax[1][band][r]), i + 1, P.p, S, bits, dbg, lane);
+      topp_band_row(rmax, n, P.p, S, bits, dbg, lane);
       if (band == 1) {
-        uint32_t* dst = P.mask + ((size_t)bh * P.nb + i) * P.W;
         for (int w = lane; w < P.W; w += 32) dst[w] = bits[w];
         __syncwarp();
       }
