@@ -53,6 +53,7 @@ constexpr uint32_t kTileBytes = 128 * 128 * 2;
 constexpr int kMaxPoolStages = 6;      // TMA ring depth (32 KB stages)
 constexpr int kPoolN = 16;             // N of a pooling product: block b sums into TMEM columns [16 b, 16 b + 16)
 constexpr int kScoreRows = 128;       // query blocks (of one head) per score item = MMA M
+constexpr int kToppRows = 32;         // query blocks (of one head) per Top-P item
 constexpr uint32_t kOpChunk = 128 * 64 * 2;  // one 64-dim x 128-row bf16 operand chunk (SW128)
 constexpr int kTerms = 3;             // bf16 terms per pooled value
 // product operands: A (3 terms x dp/64 chunks of 128 rows) once, B one term at
@@ -83,10 +84,13 @@ struct EstParams {
   float* dbg_scores;  // optional copy in packed lower-triangular rows [q_rows, 2, nb(nb+1)/2]
   uint32_t* mask;
   float* dbg_tau;
-  uint32_t* sync;  // [0] queue head, [1 + g] pool items done, [1 + n_groups + g] group ready
+  float* rmax;     // [q_rows, nb, 2] scaled band logits' row maxima over j <= i
+  uint32_t* sync;  // [0] queue head, [1 + g] pool items done, [1 + n_groups + g] group ready,
+                   // [1 + 2 n_groups + bh * nchunk + c] score chunk c of (batch, Q head) bh written
   int hq, hkv, G, nb, W, q_rows, n_groups;
   int pool_items;      // per group
   int score_items;     // per group
+  int topp_items;      // per group
   int pool_item_span;  // pool items per head row
   int topp_warps;
   int topp_stride;  // bytes of shared memory per Top-P warp
@@ -242,10 +246,114 @@ __device__ __forceinline__ void group_temperatures(const EstParams& P, int g, Po
 // as three bf16 terms and the per-block energy partials.
 struct PoolState {  // per-role counters of ring stages and items, carried across items
   uint32_t prod, cons, done;
+  int pre;  // producer: tiles of the next pool item already streamed into the ring
 };
 
-__device__ __forceinline__ void pool_item(const EstParams& P, const CUtensorMap* tm, int g, int y, PoolSmem& sm,
-                                          unsigned char* ring, int stages, PoolState& st) {
+// Queue order, with PI / SI / TI pool / score / Top-P items per group g of n:
+//   pool(0) | pool(1) score(0) | pool(2) score(1) topp(0) | ... |
+//   pool(n-1) score(n-2) topp(n-3) | score(n-1) topp(n-2) | topp(n-1)
+// so scoring of group g overlaps pooling of group g + 1, and the Top-P items of
+// group g come one group after its score items.  Returns the item kind (0
+// pool, 1 score, 2 Top-P, -1 past the end) and sets (g, y), y the index within
+// the group's items of that kind.
+enum : int { kItemPool = 0, kItemScore = 1, kItemTopp = 2, kItemNone = -1 };
+__device__ __forceinline__ int decode_item(const EstParams& P, int x, int& g, int& y) {
+  const int n = P.n_groups, PI = P.pool_items, SI = P.score_items, TI = P.topp_items;
+  if (x < PI) {
+    g = 0;
+    y = x;
+    return kItemPool;
+  }
+  x -= PI;
+  const int first = (n > 1 ? PI : 0) + SI;  // pair 0: pool(1) score(0)
+  if (x < first) {
+    if (n > 1 && x < PI) {
+      g = 1;
+      y = x;
+      return kItemPool;
+    }
+    g = 0;
+    y = x - (n > 1 ? PI : 0);
+    return kItemScore;
+  }
+  x -= first;
+  const int L = PI + SI + TI, M = max(n - 2, 0);  // pairs 1 .. n-2: pool(p+1) score(p) topp(p-1)
+  if (x < M * L) {
+    const int p = 1 + x / L, rem = x - (p - 1) * L;
+    if (rem < PI) {
+      g = p + 1;
+      y = rem;
+      return kItemPool;
+    }
+    if (rem < PI + SI) {
+      g = p;
+      y = rem - PI;
+      return kItemScore;
+    }
+    g = p - 1;
+    y = rem - PI - SI;
+    return kItemTopp;
+  }
+  x -= M * L;
+  if (n > 1) {  // pair n-1: score(n-1) topp(n-2)
+    if (x < SI) {
+      g = n - 1;
+      y = x;
+      return kItemScore;
+    }
+    if (x < SI + TI) {
+      g = n - 2;
+      y = x - SI;
+      return kItemTopp;
+    }
+    x -= SI + TI;
+  }
+  if (x < TI) {
+    g = n - 1;
+    y = x;
+    return kItemTopp;
+  }
+  return kItemNone;
+}
+
+// The tiles of pool item (g, y): tensor map, first token row, tile count.
+struct PoolCoords {
+  const CUtensorMap* map;
+  int row0, nt;
+};
+__device__ __forceinline__ PoolCoords pool_coords(const EstParams& P, const CUtensorMap* tm, int g, int y) {
+  const int slot = y / P.pool_item_span;
+  const int blk0 = (y - slot * P.pool_item_span) * kPoolTilesPerItem;
+  const int bi = g / P.hkv, kv = g - bi * P.hkv;
+  const bool is_q = slot < P.G;
+  PoolCoords c;
+  c.map = &tm[is_q ? 6 : 7];
+  c.row0 = (is_q ? bi * P.hq + kv * P.G + slot : g) * P.nb * 128 + blk0 * 128;
+  c.nt = min(blk0 + kPoolTilesPerItem, P.nb) - blk0;
+  return c;
+}
+
+// Producer: streams tiles [t0, t1) of an item into the ring.
+__device__ __forceinline__ void pool_stream(const PoolCoords& c, int t0, int t1, PoolSmem& sm, uint32_t ring0,
+                                            int stages, PoolState& st) {
+  for (int tt = t0; tt < t1; ++tt, ++st.prod) {
+    const uint32_t s = st.prod % (uint32_t)stages;
+    if (st.prod >= (uint32_t)stages)  // the stage's previous tile has been multiplied
+      mbar_wait(smem_u32(&sm.bars_free[s]), (st.prod / (uint32_t)stages - 1u) & 1u);
+    const uint32_t dst = ring0 + s * kTileBytes, bar = smem_u32(&sm.bars[s]);
+    mbar_arrive_expect_tx(bar, kTileBytes);
+    tma_load_2d(dst, c.map, 0, c.row0 + tt * 128, bar);
+    tma_load_2d(dst + kTileBytes / 2, c.map, 64, c.row0 + tt * 128, bar);
+  }
+}
+
+//
+// When the CTA's next queue item (x_next, already claimed) is a pool item too,
+// the producer goes on to stream its first tiles (up to the ring depth) as soon
+// as this item's products release the stages, so the next item's loads are in
+// flight while this one is read out and published.
+__device__ __forceinline__ void pool_item(const EstParams& P, const CUtensorMap* tm, int g, int y, int x_next,
+                                          PoolSmem& sm, unsigned char* ring, int stages, PoolState& st) {
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int slot = y / P.pool_item_span;
   const int blk0 = (y - slot * P.pool_item_span) * kPoolTilesPerItem;
@@ -255,17 +363,14 @@ __device__ __forceinline__ void pool_item(const EstParams& P, const CUtensorMap*
   const int hr = is_q ? bi * P.hq + kv * P.G + slot : P.q_rows + g;
   const uint32_t ring0 = (smem_u32(ring) + 1023u) & ~1023u;
   if (t == 0) {  // producer
-    const CUtensorMap* map = &tm[is_q ? 6 : 7];
-    const int row0 = (is_q ? hr : g) * P.nb * 128 + blk0 * 128;  // first token row of the item
     fence_proxy_async_smem();  // generic writes of the last item before the async ones
-    for (int tt = 0; tt < nt; ++tt, ++st.prod) {
-      const uint32_t s = st.prod % (uint32_t)stages;
-      if (st.prod >= (uint32_t)stages)  // the stage's previous tile has been multiplied
-        mbar_wait(smem_u32(&sm.bars_free[s]), (st.prod / (uint32_t)stages - 1u) & 1u);
-      const uint32_t dst = ring0 + s * kTileBytes, bar = smem_u32(&sm.bars[s]);
-      mbar_arrive_expect_tx(bar, kTileBytes);
-      tma_load_2d(dst, map, 0, row0 + tt * 128, bar);
-      tma_load_2d(dst + kTileBytes / 2, map, 64, row0 + tt * 128, bar);
+    pool_stream(pool_coords(P, tm, g, y), st.pre, nt, sm, ring0, stages, st);
+    st.pre = 0;
+    int gn, yn;
+    if (decode_item(P, x_next, gn, yn) == kItemPool) {
+      const PoolCoords cn = pool_coords(P, tm, gn, yn);
+      st.pre = min(cn.nt, stages);
+      pool_stream(cn, 0, st.pre, sm, ring0, stages, st);
     }
   } else if (t == 32) {  // product issuer
     const uint32_t idesc = idesc_bf16_f32(128, kPoolN, 1, 0);
@@ -760,7 +865,6 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
   const int ncolw = score_cols(P.bl.dp);  // N: key blocks per column chunk
   const int ncol = max_i / ncolw + 1;
   const int units = 3 * ncol;
-  const size_t tri = (size_t)P.nb * (P.nb + 1) / 2;
   const uint32_t idesc = ncolw == 128 ? idesc_bf16_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 64, 0, 0);
   const uint32_t sbase = (smem_u32(smem) + 1023u) & ~1023u;
   if (sbase - smem_u32(smem) + (uint32_t)gemm_smem_bytes(P.bl.dp) - 1024u > (uint32_t)P.smem_bytes) {
@@ -902,12 +1006,37 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
         }
     }
   }
-  __syncthreads();  // score tiles and row maxima are visible to all threads
+  __syncthreads();  // score tiles and row maxima complete
+  // publish: the chunk's row maxima, then "chunk scored" for its Top-P items
+  if (t < 256) {
+    const int rl = t & 127, band = t >> 7, i = i0 + rl;
+    if (i <= max_i) P.rmax[((size_t)bh * P.nb + i) * 2 + band] = fmaxf(sm.rmax[0][band][rl], sm.rmax[1][band][rl]);
+  }
+  __syncthreads();
+  if (t == 0) {
+    __threadfence();
+    st_release_gpu(&P.sync[1 + 2 * P.n_groups + bh * nchunk + chunk], 1u);
+  }
+  __syncthreads();  // shared memory is reused by the next item
+}
 
-  // steps (5)-(7): one warp per row, both bands, union, whole mask row.  A
-  // warp's tasks are (row, band) pairs; the logits of the next task stream
-  // into the other half of a double buffer (cp.async) while the current one
-  // is ranked.
+// ---------------------------------------------------------------------------
+// Top-P item: steps (5)-(7) for kToppRows consecutive query blocks of one
+// (batch, Q head): one warp per row at a time, both bands, union, whole mask
+// row.  A warp's tasks are (row, band) pairs; the logits of the next task
+// stream into the other half of a double buffer (cp.async) while the current
+// one is ranked.  The rows' score chunk has been published by its score item.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void topp_item(const EstParams& P, int g, int y, unsigned char* smem) {
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int bi = g / P.hkv, kv = g - bi * P.hkv;
+  const int nseg = (P.nb + kToppRows - 1) / kToppRows;
+  const int seg = nseg - 1 - y / P.G;  // longest rows first
+  const int bh = bi * P.hq + kv * P.G + y % P.G;
+  const int r0 = seg * kToppRows;
+  const int max_i = min(P.nb, r0 + kToppRows) - 1;
+  const int chunk = r0 / kScoreRows, i0 = chunk * kScoreRows;
+  const size_t tri = (size_t)P.nb * (P.nb + 1) / 2;
   if (warp < P.topp_warps) {
     unsigned char* wb = smem + (size_t)warp * P.topp_stride;
     const int nbp = (P.nb + 7) & ~7;
@@ -915,11 +1044,11 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
     S.cand = reinterpret_cast<uint16_t*>(wb + (size_t)nbp * 8);
     S.h = reinterpret_cast<unsigned long long*>(wb + (size_t)nbp * 10);
     uint32_t* bits = reinterpret_cast<uint32_t*>(wb + (size_t)nbp * 10 + kTopPBins * 8);
-    const int nrows = max_i - i0 - warp >= 0 ? (max_i - i0 - warp) / P.topp_warps + 1 : 0;
+    const int nrows = max_i - r0 - warp >= 0 ? (max_i - r0 - warp) / P.topp_warps + 1 : 0;
     const int ntasks = 2 * nrows;
     const float* tiles = score_tile(P, bh, chunk, 0);
     auto fetch = [&](int task) {  // logits of task -> buffer (task & 1), 16-byte pieces
-      const int i = i0 + warp + (task >> 1) * P.topp_warps;
+      const int i = r0 + warp + (task >> 1) * P.topp_warps;
       const float* row = tiles + (i - i0) * 128 + (task & 1) * 128 * 128;
       const uint32_t dst = smem_u32(wb) + (uint32_t)(task & 1) * (uint32_t)nbp * 4u;
       for (int c = lane; c * 4 <= i; c += 32)
@@ -934,9 +1063,9 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
         cp_async_commit();  // an empty group keeps the count of groups in flight uniform
       cp_async_wait<1>();   // this task's pieces have landed
       __syncwarp();
-      const int i = i0 + warp + (task >> 1) * P.topp_warps, band = task & 1, r = i - i0;
+      const int i = r0 + warp + (task >> 1) * P.topp_warps, band = task & 1;
       const int n = i + 1;
-      const float rmax = fmaxf(sm.rmax[0][band][r], sm.rmax[1][band][r]);
+      const float rmax = P.rmax[((size_t)bh * P.nb + i) * 2 + band];
       S.d = reinterpret_cast<uint32_t*>(wb + (size_t)(task & 1) * nbp * 4);
       float* dbg = P.dbg_scores ? P.dbg_scores + (size_t)bh * 2 * tri + (size_t)band * tri + (size_t)i * (i + 1) / 2
                                 : nullptr;
@@ -963,11 +1092,10 @@ __global__ void __launch_bounds__(kEstThreads, 1)
 estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ TermMaps tms) {
   extern __shared__ __align__(16) unsigned char est_smem[];
   __shared__ PoolSmem psm;
-  __shared__ int s_item;
+  __shared__ int s_next;
   __shared__ int s_ok;
-  const int per_pair = P.pool_items + P.score_items;
   const int stages = P.pool_stages;
-  PoolState pst = {0u, 0u, 0u};
+  PoolState pst = {0u, 0u, 0u, 0};
   ScoreState ss = {0u, 0u, 0u, 0u, 0u};
   for (int i = threadIdx.x; i < 16 * 32; i += kEstThreads) psm.ones[i] = 0x3F803F80u;  // bf16 1.0 pairs
   fence_proxy_async_smem();  // read by the tensor cores
@@ -996,41 +1124,39 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const int total = P.n_groups * per_pair;
+  const int total = P.n_groups * (P.pool_items + P.score_items + P.topp_items);
+  // During a pool item thread 0 already claims the CTA's next item (the
+  // claim's latency is hidden, and a following pool item's tiles can start
+  // streaming); a score item, long and not waited for by anyone, claims its
+  // successor only when it is done, so no pool item is held back behind it.
+  // A claimed item only waits for items earlier in the queue, so the schedule
+  // still cannot deadlock.
+  if (threadIdx.x == 0) s_next = (int)atomicAdd(&P.sync[0], 1u);
   for (;;) {
-    if (threadIdx.x == 0) s_item = (int)atomicAdd(&P.sync[0], 1u);
     __syncthreads();
-    const int x = s_item;
+    const int x = s_next;
     __syncthreads();
     if (x >= total) break;
-    // queue order: pool(0), then pairs (pool(g+1), score(g)), last pair score(n-1) only
     int g, y;
-    bool is_pool;
-    if (x < P.pool_items) {
-      is_pool = true;
-      g = 0;
-      y = x;
-    } else {
-      const int x2 = x - P.pool_items;
-      const int pair = x2 / per_pair;
-      const int rem = x2 - pair * per_pair;
-      if (pair < P.n_groups - 1 && rem < P.pool_items) {
-        is_pool = true;
-        g = pair + 1;
-        y = rem;
-      } else {
-        is_pool = false;
-        g = pair;
-        y = pair < P.n_groups - 1 ? rem - P.pool_items : rem;
-      }
-    }
-    if (is_pool) {
-      pool_item(P, tms.m, g, y, psm, est_smem, stages, pst);
+    const int kind = decode_item(P, x, g, y);
+    if (kind == kItemPool) {
+      const int x_next = threadIdx.x == 0 ? (int)atomicAdd(&P.sync[0], 1u) : total;
+      if (threadIdx.x == 0) s_next = x_next;  // read by all after the item's last barrier
+      pool_item(P, tms.m, g, y, x_next, psm, est_smem, stages, pst);
       continue;
     }
-    // wait until the group's pooling and temperatures are published
+    // wait until what the item reads is published: the group's pooling and
+    // temperatures (score item), or the score chunk of its rows (Top-P item)
     if (threadIdx.x == 0) {
-      const uint32_t* ready = &P.sync[1 + P.n_groups + g];
+      const uint32_t* ready;
+      if (kind == kItemScore) {
+        ready = &P.sync[1 + P.n_groups + g];
+      } else {
+        const int nseg = (P.nb + kToppRows - 1) / kToppRows;
+        const int bh = (g / P.hkv) * P.hq + (g % P.hkv) * P.G + y % P.G;
+        const int chunk = (nseg - 1 - y / P.G) * kToppRows / kScoreRows;
+        ready = &P.sync[1 + 2 * P.n_groups + bh * ((P.nb + kScoreRows - 1) / kScoreRows) + chunk];
+      }
       int ok = 1;
       if (ld_acquire_gpu(ready) == 0u) {
         const uint64_t t0 = globaltimer_ns();
@@ -1045,8 +1171,14 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
       s_ok = ok;
     }
     __syncthreads();
-    if (s_ok) score_item(P, tms.m, g, y, est_smem, psm, ss);
+    if (s_ok) {
+      if (kind == kItemScore)
+        score_item(P, tms.m, g, y, est_smem, psm, ss);
+      else
+        topp_item(P, g, y, est_smem);
+    }
     __syncthreads();
+    if (threadIdx.x == 0) s_next = (int)atomicAdd(&P.sync[0], 1u);
   }
   tc_fence_before();
   __syncthreads();

@@ -32,7 +32,7 @@ struct Plan {
   int explicit_tau;
   float tau_hi, tau_lo;
   float scale;
-  size_t off_pool[kTerms], off_part, off_tau, off_scores, off_mask, off_sync, sync_bytes, total;
+  size_t off_pool[kTerms], off_part, off_tau, off_scores, off_rmax, off_mask, off_sync, sync_bytes, total;
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -117,10 +117,13 @@ int validate(const prism_config* cfg, Plan* pl) {
   P.off_scores = off;
   const size_t nch = ((size_t)P.nb + 127) / 128;
   off = align_up(off + (size_t)P.q_rows * (nch * (nch + 1) / 2) * 2 * 128 * 128 * sizeof(float), 256);
+  P.off_rmax = off;
+  off = align_up(off + (size_t)P.q_rows * P.nb * 2 * sizeof(float), 256);
   P.off_mask = off;
   off = align_up(off + (size_t)P.q_rows * P.nb * P.W * sizeof(uint32_t), 256);
   P.off_sync = off;
-  P.sync_bytes = (1 + 2 * (size_t)P.kv_rows) * sizeof(uint32_t);
+  // queue head, per-group counters and ready flags, per (batch, Q head, score chunk) flags
+  P.sync_bytes = (1 + 2 * (size_t)P.kv_rows + (size_t)P.q_rows * nch) * sizeof(uint32_t);
   off = align_up(off + P.sync_bytes, 256);
   P.total = off;
   return PRISM_OK;
@@ -248,6 +251,7 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   E.dbg_scores = dbg_scores;
   E.mask = mask;
   E.dbg_tau = dbg_tau;
+  E.rmax = reinterpret_cast<float*>(ws + P.off_rmax);
   E.sync = reinterpret_cast<uint32_t*>(ws + P.off_sync);
   E.hq = P.hq;
   E.hkv = P.hkv;
@@ -259,6 +263,7 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   E.pool_item_span = (P.nb + kPoolTilesPerItem - 1) / kPoolTilesPerItem;
   E.pool_items = (E.G + 1) * E.pool_item_span;
   E.score_items = E.G * ((P.nb + kScoreRows - 1) / kScoreRows);
+  E.topp_items = E.G * ((P.nb + kToppRows - 1) / kToppRows);
   const EstLaunch L = est_launch_shape(P.nb);
   E.topp_warps = L.topp_warps;
   E.topp_stride = L.topp_stride;
@@ -274,7 +279,7 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, estimator_kernel, kEstThreads, L.smem) !=
           cudaSuccess)
     return PRISM_ERR_CUDA;
-  const long long items = (long long)E.n_groups * (E.pool_items + E.score_items);
+  const long long items = (long long)E.n_groups * (E.pool_items + E.score_items + E.topp_items);
   const long long grid = std::min<long long>(items, (long long)g_num_sms[dev] * std::max(per_sm, 1));
   // the score items' operands: pooled rows as bf16 [rows, dp], boxes of 64
   // dims x 128 rows (A, and B when dp <= 128) or x 64 rows (B when dp = 192)

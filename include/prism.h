@@ -170,8 +170,8 @@ int prism_prefill(const prism_config* cfg, const void* q, const void* k, const v
  * (device pointers, layouts as above); no dbg outputs.
  *   - Problems whose workspace (prism_workspace_size) exceeds 32 MiB are
  *     rejected with PRISM_ERR_SCRATCH_LIMIT before anything is enqueued
- *     (the Llama-3-8B shape, 32 Q / 8 KV heads, batch 1, fits up to 32,896
- *     tokens = 257 blocks).
+ *     (the Llama-3-8B shape, 32 Q / 8 KV heads, batch 1, fits up to 32,768
+ *     tokens = 256 blocks).
  *   - The first call on a device looks up the array's device address with
  *     cudaGetSymbolAddress while that device is current; make that first call
  *     before any stream capture.

@@ -65,8 +65,10 @@ def test_workspace_size_formula():
         return (x + 255) // 256 * 256
     kv_rows = rows - q_rows
     dp = 128  # default bands: 32 high-only + 32 shared + 64 low-only padded columns
+    nch = 1  # score chunks of 128 query blocks
     expect = 3 * up(rows * nb * dp * 2) + up(rows * nb * 4 * 4) + up(q_rows * 16) \
-        + up(q_rows * 1 * 2 * 128 * 128 * 4) + up(q_rows * nb * 1 * 4) + up((1 + 2 * kv_rows) * 4)
+        + up(q_rows * nch * 2 * 128 * 128 * 4) + up(q_rows * nb * 2 * 4) + up(q_rows * nb * 1 * 4) \
+        + up((1 + 2 * kv_rows + q_rows * nch) * 4)
     assert n == expect
 
 

@@ -50,8 +50,8 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda_device):
 
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda_device):
     hi, lo = gen.default_bands()
-    fits = pb.PrismConfig(1, 32, 8, 257 * 128, hi, lo, 0.95)
-    too_big = pb.PrismConfig(1, 32, 8, 258 * 128, hi, lo, 0.95)
+    fits = pb.PrismConfig(1, 32, 8, 256 * 128, hi, lo, 0.95)
+    too_big = pb.PrismConfig(1, 32, 8, 257 * 128, hi, lo, 0.95)
     assert pb.prism_workspace_size(fits) <= pb.prism_noalloc_scratch_bytes()
     assert pb.prism_workspace_size(too_big) > pb.prism_noalloc_scratch_bytes()
     a = 1 << 20  # never dereferenced: the size check runs before anything is enqueued
