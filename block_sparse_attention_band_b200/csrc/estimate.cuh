@@ -48,12 +48,12 @@ struct BandLayout {
 };
 
 constexpr int kEstThreads = 512;      // 16 warps, one CTA per SM
-constexpr int kPoolTilesPerItem = 16;  // 16 x 32 KB of Q or K per pool item
+constexpr int kPoolTilesPerItem = 32;  // 32 x 32 KB of Q or K per pool item (its block sums fill tensor memory)
 constexpr uint32_t kTileBytes = 128 * 128 * 2;
 constexpr int kMaxPoolStages = 6;      // TMA ring depth (32 KB stages)
 constexpr int kPoolN = 16;             // N of a pooling product: block b sums into TMEM columns [16 b, 16 b + 16)
 constexpr int kScoreRows = 128;       // query blocks (of one head) per score item = MMA M
-constexpr int kToppRows = 32;         // query blocks (of one head) per Top-P item
+constexpr int kToppRows = 64;         // query blocks (of one head) per Top-P item
 constexpr uint32_t kOpChunk = 128 * 64 * 2;  // one 64-dim x 128-row bf16 operand chunk (SW128)
 constexpr int kTerms = 3;             // bf16 terms per pooled value
 // product operands: A (3 terms x dp/64 chunks of 128 rows) once, B one term at
@@ -158,9 +158,9 @@ struct PoolSmem {
   int flag;
 };
 
-// Transpose-reduction across a warp of N (16 or 32) values per lane: lane L
-// ends with the warp's sum of value L % N, in a fixed order (N - 1 shuffles,
-// plus one when N = 16).
+// Transpose-reduction across a warp of N (8, 16 or 32) values per lane: lane
+// L ends with the warp's sum of value L % N, in a fixed order (N - 1
+// shuffles, plus log2(32 / N)).
 template <int N>
 __device__ __forceinline__ float warp_reduce_n(float (&v)[N], int lane) {
 #pragma unroll
@@ -173,7 +173,8 @@ __device__ __forceinline__ float warp_reduce_n(float (&v)[N], int lane) {
       v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
     }
   }
-  if (N == 16) v[0] += __shfl_xor_sync(0xffffffffu, v[0], 16);
+#pragma unroll
+  for (int o = N; o < 32; o <<= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
   return v[0];
 }
 
@@ -394,35 +395,44 @@ __device__ __forceinline__ void pool_item(const EstParams& P, const CUtensorMap*
     mbar_wait(smem_u32(&sm.bar_pool), st.done & 1u);
     ++st.done;
     tc_fence_after();
-    uint32_t v[kPoolTilesPerItem];
-#pragma unroll
-    for (int b = 0; b < kPoolTilesPerItem; ++b)
-      v[b] = tmem_ld1(sm.tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(b * kPoolN));
-    tmem_wait_ld_dep16(v);
-    tc_fence_before();
     const int c = P.bl.col[d];
     const bool ih = c < P.bl.s2, il = c >= P.bl.s1 && c < P.bl.s3;  // c = 255: neither
     const size_t o0 = ((size_t)hr * P.nb + blk0) * P.bl.dp;
-    float ehl[2 * kPoolTilesPerItem], ea[kPoolTilesPerItem];
+    // the item's blocks in groups of 16 (one tensor-memory read of 16 columns each)
+    for (int b0 = 0; b0 < nt; b0 += 16) {
+      uint32_t v[16];
 #pragma unroll
-    for (int b = 0; b < kPoolTilesPerItem; ++b) {
-      const float m = __uint_as_float(v[b]) * (1.0f / 128.0f);
-      const bool ok = b < nt;
-      if (ok && c != 255) {
-        const __nv_bfloat16 th = __float2bfloat16_rn(m);
-        const float r1 = m - __bfloat162float(th);
-        const __nv_bfloat16 tmid = __float2bfloat16_rn(r1);
-        const __nv_bfloat16 tl = __float2bfloat16_rn(r1 - __bfloat162float(tmid));
-        const size_t o = o0 + (size_t)b * P.bl.dp + c;
-        P.pool_t[0][o] = th;
-        P.pool_t[1][o] = tmid;
-        P.pool_t[2][o] = tl;
+      for (int b = 0; b < 16; ++b)
+        v[b] = tmem_ld1(sm.tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)((b0 + b) * kPoolN));
+      tmem_wait_ld_dep16(v);
+      float ehl[32], ea[16];
+#pragma unroll
+      for (int b = 0; b < 16; ++b) {
+        const float m = __uint_as_float(v[b]) * (1.0f / 128.0f);
+        const bool ok = b0 + b < nt;
+        if (ok && c != 255) {
+          const __nv_bfloat16 th = __float2bfloat16_rn(m);
+          const float r1 = m - __bfloat162float(th);
+          const __nv_bfloat16 tmid = __float2bfloat16_rn(r1);
+          const __nv_bfloat16 tl = __float2bfloat16_rn(r1 - __bfloat162float(tmid));
+          const size_t o = o0 + (size_t)(b0 + b) * P.bl.dp + c;
+          P.pool_t[0][o] = th;
+          P.pool_t[1][o] = tmid;
+          P.pool_t[2][o] = tl;
+        }
+        const float x = ok ? m * m : 0.f;
+        ehl[b] = ih ? x : 0.f;
+        ehl[16 + b] = il ? x : 0.f;
+        ea[b] = x;
       }
-      const float x = ok ? m * m : 0.f;
-      ehl[b] = ih ? x : 0.f;
-      ehl[kPoolTilesPerItem + b] = il ? x : 0.f;
-      ea[b] = x;
+      // energy partials: lane L holds the warp's hi (L < 16) or lo sum of
+      // block b0 + L % 16, and its all-dims sum
+      const float rhl = warp_reduce_n<32>(ehl, lane);
+      const float ra = warp_reduce_n<16>(ea, lane);
+      sm.bpart[b0 + (lane & 15)][q4][lane >> 4] = rhl;
+      if (lane < 16) sm.bpart[b0 + lane][q4][2] = ra;
     }
+    tc_fence_before();
     // zero padding columns of the segment layout
     for (int cc = d; cc < P.bl.dp; cc += 128)
       if (P.bl.src[cc] == 255)
@@ -432,15 +442,10 @@ __device__ __forceinline__ void pool_item(const EstParams& P, const CUtensorMap*
           P.pool_t[1][o] = __float2bfloat16_rn(0.f);
           P.pool_t[2][o] = __float2bfloat16_rn(0.f);
         }
-    // energy partials: lane L holds the warp's hi (L < 16) or lo sum of
-    // block L % 16, and its all-dims sum; the four warps add in a fixed order
-    const float rhl = warp_reduce_n<2 * kPoolTilesPerItem>(ehl, lane);
-    const float ra = warp_reduce_n<kPoolTilesPerItem>(ea, lane);
-    sm.bpart[lane & 15][q4][lane >> 4] = rhl;
-    if (lane < 16) sm.bpart[lane][q4][2] = ra;
+    // the four warps' partials of each block, added in a fixed order
     named_barrier(1, 128);
-    if (d < nt * 3) {
-      const int b = d / 3, e = d - 3 * b;
+    for (int q = d; q < nt * 3; q += 128) {
+      const int b = q / 3, e = q - 3 * b;
       P.part[((size_t)hr * P.nb + blk0 + b) * 4 + e] =
           (sm.bpart[b][0][e] + sm.bpart[b][1][e]) + (sm.bpart[b][2][e] + sm.bpart[b][3][e]);
     }
@@ -584,59 +589,56 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
   // e_j, keys (in place of the logits), exact bin masses; only the
   // ceil(n / 32) slots the row has are visited
   const int ns = (n + 31) >> 5;
-  for (int u0 = 0; u0 < ns; u0 += 4) {  // four slots' loads first, then their arithmetic
+  auto hist1 = [&](int j, float x) {
+    const float e = fast_exp2(fmaf(x, kLog2e, -m));
+    const uint32_t d = rank_key(e);
+    S.d[j] = d;
+    bin_add(hlo, hhi, (int)min(d >> 19, (uint32_t)(kTopPBins - 1)), fixmass(e));
+  };
+  int u = 0;
+  for (; u + 4 <= (n >> 5); u += 4) {  // four whole slots: loads first, then their arithmetic
     float x[4];
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int j = (u0 + v) * 32 + lane;
-      x[v] = j < n ? row[j] : 0.f;
-    }
+    for (int v = 0; v < 4; ++v) x[v] = row[(u + v) * 32 + lane];
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int j = (u0 + v) * 32 + lane;
-      if (j < n) {
-        const float e = fast_exp2(fmaf(x[v], kLog2e, -m));
-        const uint32_t d = rank_key(e);
-        S.d[j] = d;
-        bin_add(hlo, hhi, (int)min(d >> 19, (uint32_t)(kTopPBins - 1)), fixmass(e));
-      }
-    }
+    for (int v = 0; v < 4; ++v) hist1((u + v) * 32 + lane, x[v]);
+  }
+  for (; u < ns; ++u) {
+    const int j = u * 32 + lane;
+    if (j < n) hist1(j, row[j]);
   }
   __syncwarp();
-  unsigned long long hv[8], tot = 0ull;
+  // lane l's 8 bins: its total (the two 32-bit half sums cannot wrap)
+  unsigned long long tot;
   {
     const uint4 l0 = reinterpret_cast<const uint4*>(hlo)[2 * lane], l1 = reinterpret_cast<const uint4*>(hlo)[2 * lane + 1];
     const uint4 h0 = reinterpret_cast<const uint4*>(hhi)[2 * lane], h1 = reinterpret_cast<const uint4*>(hhi)[2 * lane + 1];
-    const uint32_t lw[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
-    const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      hv[u] = ((unsigned long long)hw[u] << 16) + lw[u];
-      tot += hv[u];
-    }
+    const uint32_t sl = (l0.x + l0.y) + (l0.z + l0.w) + (l1.x + l1.y) + (l1.z + l1.w);
+    const uint32_t sh = (h0.x + h0.y) + (h0.z + h0.w) + (h1.x + h1.y) + (h1.z + h1.w);
+    tot = ((unsigned long long)sh << 16) + sl;
   }
-  unsigned long long incl = warp_scan_u64(tot, lane);
+  const unsigned long long incl = warp_scan_u64(tot, lane);
   const unsigned long long Z = __shfl_sync(0xffffffffu, incl, 31);
   const unsigned long long target = (unsigned long long)((double)p * (double)Z);
-  // crossing bin: the first with (mass before it + its mass) >= target
+  const unsigned long long lim = target > 0ull ? target : 1ull;
+  // crossing bin: the first whose cumulative mass reaches lim (it holds mass;
+  // lim <= Z, so it exists).  Its lane is found by a ballot over the lanes'
+  // inclusive sums, then lanes 0-7 scan that lane's 8 bins.
   int xb;
   unsigned long long base;
   {
-    unsigned long long run = incl - tot;
-    int bin = -1;
-    unsigned long long bb = 0ull;
+    const int L = __ffs(__ballot_sync(0xffffffffu, incl >= lim)) - 1;
+    const unsigned long long before = __shfl_sync(0xffffffffu, incl - tot, L);
+    const unsigned long long hb = lane < 8 ? bin_mass(hlo, hhi, 8 * L + lane) : 0ull;
+    unsigned long long pre = hb;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (bin < 0 && run + hv[u] >= target && hv[u] > 0ull) {
-        bin = lane * 8 + u;
-        bb = run;
-      }
-      run += hv[u];
+    for (int o = 1; o < 8; o <<= 1) {
+      const unsigned long long v = __shfl_up_sync(0xffffffffu, pre, o);
+      if (lane >= o) pre += v;
     }
-    const unsigned found = __ballot_sync(0xffffffffu, bin >= 0);
-    const int sl = found ? __ffs(found) - 1 : 31;
-    xb = found ? __shfl_sync(0xffffffffu, bin, sl) : kTopPBins - 1;
-    base = found ? __shfl_sync(0xffffffffu, bb, sl) : Z;
+    const int ub = __ffs(__ballot_sync(0xffffffffu, lane < 8 && before + pre >= lim)) - 1;
+    xb = 8 * L + ub;
+    base = before + __shfl_sync(0xffffffffu, pre - hb, ub);
   }
   // one pass: keep the earlier bins, list the crossing bin's members; lane u
   // collects mask word u of each batch
@@ -644,22 +646,25 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
   for (int u0 = 0; u0 < ns; u0 += 32) {
     const int u1 = min(u0 + 32, ns);
     uint32_t myw = 0u;
-#pragma unroll 4
-    for (int u = u0; u < u1; ++u) {
-      const int j = u * 32 + lane;
-      const bool valid = j < n;
-      const int b = valid ? (int)min(S.d[j] >> 19, (uint32_t)(kTopPBins - 1)) : kTopPBins;
+    auto sel = [&](int u, int b) {  // b: bin of block 32 u + lane (kTopPBins: none)
       const unsigned mb = __ballot_sync(0xffffffffu, b < xb);
       const bool in = b == xb;
       const unsigned mi = __ballot_sync(0xffffffffu, in);
-      if (in) S.cand[cnt + __popc(mi & lt)] = (uint16_t)j;
+      if (in) S.cand[cnt + __popc(mi & lt)] = (uint16_t)(u * 32 + lane);
       cnt += __popc(mi);
       if (lane == u - u0) myw = mb;
+    };
+    const int uf = min(u1, n >> 5);  // whole slots
+    int u = u0;
+#pragma unroll 4
+    for (; u < uf; ++u) sel(u, (int)min(S.d[u * 32 + lane] >> 19, (uint32_t)(kTopPBins - 1)));
+    for (; u < u1; ++u) {
+      const int j = u * 32 + lane;
+      sel(u, j < n ? (int)min(S.d[j] >> 19, (uint32_t)(kTopPBins - 1)) : kTopPBins);
     }
     if (lane < u1 - u0) bits[u0 + lane] |= myw;  // slot u holds mask word u
   }
   __syncwarp();
-  const unsigned long long lim = target > 0ull ? target : 1ull;
   if (cnt <= 32) {
     // member x is kept iff base + (mass of the members ranked ahead of it) <
     // lim; the members are listed (key, j, mass) over the no longer needed
@@ -1056,6 +1061,12 @@ __device__ __forceinline__ void topp_item(const EstParams& P, int g, int y, unsi
       cp_async_commit();
     };
     if (ntasks > 0) fetch(0);
+    // row maxima of the warp's first 32 tasks, one per lane, loaded up front
+    float my_rmax = 0.f;
+    if (lane < ntasks) {
+      const int i = r0 + warp + (lane >> 1) * P.topp_warps;
+      my_rmax = P.rmax[((size_t)bh * P.nb + i) * 2 + (lane & 1)];
+    }
     for (int task = 0; task < ntasks; ++task) {
       if (task + 1 < ntasks)
         fetch(task + 1);
@@ -1065,7 +1076,8 @@ __device__ __forceinline__ void topp_item(const EstParams& P, int g, int y, unsi
       __syncwarp();
       const int i = r0 + warp + (task >> 1) * P.topp_warps, band = task & 1;
       const int n = i + 1;
-      const float rmax = P.rmax[((size_t)bh * P.nb + i) * 2 + band];
+      const float rmax_t = __shfl_sync(0xffffffffu, my_rmax, task & 31);
+      const float rmax = task < 32 ? rmax_t : P.rmax[((size_t)bh * P.nb + i) * 2 + band];
       S.d = reinterpret_cast<uint32_t*>(wb + (size_t)(task & 1) * nbp * 4);
       float* dbg = P.dbg_scores ? P.dbg_scores + (size_t)bh * 2 * tri + (size_t)band * tri + (size_t)i * (i + 1) / 2
                                 : nullptr;
@@ -1099,6 +1111,7 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
   ScoreState ss = {0u, 0u, 0u, 0u, 0u};
   for (int i = threadIdx.x; i < 16 * 32; i += kEstThreads) psm.ones[i] = 0x3F803F80u;  // bf16 1.0 pairs
   fence_proxy_async_smem();  // read by the tensor cores
+  fence_proxy_async_smem();  // read by the tensor cores
   if (threadIdx.x == 0) {
     for (int st = 0; st < stages; ++st) {
       mbar_init(smem_u32(&psm.bars[st]), 1u);
@@ -1117,7 +1130,7 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
     fence_mbar_init();
     for (int m = 0; m < 8; ++m) tma_prefetch_desc(&tms.m[m]);
   }
-  if ((threadIdx.x >> 5) == 0) {  // score items: 2 chunks x (hi, lo) x 128 columns; pool items: 16 x 16
+  if ((threadIdx.x >> 5) == 0) {  // score items: 2 chunks x (hi, lo) x 128 columns; pool items: 32 x 16
     tmem_alloc(smem_u32(&psm.tmem), 512);
     tmem_relinquish();
   }
