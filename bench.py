@@ -35,6 +35,9 @@ from tests import gen  # noqa: E402
 METRIC = "Prism prefill ms/layer @128K (estimate+sparse attn); estimator overhead %"
 UNIT = "ms/layer"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_llama3_8b_128k.md")
+KERNEL_SOURCES = ("estimate.cuh", "attention.cuh", "ptx.cuh", "prism.cu")
+KERNELS_PER_STEP = 2  # estimator_kernel + sparse_attn_kernel (the queue reset is a memset)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -45,6 +48,35 @@ def load_peaks():
         return d, "measured"
     except (OSError, ValueError):
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    """sha256 over the CUDA sources, to tell whether profiled counters are stale."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "block_sparse_attention_band_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, keyed by kernel;
+    empty when the summary is missing or the kernels changed since it was taken."""
+    try:
+        text = open(TRAFFIC_FILE).read()
+    except OSError:
+        return {}
+    vals, sha = {}, None
+    for line in text.splitlines():
+        line = line.strip().strip("`")
+        if line.startswith("source_sha256_16:"):
+            sha = line.split(":", 1)[1].strip()
+        elif line.startswith("dram_bytes_per_launch:"):
+            for kv in line.split(":", 1)[1].split():
+                k, v = kv.split("=")
+                vals[k] = float(v)
+    return vals if sha == kernel_source_hash() else {}
 
 
 def dist_env():
@@ -207,6 +239,75 @@ def run_reference(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
+TABLE_WORKLOADS = ("tiny_2k", "llama3_8b_32k", "llama3_8b_128k", "qwen3_8b_64k_planted", "sweep_8k",
+                   "sweep_16k", "sweep_64k", "sweep_128k", "sweep_256k")
+
+
+def run_table(args):
+    """One JSON line per workload of the five configurations (the sweep's N
+    values included): estimator, attention and prefill ms/layer with CUDA
+    events, density and both rooflines.  Separate from the headline line."""
+    import block_sparse_attention_band_b200 as pb
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    peak_tensor = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    names = args.table.split(",") if args.table != "all" else TABLE_WORKLOADS
+    for name in names:
+        w = gen.WORKLOADS[name]
+        q, k, v = gen.make_inputs(w)
+        qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+        del q, k, v
+        hi, lo = gen.default_bands()
+        cfg = pb.PrismConfig(w.batch, w.hq, w.hkv, w.seqlen, hi, lo, w.p)
+        ws = torch.empty(pb.prism_workspace_size(cfg), dtype=torch.uint8, device=dev)
+        mask = torch.empty(w.batch, w.hq, w.nb, cfg.words, dtype=torch.int32, device=dev)
+        o = torch.empty_like(qd)
+        stream = torch.cuda.current_stream(dev)
+        flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)  # > L2, written before each estimator run
+        steps = args.steps
+        for _ in range(max(args.warmup, 3)):
+            pb.prism_prefill(cfg, qd, kd, vd, mask, o, ws, stream=stream)
+        torch.cuda.synchronize()
+        est, att, pre = [], [], []
+        for _ in range(steps):
+            flush.fill_(1)
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            e[0].record(stream)
+            pb.prism_estimate(cfg, qd, kd, mask, ws, stream=stream)
+            e[1].record(stream)
+            pb.prism_sparse_attn(cfg, qd, kd, vd, mask, o, stream=stream)
+            e[2].record(stream)
+            flush.fill_(2)
+            e[3].record(stream)
+            pb.prism_prefill(cfg, qd, kd, vd, mask, o, ws, stream=stream)
+            e[4].record(stream)
+            torch.cuda.synchronize()
+            est.append(e[0].elapsed_time(e[1]))
+            att.append(e[1].elapsed_time(e[2]))
+            pre.append(e[3].elapsed_time(e[4]))
+        assert pb.prism_get_last_device_error() == 0
+        t_est, t_att, t_pre = (statistics.median(x) for x in (est, att, pre))
+        words = mask.cpu().numpy().view(np.uint32)
+        causal_tiles = w.batch * w.hq * w.nb * (w.nb + 1) // 2
+        kept = int(np.unpackbits(words.view(np.uint8)).sum())
+        flops = kept * 4 * 128 ** 3
+        est_bytes = (w.hq + w.hkv) * w.batch * w.seqlen * 128 * 2 + words.nbytes
+        line = {"table": True, "workload": w.name, "seq_len": w.seqlen, "p": w.p, "steps": steps,
+                "estimate_ms": t_est, "attention_ms": t_att, "prefill_ms": t_pre,
+                "estimator_overhead_pct": 100.0 * t_est / (t_est + t_att), "density": kept / causal_tiles,
+                "kept_tiles": kept, "attention_tflops": flops / (t_att * 1e-3) / 1e12,
+                "attention_tensor_frac": flops / (t_att * 1e-3) / 1e12 / peak_tensor,
+                "effective_tflops_vs_dense": causal_tiles * 4 * 128 ** 3 / (t_pre * 1e-3) / 1e12,
+                "estimator_gbs": est_bytes / (t_est * 1e-3) / 1e9,
+                "estimator_hbm_frac": est_bytes / (t_est * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s, {peak_tensor} TFLOP/s bf16 sustained",
+                "timing": "CUDA events; a 512 MB buffer written before each estimator run (L2 flush)"}
+        print(json.dumps(line), flush=True)
+        del qd, kd, vd, ws, mask, o, flush
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -215,7 +316,12 @@ def main():
     ap.add_argument("--impl", default="prism", choices=["prism", "reference"])
     ap.add_argument("--workload", default="llama3_8b_128k", choices=sorted(gen.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--table", default=None,
+                    help="'all' or a comma list of workloads: per-configuration lines instead of the headline")
     args = ap.parse_args()
+    if args.table:
+        run_table(args)
+        return
     rank, world, local = dist_env()
     w = gen.WORKLOADS[args.workload]
     if args.impl == "reference":
@@ -297,6 +403,7 @@ def main():
     est_bytes = (w.hq + w.hkv) * w.batch * w.seqlen * 128 * 2 + words.nbytes
 
     peaks, peak_src = load_peaks()
+    traffic = profiled_traffic() if w.name == "llama3_8b_128k" else {}
     peak_tensor = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     peak_hbm = peaks["hbm_gbs"]
     est_gbs = est_bytes / (t_est * 1e-3) / 1e9
@@ -348,11 +455,14 @@ def main():
                    "estimator_gbs": est_gbs, "estimator_hbm_frac": est_gbs / peak_hbm},
         "roofline": {"kernel": "sparse_attn_kernel", "bound": "tensor", "achieved": attn_tflops,
                      "peak": peak_tensor, "unit": "TFLOP/s", "frac": attn_tflops / peak_tensor,
-                     "traffic": None, "peak_source": f"{peak_src} bf16 sustained"},
-        "estimator_roofline": {"bound": "hbm", "achieved": est_gbs, "peak": peak_hbm, "unit": "GB/s",
-                               "frac": est_gbs / peak_hbm, "bytes": est_bytes, "peak_source": peak_src},
+                     "traffic": traffic.get("sparse_attn_kernel"),
+                     "peak_source": f"{peak_src} bf16 sustained (of {peak_src})"},
+        "estimator_roofline": {"kernel": "estimator_kernel", "bound": "hbm", "achieved": est_gbs,
+                               "peak": peak_hbm, "unit": "GB/s", "frac": est_gbs / peak_hbm,
+                               "algorithmic_bytes": est_bytes, "traffic": traffic.get("estimator_kernel"),
+                               "peak_source": f"{peak_src} copy bandwidth (of {peak_src})"},
         "e2e": {"value": job_value(e2e_ms, world), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }

@@ -213,11 +213,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const int G = hq / hkv;
   const int rows_per_kv = G * nb;
   const int items_per_kv = (rows_per_kv + 1) >> 1;
-  const int kv_total = batch * hkv;
-  const int m = (int)(blockIdx.x / kv_total);
-  const int kv_global = (int)(blockIdx.x % kv_total);
+  // KV-head-major order: the CTAs running at any time share one KV head, whose
+  // K/V (2 N x 256 bytes) then stays in L2 for all its query blocks
+  const int m = (int)(blockIdx.x % items_per_kv);
+  const int kv_global = (int)(blockIdx.x / items_per_kv);
   const int W = (nb + 31) >> 5;
-  (void)items_per_kv;
   Tile tiles[2];
   make_tile(tiles[0], 2 * m, rows_per_kv, G, nb, kv_global, hq, mask, W);
   make_tile(tiles[1], 2 * m + 1, rows_per_kv, G, nb, kv_global, hq, mask, W);
