@@ -20,14 +20,17 @@
 //               S = Q K_j^T (A and B from shared memory), then O += P V_j
 //               with P read from tensor memory (bf16, written over S).
 //               Issue order: PV_A(t), QK_A(t+1), PV_B(t), QK_B(t+1), so one
-//               tile's softmax overlaps the other tile's matrix products.
+//               tile's softmax overlaps the other tile's matrix products;
+//               each P V product starts on keys 0-63 as soon as the softmax
+//               has published that half of P, while it computes the other.
 //   warps 2-3   idle
 //   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: thread =
 //               query row = tensor-memory lane 32*(warp%4)+lane.  Online
 //               softmax in base 2; O is rescaled in tensor memory only when
 //               the running max grows by more than 8 (a factor 256), so the
 //               unnormalised values stay bounded and most steps skip it.
-// The grid runs items from the last query block (most key blocks) down.
+// The grid runs the items of one KV head after the other, within a head from
+// the last query block (most key blocks) down.
 #pragma once
 #include "ptx.cuh"
 
@@ -60,8 +63,9 @@ enum : uint32_t {
   kBarSFull = 7,    // [2] per tile
   kBarPFull = 9,    // [2] per tile
   kBarODone = 11,   // [2] per tile
-  kBarDone = 13,    // softmax threads finished with tensor memory
-  kNumBars = 14
+  kBarPHalf = 13,   // [2] per tile: P of keys 0-63 written
+  kBarDone = 15,    // softmax threads finished with tensor memory
+  kNumBars = 16
 };
 
 // One 128-query tile of a work item.
@@ -137,12 +141,16 @@ __device__ __forceinline__ void mma_qk(uint32_t d_tmem, uint32_t q_smem, uint32_
   }
 }
 
-__device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate) {
+// O += P V over keys [64 part, 64 part + 64): four K steps of 16 keys
+__device__ __forceinline__ void mma_pv_part(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate,
+                                            int part) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 1);  // P K-major (TMEM), V MN-major
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
+  for (int k4 = 0; k4 < 4; ++k4) {
+    const int kk = part * 4 + k4;
     mma_bf16_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(v_smem + kk * 2048, kHalfBytes, 1024), idesc,
                 (accumulate || kk > 0) ? 1u : 0u);
+  }
 }
 
 // Row max of this thread's S row held in registers; DIAG skips keys c > r.
@@ -165,9 +173,12 @@ __device__ __forceinline__ float row_max(const uint32_t (&sv)[128], int r) {
 // thread's S row and returns the row sum of the fp32 values.  Packed f32x2
 // arithmetic for the scale/shift and the sum; four independent partial sums
 // keep the dependency chains short.  DIAG zeroes keys c > r (causal diagonal).
+// The first half (keys 0-63) is published on bar_half as soon as it is in
+// tensor memory, so the P V product can start on it while the second half is
+// computed.
 template <bool DIAG>
 __device__ __forceinline__ float softmax_p(const uint32_t (&sv)[128], uint32_t tS, float scale_log2, float m,
-                                           int r) {
+                                           int r, uint32_t bar_half) {
   const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
   const uint64_t nm2 = f2_pack(-m, -m);
   uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
@@ -189,6 +200,11 @@ __device__ __forceinline__ float softmax_p(const uint32_t (&sv)[128], uint32_t t
       pk[e] = pack_bf16x2(p0, p1);
     }
     tmem_st32(tS + h2 * 32, pk);
+    if (h2 == 0) {
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_half);
+    }
   }
   const uint64_t t2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
   float a0, a1;
@@ -225,7 +241,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   if (threadIdx.x == 0) {
     for (uint32_t s = 0; s < kNumBars; ++s)
-      mbar_init(bar(s), (s == kBarPFull || s == kBarPFull + 1) ? 128u : (s == kBarDone ? 256u : 1u));
+      mbar_init(bar(s), (s == kBarPFull || s == kBarPFull + 1 || s == kBarPHalf || s == kBarPHalf + 1)
+                            ? 128u
+                            : (s == kBarDone ? 256u : 1u));
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -304,9 +322,12 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           bool k_ready = false;
           for (int x = 0; x < 2; ++x) {
             if (in_cur[x]) {
+              if (!(ok = mbar_wait(bar(kBarPHalf + x), u[x] & 1))) break;
+              tc_fence_after();
+              mma_pv_part(tO[x], tS[x], sbase + kOffV + s * kTileBytes, u[x] > 0, 0);
               if (!(ok = mbar_wait(bar(kBarPFull + x), u[x] & 1))) break;
               tc_fence_after();
-              mma_pv(tO[x], tS[x], sbase + kOffV + s * kTileBytes, u[x] > 0);
+              mma_pv_part(tO[x], tS[x], sbase + kOffV + s * kTileBytes, true, 1);
               mma_commit(bar(kBarODone + x));
               ++u[x];
             }
@@ -395,8 +416,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
       m_run = m_new;
       // pass 2 over S: P = exp2(S * scale - m) in bf16, written over S[:, 0:64)
-      const float rs = diag ? softmax_p<true>(sv, tS, scale_log2, m_run, r)
-                            : softmax_p<false>(sv, tS, scale_log2, m_run, r);
+      const float rs = diag ? softmax_p<true>(sv, tS, scale_log2, m_run, r, bar(kBarPHalf + x))
+                            : softmax_p<false>(sv, tS, scale_log2, m_run, r, bar(kBarPHalf + x));
       l_run += rs;
       tmem_wait_st();
       tc_fence_before();
