@@ -308,6 +308,72 @@ def run_table(args):
         torch.cuda.empty_cache()
 
 
+def run_compare_plain(args):
+    """Prism's estimator against the plain mean-pooling estimator (one band of
+    all dims, no temperature) on one workload: density, estimator time, and the
+    error of the block-sparse attention output (our kernel, each estimator's
+    mask) against exact dense causal attention (fp64 oracle) on sampled rows.
+    The dense line (p = 1, every causal block) is the kernel's own bf16 floor."""
+    import block_sparse_attention_band_b200 as pb
+    import oracle
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    w = gen.WORKLOADS[args.compare_plain]
+    q, k, v = gen.make_inputs(w)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    hi, lo = gen.default_bands()
+    g = w.hq // w.hkv
+    rng = np.random.default_rng(11)
+    heads = [kv * g + int(rng.integers(g)) for kv in (0, 2, 5, 7) if kv < w.hkv]
+    blocks = sorted({w.nb - 1, w.nb // 2, w.nb // 4} | {int(x) for x in rng.integers(w.nb // 8, w.nb, 3)})
+    dense_ref = {(h, i): oracle.sparse_attention_block(q, k, v, np.ones(w.nb, dtype=bool), 0, h, i, g)
+                 for h in heads for i in blocks}
+    def density_of(cfg):
+        ws = torch.empty(pb.prism_workspace_size(cfg), dtype=torch.uint8, device=dev)
+        mask = torch.empty(w.batch, w.hq, w.nb, cfg.words, dtype=torch.int32, device=dev)
+        pb.prism_estimate(cfg, qd, kd, mask, ws)
+        words = mask.cpu().numpy().view(np.uint32)
+        return int(np.unpackbits(words.view(np.uint8)).sum()) / (w.batch * w.hq * w.nb * (w.nb + 1) // 2)
+
+    # the plain estimator's p that keeps as many blocks as Prism does (bisection)
+    target = density_of(pb.PrismConfig(w.batch, w.hq, w.hkv, w.seqlen, hi, lo, w.p))
+    lo_p, hi_p = w.p, 0.99999
+    for _ in range(20):
+        mid = 0.5 * (lo_p + hi_p)
+        if density_of(pb.plain_pooling_config(w.batch, w.hq, w.hkv, w.seqlen, mid)) < target:
+            lo_p = mid
+        else:
+            hi_p = mid
+    variants = [("prism", pb.PrismConfig(w.batch, w.hq, w.hkv, w.seqlen, hi, lo, w.p)),
+                ("plain_pooling", pb.plain_pooling_config(w.batch, w.hq, w.hkv, w.seqlen, w.p)),
+                ("plain_pooling_matched_density", pb.plain_pooling_config(w.batch, w.hq, w.hkv, w.seqlen, hi_p)),
+                ("dense", pb.PrismConfig(w.batch, w.hq, w.hkv, w.seqlen, hi, lo, 1.0))]
+    for name, cfg in variants:
+        ws = torch.empty(pb.prism_workspace_size(cfg), dtype=torch.uint8, device=dev)
+        mask = torch.empty(w.batch, w.hq, w.nb, cfg.words, dtype=torch.int32, device=dev)
+        o = torch.empty_like(qd)
+        for _ in range(3):
+            pb.prism_estimate(cfg, qd, kd, mask, ws)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        pb.prism_estimate(cfg, qd, kd, mask, ws)
+        e1.record()
+        pb.prism_sparse_attn(cfg, qd, kd, vd, mask, o)
+        torch.cuda.synchronize()
+        assert pb.prism_get_last_device_error() == 0
+        words = mask.cpu().numpy().view(np.uint32)
+        density = int(np.unpackbits(words.view(np.uint8)).sum()) / (w.batch * w.hq * w.nb * (w.nb + 1) // 2)
+        errs = []
+        for (h, i), ref in dense_ref.items():
+            got = o[0, h, i * 128:(i + 1) * 128].float().cpu().numpy().astype(np.float64)
+            errs.append(float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)))
+        print(json.dumps({"compare": True, "workload": w.name, "estimator": name, "p": cfg.c.p,
+                          "density": density, "estimate_ms": e0.elapsed_time(e1),
+                          "attn_rel_l2_err_vs_dense_mean": float(np.mean(errs)),
+                          "attn_rel_l2_err_vs_dense_max": float(np.max(errs)),
+                          "sampled_rows": f"heads {heads} x query blocks {blocks}"}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -316,11 +382,16 @@ def main():
     ap.add_argument("--impl", default="prism", choices=["prism", "reference"])
     ap.add_argument("--workload", default="llama3_8b_128k", choices=sorted(gen.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--compare-plain", default=None, choices=sorted(gen.WORKLOADS),
+                    help="Prism vs the plain mean-pooling estimator on one workload (attention error vs dense)")
     ap.add_argument("--table", default=None,
                     help="'all' or a comma list of workloads: per-configuration lines instead of the headline")
     args = ap.parse_args()
     if args.table:
         run_table(args)
+        return
+    if args.compare_plain:
+        run_compare_plain(args)
         return
     rank, world, local = dist_env()
     w = gen.WORKLOADS[args.workload]

@@ -14,7 +14,7 @@ import os
 from typing import Optional, Sequence
 
 __all__ = [
-    "PrismError", "PrismConfig", "lib", "lib_path", "prism_version", "prism_status_str",
+    "PrismError", "PrismConfig", "plain_pooling_config", "lib", "lib_path", "prism_version", "prism_status_str",
     "prism_workspace_size", "prism_estimate", "prism_sparse_attn", "prism_prefill",
     "prism_get_last_device_error", "prism_estimate_noalloc", "prism_noalloc_scratch_bytes",
     "PRISM_TAU_RMS", "PRISM_TAU_EXPLICIT", "EXPORTED_SYMBOLS",
@@ -107,6 +107,18 @@ class PrismConfig:
 
     def ptr(self):
         return ctypes.byref(self.c)
+
+
+def plain_pooling_config(batch: int, hq: int, hkv: int, seqlen: int, p: float,
+                         head_dim: int = 128) -> PrismConfig:
+    """The standard coarse-grained block estimator that Prism is set against
+    (gist.science, Technical Summary section 1): one band of all dims, no
+    temperature, i.e. Top-P of softmax(Q_bar K_bar^T / sqrt(head_dim)) per
+    query-block row, mean pooling over each block.  Both Prism bands are set
+    to the full index set, so M = M_high = M_low."""
+    dims = list(range(head_dim))
+    return PrismConfig(batch, hq, hkv, seqlen, dims, dims, p, head_dim=head_dim,
+                       tau_mode=PRISM_TAU_EXPLICIT, tau_hi=1.0, tau_lo=1.0)
 
 
 def _addr(x) -> Optional[int]:

@@ -114,3 +114,12 @@ def test_python_binding_rejects_host_tensors():
     q = torch.zeros(1, 4, 1024, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         pb.prism_sparse_attn(cfg, q, q, q, q, q, stream=0)
+
+
+def test_plain_pooling_config_is_one_band_without_temperature():
+    cfg = pb.plain_pooling_config(1, 4, 2, 1024, 0.9)
+    assert cfg.c.n_hi == cfg.c.n_lo == 128
+    assert [cfg.c.band_hi[i] for i in range(128)] == list(range(128))
+    assert cfg.c.tau_mode == pb.PRISM_TAU_EXPLICIT and cfg.c.tau_hi == cfg.c.tau_lo == 1.0
+    s, n = _ws_size(cfg)
+    assert s == 0 and n > 0

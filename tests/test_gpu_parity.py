@@ -114,6 +114,20 @@ def test_explicit_tau_and_custom_bands(cuda_device):
     P.check_mask(mask, ref, w.p)
 
 
+def test_plain_pooling_baseline(cuda_device):
+    """The single-band, temperature-free estimator (the coarse-grained baseline)
+    matches the oracle run with the same settings, and its two bands coincide."""
+    w = gen.small_workload("plain_nb24", 1, 4, 2, 24 * 128, seed=36, p=0.9)
+    q, k, v, qd, kd, vd = _inputs(w, cuda_device)
+    cfg = pb.plain_pooling_config(w.batch, w.hq, w.hkv, w.seqlen, w.p)
+    mask, sc, tau, _ = P.run_estimate(cfg, qd, kd)
+    dims = list(range(128))
+    ref = oracle.estimate(q, k, dims, dims, w.p, tau_mode="explicit", tau_explicit=(1.0, 1.0))
+    np.testing.assert_array_equal(ref["keep_hi"], ref["keep_lo"])
+    P.check_scores(sc, ref)
+    P.check_mask(mask, ref, w.p)
+
+
 @pytest.mark.parametrize("seed,n_hi,n_lo", [(41, 17, 50), (42, 60, 90), (43, 5, 3), (44, 100, 100)])
 def test_irregular_bands(seed, n_hi, n_lo, cuda_device):
     """Arbitrary band index sets (any sizes, overlaps, dims in neither band):
