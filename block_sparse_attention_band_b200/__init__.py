@@ -99,7 +99,7 @@ class PrismConfig:
 
     @property
     def nb(self) -> int:
-        return self.c.seqlen // self.c.block
+        return -(-self.c.seqlen // self.c.block)  # the last block may be short
 
     @property
     def words(self) -> int:

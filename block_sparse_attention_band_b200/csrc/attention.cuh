@@ -237,7 +237,6 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   Tile tiles[2];
   make_tile(tiles[0], 2 * m, rows_per_kv, G, nb, kv_global, hq, mask, W);
   make_tile(tiles[1], 2 * m + 1, rows_per_kv, G, nb, kv_global, hq, mask, W);
-  const int kv_row0 = kv_global * seqlen;
 
   if (threadIdx.x == 0) {
     for (uint32_t s = 0; s < kNumBars; ++s)
@@ -270,9 +269,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         mbar_arrive_expect_tx(bar(kBarQ), (nA > 0 ? kTileBytes : 0) + (nB > 0 ? kTileBytes : 0));
         for (int x = 0; x < 2; ++x) {
           if ((x == 0 ? nA : nB) == 0) continue;
-          const int q_row = tiles[x].bh * seqlen + tiles[x].i * 128;
-          tma_load_2d(sbase + kOffQ + x * kTileBytes, &tmQ, 0, q_row, bar(kBarQ));
-          tma_load_2d(sbase + kOffQ + x * kTileBytes + kHalfBytes, &tmQ, 64, q_row, bar(kBarQ));
+          const int q_tok = tiles[x].i * 128;  // rows past the sequence end read as zeros
+          tma_load_3d(sbase + kOffQ + x * kTileBytes, &tmQ, 0, q_tok, tiles[x].bh, bar(kBarQ));
+          tma_load_3d(sbase + kOffQ + x * kTileBytes + kHalfBytes, &tmQ, 64, q_tok, tiles[x].bh, bar(kBarQ));
         }
         UnionIter it;
         it.init(&tiles[0], &tiles[1]);
@@ -282,14 +281,14 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           if (j < 0) break;
           const int s = t & 1;
           if (t >= 2 && !mbar_wait(bar(kBarKVEmpty + s), ((t >> 1) - 1) & 1)) break;
-          const int kr = kv_row0 + j * 128;
+          const int kr = j * 128;
           const uint32_t kd = sbase + kOffK + s * kTileBytes, vd = sbase + kOffV + s * kTileBytes;
           mbar_arrive_expect_tx(bar(kBarKFull + s), kTileBytes);
-          tma_load_2d(kd, &tmK, 0, kr, bar(kBarKFull + s));
-          tma_load_2d(kd + kHalfBytes, &tmK, 64, kr, bar(kBarKFull + s));
+          tma_load_3d(kd, &tmK, 0, kr, kv_global, bar(kBarKFull + s));
+          tma_load_3d(kd + kHalfBytes, &tmK, 64, kr, kv_global, bar(kBarKFull + s));
           mbar_arrive_expect_tx(bar(kBarVFull + s), kTileBytes);
-          tma_load_2d(vd, &tmV, 0, kr, bar(kBarVFull + s));
-          tma_load_2d(vd + kHalfBytes, &tmV, 64, kr, bar(kBarVFull + s));
+          tma_load_3d(vd, &tmV, 0, kr, kv_global, bar(kBarVFull + s));
+          tma_load_3d(vd + kHalfBytes, &tmV, 64, kr, kv_global, bar(kBarVFull + s));
         }
       }
     }
@@ -424,11 +423,14 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_arrive(bar(kBarPFull + x));
     }
     // ------------------------------------------------------------ epilogue
-    __nv_bfloat16* orow = T.valid ? out + ((size_t)T.bh * seqlen + (size_t)T.i * 128 + r) * 128 : nullptr;
-    if (T.valid && n == 0) {
+    // query rows past the end of a short last block are computed but not stored
+    const bool row_ok = T.valid && T.i * 128 + r < seqlen;
+    __nv_bfloat16* orow = row_ok ? out + ((size_t)T.bh * seqlen + (size_t)T.i * 128 + r) * 128 : nullptr;
+    if (T.valid && n == 0) {  // (warp-uniform branches: the loads below are warp-collective)
       const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+      if (row_ok)
 #pragma unroll
-      for (int c = 0; c < 16; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
+        for (int c = 0; c < 16; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
     } else if (T.valid && ok && __all_sync(0xffffffffu, mbar_wait(bar(kBarODone + x), (n - 1) & 1))) {
       tc_fence_after();
       const float inv = 1.0f / l_run;
@@ -444,7 +446,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           pk.y = pack_bf16x2(__uint_as_float(v[q4 * 8 + 2]) * inv, __uint_as_float(v[q4 * 8 + 3]) * inv);
           pk.z = pack_bf16x2(__uint_as_float(v[q4 * 8 + 4]) * inv, __uint_as_float(v[q4 * 8 + 5]) * inv);
           pk.w = pack_bf16x2(__uint_as_float(v[q4 * 8 + 6]) * inv, __uint_as_float(v[q4 * 8 + 7]) * inv);
-          reinterpret_cast<uint4*>(orow)[c4 * 4 + q4] = pk;
+          if (row_ok) reinterpret_cast<uint4*>(orow)[c4 * 4 + q4] = pk;
         }
       }
     }

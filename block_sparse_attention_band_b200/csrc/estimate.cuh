@@ -87,7 +87,7 @@ struct EstParams {
   float* rmax;     // [q_rows, nb, 2] scaled band logits' row maxima over j <= i
   uint32_t* sync;  // [0] queue head, [1 + g] pool items done, [1 + n_groups + g] group ready,
                    // [1 + 2 n_groups + bh * nchunk + c] score chunk c of (batch, Q head) bh written
-  int hq, hkv, G, nb, W, q_rows, n_groups;
+  int hq, hkv, G, n, nb, W, q_rows, n_groups;  // n: tokens per head (the last block may be short)
   int pool_items;      // per group
   int score_items;     // per group
   int topp_items;      // per group
@@ -317,10 +317,11 @@ __device__ __forceinline__ int decode_item(const EstParams& P, int x, int& g, in
   return kItemNone;
 }
 
-// The tiles of pool item (g, y): tensor map, first token row, tile count.
+// The tiles of pool item (g, y): tensor map ([heads, n, 128]), head, first
+// token, tile count.
 struct PoolCoords {
   const CUtensorMap* map;
-  int row0, nt;
+  int head, tok0, nt;
 };
 __device__ __forceinline__ PoolCoords pool_coords(const EstParams& P, const CUtensorMap* tm, int g, int y) {
   const int slot = y / P.pool_item_span;
@@ -329,7 +330,8 @@ __device__ __forceinline__ PoolCoords pool_coords(const EstParams& P, const CUte
   const bool is_q = slot < P.G;
   PoolCoords c;
   c.map = &tm[is_q ? 6 : 7];
-  c.row0 = (is_q ? bi * P.hq + kv * P.G + slot : g) * P.nb * 128 + blk0 * 128;
+  c.head = is_q ? bi * P.hq + kv * P.G + slot : g;
+  c.tok0 = blk0 * 128;
   c.nt = min(blk0 + kPoolTilesPerItem, P.nb) - blk0;
   return c;
 }
@@ -343,8 +345,8 @@ __device__ __forceinline__ void pool_stream(const PoolCoords& c, int t0, int t1,
       mbar_wait(smem_u32(&sm.bars_free[s]), (st.prod / (uint32_t)stages - 1u) & 1u);
     const uint32_t dst = ring0 + s * kTileBytes, bar = smem_u32(&sm.bars[s]);
     mbar_arrive_expect_tx(bar, kTileBytes);
-    tma_load_2d(dst, c.map, 0, c.row0 + tt * 128, bar);
-    tma_load_2d(dst + kTileBytes / 2, c.map, 64, c.row0 + tt * 128, bar);
+    tma_load_3d(dst, c.map, 0, c.tok0 + tt * 128, c.head, bar);
+    tma_load_3d(dst + kTileBytes / 2, c.map, 64, c.tok0 + tt * 128, c.head, bar);
   }
 }
 
@@ -408,7 +410,10 @@ __device__ __forceinline__ void pool_item(const EstParams& P, const CUtensorMap*
       float ehl[32], ea[16];
 #pragma unroll
       for (int b = 0; b < 16; ++b) {
-        const float m = __uint_as_float(v[b]) * (1.0f / 128.0f);
+        // block mean: the last block may hold fewer than 128 tokens (zeros past the end)
+        const int blk = blk0 + b0 + b;
+        const float inv = blk == P.nb - 1 ? 1.0f / (float)(P.n - 128 * (P.nb - 1)) : (1.0f / 128.0f);
+        const float m = __uint_as_float(v[b]) * inv;
         const bool ok = b0 + b < nt;
         if (ok && c != 255) {
           const __nv_bfloat16 th = __float2bfloat16_rn(m);

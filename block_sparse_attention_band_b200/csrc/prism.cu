@@ -43,8 +43,7 @@ int validate(const prism_config* cfg, Plan* pl) {
   if (cfg->head_dim != 128 || cfg->block != 128 || cfg->causal != 1) return PRISM_ERR_UNSUPPORTED;
   if (cfg->hq % cfg->hkv != 0) return PRISM_ERR_SHAPE;
   if (cfg->hq / cfg->hkv > kMaxGroupHeads) return PRISM_ERR_UNSUPPORTED;
-  if (cfg->seqlen % cfg->block != 0) return PRISM_ERR_SHAPE;
-  const long long nb = cfg->seqlen / cfg->block;
+  const long long nb = ((long long)cfg->seqlen + cfg->block - 1) / cfg->block;  // the last block may be short
   // TMA row coordinates are 32-bit; Top-P indices are 16-bit
   if ((long long)cfg->batch * cfg->hq * cfg->seqlen >= (1ll << 31)) return PRISM_ERR_SHAPE;
   if (nb > 16384) return PRISM_ERR_UNSUPPORTED;
@@ -233,6 +232,22 @@ int make_map(CUtensorMap* map, const void* base, size_t rows, int cols = 128, in
   return r == CUDA_SUCCESS ? PRISM_OK : PRISM_ERR_CUDA;
 }
 
+// Q, K or V of `heads` heads of n tokens as a 3-D [heads, n, 128] bf16 view:
+// boxes of 64 dims x 128 tokens x 1 head, 128-byte swizzle; tokens past n
+// (a short last block) read as zeros.
+int make_map_tokens(CUtensorMap* map, const void* base, size_t heads, size_t n) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return PRISM_ERR_CUDA;
+  cuuint64_t dims[3] = {128, (cuuint64_t)n, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {128 * sizeof(__nv_bfloat16), (cuuint64_t)n * 128 * sizeof(__nv_bfloat16)};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PRISM_OK : PRISM_ERR_CUDA;
+}
+
 int launched() { return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA; }
 
 // ---------------------------------------------------------------------------
@@ -256,6 +271,7 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   E.hq = P.hq;
   E.hkv = P.hkv;
   E.G = P.hq / P.hkv;
+  E.n = P.n;
   E.nb = P.nb;
   E.W = P.W;
   E.q_rows = P.q_rows;
@@ -289,9 +305,9 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
     if (make_map(&tms.m[term], E.pool_t[term], prow, P.bl.dp, 128) != PRISM_OK ||
         make_map(&tms.m[3 + term], E.pool_t[term], prow, P.bl.dp, 64) != PRISM_OK)
       return PRISM_ERR_CUDA;
-  // the pool items' tiles: Q and K as [rows x tokens, 128], boxes of 64 dims x 128 tokens
-  if (make_map(&tms.m[6], q, (size_t)P.q_rows * P.n) != PRISM_OK ||
-      make_map(&tms.m[7], k, (size_t)P.kv_rows * P.n) != PRISM_OK)
+  // the pool items' tiles: Q and K as [heads, tokens, 128], boxes of 64 dims x 128 tokens
+  if (make_map_tokens(&tms.m[6], q, (size_t)P.q_rows, (size_t)P.n) != PRISM_OK ||
+      make_map_tokens(&tms.m[7], k, (size_t)P.kv_rows, (size_t)P.n) != PRISM_OK)
     return PRISM_ERR_CUDA;
   // the queue head and the per-group counters start at zero on every call
   if (cudaMemsetAsync(E.sync, 0, P.sync_bytes, st) != cudaSuccess) return PRISM_ERR_CUDA;
@@ -302,9 +318,9 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
 int run_attention(const Plan& P, const void* q, const void* k, const void* v, const uint32_t* mask,
                   void* o, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
-  if (make_map(&mq, q, (size_t)P.q_rows * P.n) != PRISM_OK ||
-      make_map(&mk, k, (size_t)P.kv_rows * P.n) != PRISM_OK ||
-      make_map(&mv, v, (size_t)P.kv_rows * P.n) != PRISM_OK)
+  if (make_map_tokens(&mq, q, (size_t)P.q_rows, (size_t)P.n) != PRISM_OK ||
+      make_map_tokens(&mk, k, (size_t)P.kv_rows, (size_t)P.n) != PRISM_OK ||
+      make_map_tokens(&mv, v, (size_t)P.kv_rows, (size_t)P.n) != PRISM_OK)
     return PRISM_ERR_CUDA;
   const float scale_log2 = P.scale * 1.4426950408889634f;
   const unsigned grid = attn::grid_size(P.b, P.hq, P.hkv, P.nb);
@@ -350,7 +366,7 @@ const char* prism_status_str(int s) {
   switch (s) {
     case PRISM_OK: return "ok";
     case PRISM_ERR_NULL: return "a required pointer is NULL";
-    case PRISM_ERR_SHAPE: return "invalid shape (sizes, hq % hkv, seqlen % block, or size overflow)";
+    case PRISM_ERR_SHAPE: return "invalid shape (sizes, hq % hkv, or size overflow)";
     case PRISM_ERR_ALIGN: return "a pointer is not suitably aligned";
     case PRISM_ERR_BAND: return "invalid band index set";
     case PRISM_ERR_P: return "p must be > 0";

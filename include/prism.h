@@ -49,7 +49,7 @@ enum {
   PRISM_OK = 0,
   PRISM_ERR_NULL = -1,        /* a required pointer is NULL                        */
   PRISM_ERR_SHAPE = -2,       /* batch/heads/seqlen non-positive, hq % hkv != 0,
-                                 seqlen % block != 0, or sizes overflow            */
+                                 or sizes overflow                                 */
   PRISM_ERR_ALIGN = -3,       /* a tensor pointer is not 16-byte aligned           */
   PRISM_ERR_BAND = -4,        /* band index out of [0, head_dim), duplicated, or an
                                  empty band                                        */
@@ -95,7 +95,10 @@ typedef struct prism_config {
   int hkv;
   int seqlen;
   int head_dim;          /* must be 128 */
-  int block;             /* B; must be 128; seqlen % block == 0 */
+  int block;             /* B; must be 128.  seqlen need not be a multiple of B:
+                            nb = ceil(seqlen / B) blocks, the last one short; its
+                            pooled value is the mean over the tokens it has, and
+                            attention sees only real tokens (causal) */
   const int32_t* band_hi;
   int n_hi;
   const int32_t* band_lo;

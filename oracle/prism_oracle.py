@@ -75,12 +75,21 @@ def band_slice(x: np.ndarray, dims: Sequence[int]) -> np.ndarray:
 def mean_pool(x: np.ndarray, block: int) -> np.ndarray:
     """Step (2): mean over each run of ``block`` tokens on axis -2.
 
-    x [..., N, d] -> [..., N / block, d]; N must be a multiple of block.
+    x [..., N, d] -> [..., ceil(N / block), d].  When N is not a multiple of
+    block, the last block is the mean over the tokens it has (the pages define
+    blocks of B tokens only; this is the plainest reading for a short tail).
     """
     n = x.shape[-2]
-    assert n % block == 0, "sequence length must be a multiple of the block size"
+    nb = -(-n // block)
+    full = (n // block) * block
     shp = x.shape[:-2] + (n // block, block, x.shape[-1])
-    return x.reshape(shp).mean(axis=-2)
+    head = x[..., :full, :].reshape(shp).mean(axis=-2)
+    if full == n:
+        return head
+    tail = x[..., full:, :].mean(axis=-2, keepdims=True)
+    out = np.concatenate([head, tail], axis=-2)
+    assert out.shape[-2] == nb
+    return out
 
 
 # --------------------------------------------------------------------------
@@ -251,19 +260,21 @@ def sparse_attention_block(q, k, v, mask_row: np.ndarray, b: int, h: int, i: int
     (batch b, Q head h), attending only to the key blocks j <= i whose bit is set
     in ``mask_row`` [nb] (bool), with key s <= query t inside block i.
 
-    Returns [block, D].  A row with no visible key returns 0.
+    Returns [rows, D], rows = the tokens block i has (block, or fewer for a
+    short last block).  A row with no visible key returns 0.
     """
-    qf = to_f64(q[b, h, i * block:(i + 1) * block])
+    n = q.shape[2]
+    qf = to_f64(q[b, h, i * block:min((i + 1) * block, n)])
     kv = h // group
     d = qf.shape[-1]
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     js = [j for j in range(i + 1) if bool(mask_row[j])]
     if not js:
-        return np.zeros((block, d))
-    kf = np.concatenate([to_f64(k[b, kv, j * block:(j + 1) * block]) for j in js])
-    vf = np.concatenate([to_f64(v[b, kv, j * block:(j + 1) * block]) for j in js])
-    key_pos = np.concatenate([np.arange(j * block, (j + 1) * block) for j in js])
-    q_pos = np.arange(i * block, (i + 1) * block)
+        return np.zeros((qf.shape[0], d))
+    kf = np.concatenate([to_f64(k[b, kv, j * block:min((j + 1) * block, n)]) for j in js])
+    vf = np.concatenate([to_f64(v[b, kv, j * block:min((j + 1) * block, n)]) for j in js])
+    key_pos = np.concatenate([np.arange(j * block, min((j + 1) * block, n)) for j in js])
+    q_pos = np.arange(i * block, i * block + qf.shape[0])
     s = (qf @ kf.T) * scale
     visible = key_pos[None, :] <= q_pos[:, None]
     s = np.where(visible, s, -np.inf)

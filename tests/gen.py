@@ -54,7 +54,7 @@ class Workload:
 
     @property
     def nb(self) -> int:
-        return self.seqlen // self.block
+        return -(-self.seqlen // self.block)  # the last block may be short
 
 
 # The five workloads: a tiny single head, the Llama-3-8B-shaped layer at 32K

@@ -73,7 +73,7 @@ def test_workspace_size_formula():
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(seqlen=1000), -2), (dict(hq=3, hkv=2), -2), (dict(batch=0), -2), (dict(seqlen=0), -2),
+    (dict(hq=3, hkv=2), -2), (dict(batch=0), -2), (dict(seqlen=0), -2),
     (dict(head_dim=64), -6), (dict(block=64), -6), (dict(causal=0), -6), (dict(tau_mode=7), -6),
     (dict(p=0.0), -5), (dict(p=-1.0), -5), (dict(p=float("nan")), -5),
     (dict(band_hi=[]), -4), (dict(band_lo=[0, 0]), -4), (dict(band_hi=[128]), -4), (dict(band_lo=[-1]), -4),
@@ -123,3 +123,10 @@ def test_plain_pooling_config_is_one_band_without_temperature():
     assert cfg.c.tau_mode == pb.PRISM_TAU_EXPLICIT and cfg.c.tau_hi == cfg.c.tau_lo == 1.0
     s, n = _ws_size(cfg)
     assert s == 0 and n > 0
+
+
+def test_short_last_block_is_accepted():
+    """seqlen need not be a multiple of the block: ceil(seqlen / 128) blocks."""
+    s, n = _ws_size(_cfg(seqlen=1000))
+    assert s == 0 and n > 0
+    assert _cfg(seqlen=1000).nb == 8 and _cfg(seqlen=1000).words == 1

@@ -68,6 +68,28 @@ def test_attention_parity_with_estimator_mask(w, cuda_device):
     P.check_attention_rows(o, q, k, v, mask, rows, w.hq // w.hkv)
 
 
+@pytest.mark.parametrize("w", [gen.small_workload("short_5x128p1", 1, 2, 1, 5 * 128 + 1, seed=51, p=0.9),
+                               gen.small_workload("short_9x128p77", 1, 4, 2, 9 * 128 + 77, seed=52, p=0.9),
+                               gen.small_workload("short_33x128p127", 2, 4, 1, 33 * 128 + 127, seed=53, p=0.9),
+                               gen.small_workload("short_100", 1, 2, 2, 100, seed=54, p=0.9)],
+                         ids=lambda w: w.name)
+def test_short_last_block(w, cuda_device):
+    """seqlen not a multiple of 128: the last block pools over its own tokens,
+    and attention sees only real tokens; estimator and attention match the
+    oracle on every row, the short last query block included."""
+    q, k, v, qd, kd, vd = _inputs(w, cuda_device)
+    hi, lo = gen.default_bands()
+    cfg = P.make_cfg(w)
+    mask, sc, tau, words = P.run_estimate(cfg, qd, kd)
+    ref = oracle.estimate(q, k, hi, lo, w.p)
+    P.check_tau(tau, ref)
+    P.check_scores(sc, ref)
+    P.check_mask(mask, ref, w.p)
+    o = P.run_attention(cfg, qd, kd, vd, torch.from_numpy(words.view(np.int32)).to(cuda_device))
+    rows = [(b, h, i) for b in range(w.batch) for h in range(w.hq) for i in range(w.nb)]
+    P.check_attention_rows(o, q, k, v, mask, rows, w.hq // w.hkv)
+
+
 @pytest.mark.parametrize("w", [gen.small_workload("dense_nb9", 1, 4, 2, 9 * 128, seed=31),
                                gen.small_workload("dense_b2", 2, 2, 2, 4 * 128, seed=32)],
                          ids=lambda w: w.name)

@@ -32,6 +32,37 @@ def test_pool_constant_and_ramp():
     np.testing.assert_allclose(pooled[:, 0], [1.5, 5.5, 9.5], rtol=0, atol=1e-15)
 
 
+def test_pool_short_last_block():
+    """A sequence that is not a multiple of the block: the last block is the
+    mean over its own tokens (constant -> the constant, ramp -> its midpoint)."""
+    c = np.array([0.5, -2.0, 3.25])
+    x = np.tile(c, (11, 1))  # 11 tokens, blocks of 4: 4 + 4 + 3
+    np.testing.assert_allclose(oracle.mean_pool(x, 4), np.tile(c, (3, 1)), rtol=0, atol=1e-15)
+    t = np.arange(11, dtype=np.float64)[:, None] * np.ones((1, 2))
+    pooled = oracle.mean_pool(t, 4)
+    np.testing.assert_allclose(pooled[:, 0], [1.5, 5.5, 9.0], rtol=0, atol=1e-15)
+    # the exact case still agrees with the reshape definition
+    np.testing.assert_allclose(oracle.mean_pool(t[:8], 4)[:, 0], [1.5, 5.5], rtol=0, atol=0)
+
+
+def test_short_last_block_attention_is_dense_on_valid_tokens():
+    """Attention of the short last query block over all kept blocks equals
+    plain causal attention of those tokens over the whole (short) sequence."""
+    rng = np.random.default_rng(5)
+    n, d = 2 * 16 + 5, 8
+    q = rng.standard_normal((1, 1, n, d))
+    k = rng.standard_normal((1, 1, n, d))
+    v = rng.standard_normal((1, 1, n, d))
+    full = np.ones(3, dtype=bool)
+    got = oracle.sparse_attention_block(q, k, v, full, 0, 0, 2, 1, block=16)
+    s = q[0, 0] @ k[0, 0].T / np.sqrt(d)
+    s = np.where(np.tril(np.ones((n, n), dtype=bool)), s, -np.inf)
+    pr = np.exp(s - s.max(axis=1, keepdims=True))
+    ref = (pr / pr.sum(axis=1, keepdims=True)) @ v[0, 0]
+    assert got.shape == (5, d)
+    np.testing.assert_allclose(got, ref[32:], rtol=1e-12, atol=1e-12)
+
+
 def test_pool_matches_library_avg_pool():
     rng = np.random.default_rng(1)
     x = rng.standard_normal((3, 256, 16))
