@@ -17,6 +17,7 @@ __all__ = [
     "PrismError", "PrismConfig", "plain_pooling_config", "lib", "lib_path", "prism_version", "prism_status_str",
     "prism_workspace_size", "prism_estimate", "prism_sparse_attn", "prism_prefill",
     "prism_get_last_device_error", "prism_estimate_noalloc", "prism_noalloc_scratch_bytes",
+    "prism_selftest_wait_timeout",
     "PRISM_TAU_RMS", "PRISM_TAU_EXPLICIT", "EXPORTED_SYMBOLS",
 ]
 
@@ -29,7 +30,7 @@ PRISM_TAU_EXPLICIT = 1
 EXPORTED_SYMBOLS = (
     "prism_workspace_size", "prism_estimate", "prism_sparse_attn", "prism_prefill",
     "prism_get_last_device_error", "prism_status_str", "prism_version", "prism_estimate_noalloc",
-    "prism_noalloc_scratch_bytes",
+    "prism_noalloc_scratch_bytes", "prism_selftest_wait_timeout",
 )
 
 
@@ -73,6 +74,8 @@ lib.prism_estimate_noalloc.restype = ctypes.c_int
 lib.prism_estimate_noalloc.argtypes = [_cfgp, _vp, _vp, _vp, _vp]
 lib.prism_noalloc_scratch_bytes.restype = ctypes.c_size_t
 lib.prism_noalloc_scratch_bytes.argtypes = []
+lib.prism_selftest_wait_timeout.restype = ctypes.c_int
+lib.prism_selftest_wait_timeout.argtypes = [_vp, ctypes.c_uint]
 lib.prism_get_last_device_error.restype = ctypes.c_int
 lib.prism_get_last_device_error.argtypes = [_vp]
 
@@ -188,6 +191,11 @@ def prism_estimate_noalloc(cfg: PrismConfig, q, k, mask, stream=None) -> None:
 
 def prism_noalloc_scratch_bytes() -> int:
     return lib.prism_noalloc_scratch_bytes()
+
+
+def prism_selftest_wait_timeout(timeout_us: int, stream=None) -> None:
+    """Enqueue the failure-path self test (bounded waits that must give up)."""
+    _check(lib.prism_selftest_wait_timeout(_stream(stream), timeout_us), "prism_selftest_wait_timeout")
 
 
 def prism_get_last_device_error(stream=None) -> int:

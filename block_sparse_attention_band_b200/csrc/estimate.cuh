@@ -126,11 +126,6 @@ __device__ __forceinline__ float warp_max(float v) {
 __device__ __forceinline__ void named_barrier(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
 __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -1175,18 +1170,7 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
         const int chunk = (nseg - 1 - y / P.G) * kToppRows / kScoreRows;
         ready = &P.sync[1 + 2 * P.n_groups + bh * ((P.nb + kScoreRows - 1) / kScoreRows) + chunk];
       }
-      int ok = 1;
-      if (ld_acquire_gpu(ready) == 0u) {
-        const uint64_t t0 = globaltimer_ns();
-        while (ld_acquire_gpu(ready) == 0u) {
-          if (globaltimer_ns() - t0 > 2000000000ull) {
-            set_device_error(kDevErrTimeout);
-            ok = 0;
-            break;
-          }
-        }
-      }
-      s_ok = ok;
+      s_ok = flag_wait_ns(ready, kWaitLimitNs) ? 1 : 0;
     }
     __syncthreads();
     if (s_ok) {

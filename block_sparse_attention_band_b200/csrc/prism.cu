@@ -248,6 +248,25 @@ int make_map_tokens(CUtensorMap* map, const void* base, size_t heads, size_t n) 
   return r == CUDA_SUCCESS ? PRISM_OK : PRISM_ERR_CUDA;
 }
 
+// Failure-path self test: thread 0 waits, with the kernels' own bounded-wait
+// helpers and a short limit, on a device word nothing writes and on an mbarrier
+// phase nothing completes; both give up, record PRISM_ERR_TIMEOUT and the kernel
+// returns normally.
+__device__ uint32_t g_never_set;
+
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1u);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    flag_wait_ns(&g_never_set, limit_ns);
+    mbar_wait_ns(smem_u32(&bar), 0u, limit_ns);
+  }
+}
+
 int launched() { return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA; }
 
 // ---------------------------------------------------------------------------
@@ -459,6 +478,14 @@ int prism_estimate_noalloc(const prism_config* cfg, const void* q, const void* k
 }
 
 size_t prism_noalloc_scratch_bytes(void) { return kStaticScratchBytes; }
+
+int prism_selftest_wait_timeout(prism_stream_t stream, unsigned timeout_us) {
+  if (timeout_us == 0 || timeout_us > 2000000u) return PRISM_ERR_SHAPE;
+  int s = ensure_device();
+  if (s != PRISM_OK) return s;
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>((uint64_t)timeout_us * 1000ull);
+  return launched();
+}
 
 int prism_get_last_device_error(prism_stream_t stream) {
   if (ensure_device() != PRISM_OK) return PRISM_ERR_DEVICE;

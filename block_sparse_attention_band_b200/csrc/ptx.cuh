@@ -59,14 +59,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: gives up after ~2 s of wall time, records a device error and
-// returns false.  Legitimate waits in these kernels last microseconds.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Bounded waits: give up after limit_ns of wall time, record a device error
+// and return false, so the kernel can leave cleanly and the host reads
+// PRISM_ERR_TIMEOUT.  Legitimate waits in these kernels last microseconds; the
+// kernels use a 2 s limit.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+__device__ __forceinline__ bool mbar_wait_ns(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 63u && globaltimer_ns() - t0 > 2000000000ull) {
+    if ((it & 63u) == 63u && globaltimer_ns() - t0 > limit_ns) {
+      set_device_error(kDevErrTimeout);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  return mbar_wait_ns(bar, parity, kWaitLimitNs);
+}
+// Waits until a global word another CTA publishes (release) becomes nonzero.
+__device__ __forceinline__ bool flag_wait_ns(const uint32_t* flag, uint64_t limit_ns) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+  if (v != 0u) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v != 0u) return true;
+    if (globaltimer_ns() - t0 > limit_ns) {
       set_device_error(kDevErrTimeout);
       return false;
     }

@@ -199,6 +199,19 @@ size_t prism_noalloc_scratch_bytes(void);
  */
 int prism_get_last_device_error(prism_stream_t stream);
 
+/*
+ * Diagnostic for the failure path (the paper has no counterpart): enqueues a
+ * one-warp kernel on `stream` that waits, with the same bounded-wait helpers
+ * the estimator and attention kernels use but a limit of `timeout_us`
+ * microseconds (1 .. 2,000,000), on a device word nothing writes and on an
+ * mbarrier phase nothing completes.  Both waits give up and record
+ * PRISM_ERR_TIMEOUT; the kernel returns normally, so the context stays usable.
+ * Read the result with prism_get_last_device_error(stream), which then returns
+ * PRISM_ERR_TIMEOUT (and clears it).  Returns PRISM_OK once enqueued,
+ * PRISM_ERR_SHAPE for a timeout out of range, PRISM_ERR_DEVICE / _CUDA.
+ */
+int prism_selftest_wait_timeout(prism_stream_t stream, unsigned timeout_us);
+
 /* Static description of a status code; never NULL. */
 const char* prism_status_str(int status);
 
