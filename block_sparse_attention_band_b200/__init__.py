@@ -18,7 +18,7 @@ __all__ = [
     "prism_workspace_size", "prism_estimate", "prism_sparse_attn", "prism_prefill",
     "prism_get_last_device_error", "prism_estimate_noalloc", "prism_noalloc_scratch_bytes",
     "prism_selftest_wait_timeout",
-    "PRISM_TAU_RMS", "PRISM_TAU_EXPLICIT", "EXPORTED_SYMBOLS",
+    "PRISM_TAU_RMS", "PRISM_TAU_EXPLICIT", "PRISM_FORCE_SINK", "PRISM_FORCE_DIAG", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -26,6 +26,8 @@ _LIB_PATH = os.path.join(_HERE, "libprism_b200.so")
 
 PRISM_TAU_RMS = 0
 PRISM_TAU_EXPLICIT = 1
+PRISM_FORCE_SINK = 1  # keep key block 0 in every row (optional, not part of the method)
+PRISM_FORCE_DIAG = 2  # keep the diagonal block in every row (optional)
 
 EXPORTED_SYMBOLS = (
     "prism_workspace_size", "prism_estimate", "prism_sparse_attn", "prism_prefill",
@@ -54,6 +56,7 @@ class _Config(ctypes.Structure):
         ("band_lo", ctypes.POINTER(ctypes.c_int32)), ("n_lo", ctypes.c_int),
         ("p", ctypes.c_float), ("causal", ctypes.c_int), ("tau_mode", ctypes.c_int),
         ("tau_hi", ctypes.c_float), ("tau_lo", ctypes.c_float), ("softmax_scale", ctypes.c_float),
+        ("force_blocks", ctypes.c_int),
     ]
 
 
@@ -92,13 +95,13 @@ class PrismConfig:
     def __init__(self, batch: int, hq: int, hkv: int, seqlen: int, band_hi: Sequence[int],
                  band_lo: Sequence[int], p: float, head_dim: int = 128, block: int = 128,
                  causal: int = 1, tau_mode: int = PRISM_TAU_RMS, tau_hi: float = 1.0,
-                 tau_lo: float = 1.0, softmax_scale: float = 0.0):
+                 tau_lo: float = 1.0, softmax_scale: float = 0.0, force_blocks: int = 0):
         self._hi = (ctypes.c_int32 * max(len(band_hi), 1))(*band_hi)
         self._lo = (ctypes.c_int32 * max(len(band_lo), 1))(*band_lo)
         self.c = _Config(batch, hq, hkv, seqlen, head_dim, block,
                          ctypes.cast(self._hi, ctypes.POINTER(ctypes.c_int32)), len(band_hi),
                          ctypes.cast(self._lo, ctypes.POINTER(ctypes.c_int32)), len(band_lo),
-                         p, causal, tau_mode, tau_hi, tau_lo, softmax_scale)
+                         p, causal, tau_mode, tau_hi, tau_lo, softmax_scale, force_blocks)
 
     @property
     def nb(self) -> int:

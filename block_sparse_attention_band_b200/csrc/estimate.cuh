@@ -99,6 +99,7 @@ struct EstParams {
   float p;
   int explicit_tau;
   float tau_hi, tau_lo;
+  int force;  // optional forced blocks: 1 = key block 0, 2 = the diagonal
   BandLayout bl;
 };
 
@@ -1088,6 +1089,11 @@ __device__ __forceinline__ void topp_item(const EstParams& P, int g, int y, unsi
       }
       topp_band_row(rmax, n, P.p, S, bits, dbg, lane);
       if (band == 1) {
+        if (P.force && lane == 0) {  // optional additions to M_high | M_low
+          if (P.force & 1) bits[0] |= 1u;
+          if (P.force & 2) bits[i >> 5] |= 1u << (i & 31);
+        }
+        __syncwarp();
         for (int w = lane; w < P.W; w += 32) dst[w] = bits[w];
         __syncwarp();
       }

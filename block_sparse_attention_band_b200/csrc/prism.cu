@@ -32,6 +32,7 @@ struct Plan {
   int explicit_tau;
   float tau_hi, tau_lo;
   float scale;
+  int force;
   size_t off_pool[kTerms], off_part, off_tau, off_scores, off_rmax, off_mask, off_sync, sync_bytes, total;
 };
 
@@ -53,6 +54,7 @@ int validate(const prism_config* cfg, Plan* pl) {
        !std::isfinite(cfg->tau_lo)))
     return PRISM_ERR_TAU;
   if (!(cfg->p > 0.f)) return PRISM_ERR_P;  // also rejects NaN
+  if (cfg->force_blocks & ~(PRISM_FORCE_SINK | PRISM_FORCE_DIAG)) return PRISM_ERR_UNSUPPORTED;
   if (!cfg->band_hi || !cfg->band_lo) return PRISM_ERR_NULL;
   if (cfg->n_hi <= 0 || cfg->n_lo <= 0 || cfg->n_hi > 128 || cfg->n_lo > 128) return PRISM_ERR_BAND;
   bool in_hi[128] = {}, in_lo[128] = {};
@@ -103,6 +105,7 @@ int validate(const prism_config* cfg, Plan* pl) {
   P.tau_hi = cfg->tau_hi;
   P.tau_lo = cfg->tau_lo;
   P.scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.0f / std::sqrt(128.0f);
+  P.force = cfg->force_blocks;
   const size_t rows = (size_t)P.q_rows + P.kv_rows;
   size_t off = 0;
   for (int term = 0; term < kTerms; ++term) {
@@ -308,6 +311,7 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   E.explicit_tau = P.explicit_tau;
   E.tau_hi = P.tau_hi;
   E.tau_lo = P.tau_lo;
+  E.force = P.force;
   E.bl = P.bl;
   int dev = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||

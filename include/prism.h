@@ -109,7 +109,14 @@ typedef struct prism_config {
   float tau_hi;          /* used only with PRISM_TAU_EXPLICIT; must be > 0 */
   float tau_lo;
   float softmax_scale;   /* attention scale; <= 0 selects 1/sqrt(head_dim) */
+  int force_blocks;      /* 0: the mask is exactly M_high | M_low (the method).
+                            Optional additions, OR-ed bit flags:
+                            PRISM_FORCE_SINK keeps key block 0 in every row,
+                            PRISM_FORCE_DIAG keeps the diagonal block j = i.
+                            Other bits: PRISM_ERR_UNSUPPORTED. */
 } prism_config;
+
+enum { PRISM_FORCE_SINK = 1, PRISM_FORCE_DIAG = 2 };
 
 /*
  * Device workspace, in bytes, that prism_estimate / prism_prefill need for

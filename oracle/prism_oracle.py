@@ -195,8 +195,13 @@ def estimate_head(qbar_hi, qbar_lo, qbar_full, kbar_hi, kbar_lo, kbar_full, p,
 
 def estimate(q, k, band_hi: Sequence[int], band_lo: Sequence[int], p: float,
              block: int = 128, tau_mode: str = "rms", tau_explicit=(1.0, 1.0),
-             heads: Optional[Iterable[int]] = None, keep_dense: bool = True):
+             heads: Optional[Iterable[int]] = None, keep_dense: bool = True,
+             force_sink: bool = False, force_diag: bool = False):
     """Prism's estimator on q [b, Hq, N, D], k [b, Hkv, N, D] (post-RoPE).
+
+    force_sink / force_diag: optional additions to the mask after step (7),
+    key block 0 / the diagonal block of every row (off by default: the method's
+    mask is exactly M_high | M_low).
 
     Returns a dict of fp64/bool arrays with a leading [b, Hq'] (Hq' = the
     selected heads):  q_pool [.., nb, D], tau [.., 2], logits / probs / c_excl
@@ -234,6 +239,15 @@ def estimate(q, k, band_hi: Sequence[int], band_lo: Sequence[int], p: float,
             qb_full = mean_pool(band_slice(qh, full), block)
             kv = h // grp
             res = estimate_head(qb_hi, qb_lo, qb_full, *kb[kv], p, tau_mode, tau_explicit)
+            if force_sink or force_diag:
+                # optional additions after the union (not part of the method)
+                nbh = res["mask"].shape[0]
+                forced = np.zeros((nbh, nbh), dtype=bool)
+                if force_sink:
+                    forced[:, 0] = True
+                if force_diag:
+                    forced[np.arange(nbh), np.arange(nbh)] = True
+                res["mask"] = res["mask"] | forced
             rows["q_pool"].append(qb_full)
             rows["rms_q"].append(np.array([rms(qb_hi), rms(qb_lo), rms(qb_full)]))
             for key in ("tau", "logits", "probs", "c_excl", "keep_hi", "keep_lo", "mask"):

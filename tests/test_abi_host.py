@@ -130,3 +130,10 @@ def test_short_last_block_is_accepted():
     s, n = _ws_size(_cfg(seqlen=1000))
     assert s == 0 and n > 0
     assert _cfg(seqlen=1000).nb == 8 and _cfg(seqlen=1000).words == 1
+
+
+def test_force_blocks_flags_validated():
+    s, _ = _ws_size(_cfg(force_blocks=pb.PRISM_FORCE_SINK | pb.PRISM_FORCE_DIAG))
+    assert s == 0
+    s, _ = _ws_size(_cfg(force_blocks=4))
+    assert s == -6

@@ -136,6 +136,28 @@ def test_explicit_tau_and_custom_bands(cuda_device):
     P.check_mask(mask, ref, w.p)
 
 
+@pytest.mark.parametrize("force", [pb.PRISM_FORCE_SINK, pb.PRISM_FORCE_DIAG,
+                                   pb.PRISM_FORCE_SINK | pb.PRISM_FORCE_DIAG])
+def test_forced_blocks(force, cuda_device):
+    """Optional sink / diagonal blocks are OR-ed into the mask; the attention
+    with that mask matches the oracle."""
+    w = gen.small_workload(f"force{force}_nb21", 1, 4, 2, 21 * 128, seed=37, p=0.5)
+    q, k, v, qd, kd, vd = _inputs(w, cuda_device)
+    hi, lo = gen.default_bands()
+    cfg = P.make_cfg(w, force_blocks=force)
+    mask, _, _, words = P.run_estimate(cfg, qd, kd)
+    ref = oracle.estimate(q, k, hi, lo, w.p, force_sink=bool(force & 1), force_diag=bool(force & 2))
+    P.check_mask(mask, ref, w.p)
+    nb = w.nb
+    if force & 1:
+        assert mask[..., 0].all()
+    if force & 2:
+        assert mask[..., np.arange(nb), np.arange(nb)].all()
+    o = P.run_attention(cfg, qd, kd, vd, torch.from_numpy(words.view(np.int32)).to(cuda_device))
+    rows = [(0, h, i) for h in range(w.hq) for i in range(nb)]
+    P.check_attention_rows(o, q, k, v, mask, rows, w.hq // w.hkv)
+
+
 def test_plain_pooling_baseline(cuda_device):
     """The single-band, temperature-free estimator (the coarse-grained baseline)
     matches the oracle run with the same settings, and its two bands coincide."""

@@ -390,3 +390,19 @@ def test_attention_diagonal_only_is_local_and_empty_is_zero():
     np.testing.assert_allclose(o, (torch.softmax(s, -1) @ vb).numpy(), rtol=1e-10, atol=1e-12)
     z = oracle.sparse_attention_block(q, k, v, np.array([False, False]), 0, 0, 1, group=1)
     assert np.all(z == 0)
+
+
+def test_forced_blocks_are_added_after_the_union():
+    """force_sink / force_diag only add key block 0 / the diagonal to every row
+    of the union; everything else is unchanged."""
+    rng = np.random.default_rng(9)
+    q = rng.standard_normal((1, 2, 6 * 16, 128))
+    k = rng.standard_normal((1, 1, 6 * 16, 128))
+    hi, lo = list(range(64)), list(range(32, 128))
+    base = oracle.estimate(q, k, hi, lo, 0.5, block=16)["mask"]
+    forced = oracle.estimate(q, k, hi, lo, 0.5, block=16, force_sink=True, force_diag=True)["mask"]
+    nb = 6
+    extra = np.zeros((nb, nb), dtype=bool)
+    extra[:, 0] = True
+    extra[np.arange(nb), np.arange(nb)] = True
+    np.testing.assert_array_equal(forced, base | extra)
