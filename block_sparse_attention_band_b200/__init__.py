@@ -14,7 +14,7 @@ import os
 from typing import Optional, Sequence
 
 __all__ = [
-    "PrismError", "PrismConfig", "plain_pooling_config", "lib", "lib_path", "prism_version", "prism_status_str",
+    "PrismError", "PrismConfig", "plain_pooling_config", "rope_band_sets", "lib", "lib_path", "prism_version", "prism_status_str",
     "prism_workspace_size", "prism_estimate", "prism_sparse_attn", "prism_prefill",
     "prism_get_last_device_error", "prism_estimate_noalloc", "prism_noalloc_scratch_bytes",
     "prism_selftest_wait_timeout",
@@ -113,6 +113,33 @@ class PrismConfig:
 
     def ptr(self):
         return ctypes.byref(self.c)
+
+
+def rope_band_sets(layout: str = "half_split", d_high: int = 64, d_low: int = 96,
+                   head_dim: int = 128):
+    """(band_hi, band_lo) index sets for a RoPE layout.
+
+    RoPE rotates dimension pairs; pair j turns at theta_j = base^(-2j / D), j = 0
+    the fastest.  The high band is the d_high / 2 fastest pairs, the low band the
+    d_low / 2 slowest (the review's method step (1): "first d_high / last d_low",
+    read in frequency-pair order).  Pair j occupies dims (j, j + D/2) in the
+    half-split layout (GPT-NeoX / Llama-style checkpoints) and (2j, 2j + 1) in
+    the interleaved layout (GPT-J-style).  RoPE variants that keep the
+    frequencies monotone in j -- YaRN's per-band interpolation, M-RoPE's
+    temporal / height / width sections of one frequency ladder -- keep these
+    sets; only the attenuation of each pair under pooling changes."""
+    half = head_dim // 2
+    if d_high % 2 or d_low % 2 or not (0 < d_high <= head_dim) or not (0 < d_low <= head_dim):
+        raise ValueError("band sizes must be even and in (0, head_dim]")
+    hi_pairs = range(0, d_high // 2)
+    lo_pairs = range(half - d_low // 2, half)
+    if layout == "half_split":
+        dims = lambda pairs: sorted([j for j in pairs] + [j + half for j in pairs])
+    elif layout == "interleaved":
+        dims = lambda pairs: sorted([2 * j for j in pairs] + [2 * j + 1 for j in pairs])
+    else:
+        raise ValueError(f"unknown RoPE layout {layout!r}")
+    return dims(hi_pairs), dims(lo_pairs)
 
 
 def plain_pooling_config(batch: int, hq: int, hkv: int, seqlen: int, p: float,

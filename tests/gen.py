@@ -13,7 +13,9 @@ Summary section 1: Prism consumes Q/K *after* RoPE):
   V [Hkv, N, D], then the workload's extras.
 * pre-RoPE q_t = a_q + 0.5 z_t and k_t = a_k + 0.5 z'_t.
 * half-split RoPE (pair j = dims (j, j + D/2), theta_j = base^(-2j/D)) in fp64
-  at positions 0..N-1, then rounded to bf16 (round-to-nearest-even).
+  at positions 0..N-1, then rounded to bf16 (round-to-nearest-even); a
+  workload with ``interleaved`` set uses the interleaved layout (pair j =
+  dims (2j, 2j + 1)) instead.
 * extras: ``stripes`` -- 64 key positions per KV head (drawn without
   replacement) get pre-RoPE k = 3 * a_q of the group's first Q head;
   ``slash`` -- KV heads 0..Hkv/2-1 get pre-RoPE k_t = q_t(first Q head of the
@@ -51,6 +53,7 @@ class Workload:
     stripes: bool = False
     slash: bool = False
     segment: int = 0  # 0: stationary a_q for every head
+    interleaved: bool = False  # RoPE pairs (2j, 2j+1) instead of (j, j + D/2)
 
     @property
     def nb(self) -> int:
@@ -72,18 +75,27 @@ for _n in (8192, 16384, 65536, 131072, 262144):
                                                  segment=4096)
 
 
-def rope_tables(seqlen: int, head_dim: int, base: float, start: int = 0):
-    """fp64 cos/sin tables [seqlen, head_dim/2] for half-split RoPE."""
+def rope_tables(seqlen: int, head_dim: int, base: float, start: int = 0, theta=None):
+    """fp64 cos/sin tables [seqlen, head_dim/2], column j for pair j (either
+    layout).  ``theta`` overrides the plain ladder base^(-2j/D) (e.g. with a
+    YaRN-rescaled one)."""
     half = head_dim // 2
     j = torch.arange(half, dtype=torch.float64)
-    theta = base ** (-2.0 * j / head_dim)
+    theta = base ** (-2.0 * j / head_dim) if theta is None else torch.as_tensor(theta, dtype=torch.float64)
     t = torch.arange(start, start + seqlen, dtype=torch.float64)
     ang = t[:, None] * theta[None, :]
     return torch.cos(ang), torch.sin(ang)
 
 
-def apply_rope(x: torch.Tensor, cos: torch.Tensor, sin: torch.Tensor) -> torch.Tensor:
-    """Half-split RoPE on the last dim of fp64 ``x`` [..., N, D] (pair j = (j, j+D/2))."""
+def apply_rope(x: torch.Tensor, cos: torch.Tensor, sin: torch.Tensor, interleaved: bool = False) -> torch.Tensor:
+    """RoPE on the last dim of fp64 ``x`` [..., N, D]: pair j = (j, j+D/2)
+    (half-split) or (2j, 2j+1) (interleaved)."""
+    if interleaved:
+        a, b = x[..., 0::2], x[..., 1::2]
+        out = torch.empty_like(x)
+        out[..., 0::2] = a * cos - b * sin
+        out[..., 1::2] = a * sin + b * cos
+        return out
     half = x.shape[-1] // 2
     a, b = x[..., :half], x[..., half:]
     return torch.cat([a * cos - b * sin, a * sin + b * cos], dim=-1)
@@ -131,14 +143,14 @@ def make_inputs(w: Workload, seqlen: Optional[int] = None, with_v: bool = True):
             qh = base_vec + 0.5 * z[h].double()
             if w.slash and h % g == 0 and (h // g) < hkv // 2:
                 pre_q[h] = qh
-            q_out[h] = apply_rope(qh, cos, sin).to(torch.bfloat16)
+            q_out[h] = apply_rope(qh, cos, sin, w.interleaved).to(torch.bfloat16)
         for kv in range(hkv):
             kh = a_k[kv].double()[None, :] + 0.5 * zk[kv].double()
             if w.slash and kv < hkv // 2:
                 kh = pre_q[kv * g] + 0.3 * slash_noise[kv].double()
             if w.stripes:
                 kh[stripe_pos[kv]] = 3.0 * a_q[kv * g].double()
-            k_out[kv] = apply_rope(kh, cos, sin).to(torch.bfloat16)
+            k_out[kv] = apply_rope(kh, cos, sin, w.interleaved).to(torch.bfloat16)
         qs.append(q_out)
         ks.append(k_out)
         vs.append(v.to(torch.bfloat16))

@@ -37,3 +37,18 @@ def test_default_bands():
     assert len(hi) == 64 and len(lo) == 96
     assert hi[:32] == list(range(32)) and hi[32:] == list(range(64, 96))
     assert lo[:48] == list(range(16, 64)) and lo[48:] == list(range(80, 128))
+
+
+def test_interleaved_rope_is_permuted_half_split():
+    # interleaved pair j = dims (2j, 2j+1); moving dim 2j to j and 2j+1 to
+    # j + D/2 turns it into the half-split layout with the same angles
+    cos, sin = gen.rope_tables(64, 128, 10000.0)
+    x = torch.randn(3, 64, 128, dtype=torch.float64, generator=torch.Generator().manual_seed(1))
+    perm = [2 * j for j in range(64)] + [2 * j + 1 for j in range(64)]
+    a = gen.apply_rope(x, cos, sin, interleaved=True)[..., perm]
+    b = gen.apply_rope(x[..., perm], cos, sin)
+    assert torch.allclose(a, b, rtol=0, atol=1e-15)
+    # the rotation keeps every pair's norm
+    n0 = x[..., 0::2] ** 2 + x[..., 1::2] ** 2
+    n1 = gen.apply_rope(x, cos, sin, interleaved=True)
+    assert torch.allclose(n1[..., 0::2] ** 2 + n1[..., 1::2] ** 2, n0, rtol=1e-12)

@@ -189,6 +189,25 @@ def test_irregular_bands(seed, n_hi, n_lo, cuda_device):
     P.check_mask(mask, ref, w.p)
 
 
+@pytest.mark.parametrize("layout", ["interleaved", "half_split"])
+def test_rope_layout_presets(layout, cuda_device):
+    """Inputs rotated in either RoPE layout, bands from the matching preset:
+    estimator and attention match the oracle."""
+    w = gen.small_workload(f"rope_{layout}_nb21", 1, 4, 2, 21 * 128, seed=63, p=0.9,
+                           interleaved=layout == "interleaved")
+    q, k, v, qd, kd, vd = _inputs(w, cuda_device)
+    hi, lo = pb.rope_band_sets(layout)
+    cfg = P.make_cfg(w, bands=(hi, lo))
+    mask, sc, tau, words = P.run_estimate(cfg, qd, kd)
+    ref = oracle.estimate(q, k, hi, lo, w.p)
+    P.check_tau(tau, ref)
+    P.check_scores(sc, ref)
+    P.check_mask(mask, ref, w.p)
+    o = P.run_attention(cfg, qd, kd, vd, torch.from_numpy(words.view(np.int32)).to(cuda_device))
+    rows = [(0, h, i) for h in range(w.hq) for i in range(0, w.nb, 2)]
+    P.check_attention_rows(o, q, k, v, mask, rows, w.hq // w.hkv)
+
+
 def test_small_p_sparse_rows(cuda_device):
     w = gen.small_workload("sparse_nb48", 1, 2, 1, 48 * 128, seed=35, p=0.3)
     q, k, v, qd, kd, vd = _inputs(w, cuda_device)
