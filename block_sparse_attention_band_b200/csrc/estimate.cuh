@@ -53,17 +53,34 @@ constexpr uint32_t kTileBytes = 128 * 128 * 2;
 constexpr int kMaxPoolStages = 6;      // TMA ring depth (32 KB stages)
 constexpr int kPoolN = 16;             // N of a pooling product: block b sums into TMEM columns [16 b, 16 b + 16)
 constexpr int kScoreRows = 128;       // query blocks (of one head) per score item = MMA M
-constexpr int kToppRows = 64;         // query blocks (of one head) per Top-P item
+constexpr int kToppRows = 16;         // query blocks (of one head) per Top-P item
 constexpr uint32_t kOpChunk = 128 * 64 * 2;  // one 64-dim x 128-row bf16 operand chunk (SW128)
 constexpr int kTerms = 3;             // bf16 terms per pooled value
 // product operands: A (3 terms x dp/64 chunks of 128 rows) once, B one term at
 // a time in kBSlots slots (dp/64 chunks of N rows; N = 128, or 64 when dp = 192)
-constexpr int kBSlots = 3;
+constexpr int kBSlots = 2;
 __host__ __device__ constexpr int score_cols(int dp) { return dp <= 128 ? 128 : 64; }
 __host__ __device__ constexpr int gemm_smem_bytes(int dp) {
   return kTerms * (dp / 64) * (int)kOpChunk + kBSlots * (dp / 64) * score_cols(dp) * 128 + 1024;
 }
-constexpr int kGemmSmemBytes = gemm_smem_bytes(192);  // the largest layout: 144 + 3 x 24 KB + alignment
+constexpr int kGemmSmemBytes = gemm_smem_bytes(192);  // the largest layout: 144 + 2 x 24 KB + alignment
+
+// The CTA's warps form two lanes that take items from two queues at once:
+// the stream lane (warps 0, 1, 4-11) runs pool and score items, the Top-P
+// lane (warps 2, 3, 12-15) runs Top-P items, so the Top-P work of earlier
+// groups proceeds on the CUDA cores while the same SM streams Q and K.  Once
+// the stream queue is empty the stream lane's warps take Top-P items too.
+// Each lane synchronises on its own named barrier (1 is the pool read-out
+// warps' own).
+constexpr int kStreamThreads = 320;  // warps 0, 1, 4-11
+constexpr int kLaneThreads = 192;    // warps 2, 3, 12-15
+constexpr int kLaneWarpsMax = kLaneThreads / 32;
+constexpr int kTeamWarpsMax = kStreamThreads / 32;
+enum : int { kBarStream = 2, kBarLane = 3 };
+__device__ __forceinline__ bool in_stream_lane(int warp) { return warp < 2 || (warp >= 4 && warp < 12); }
+__device__ __forceinline__ int stream_tid(int t) { return t < 64 ? t : t - 64; }        // 0 .. 319
+__device__ __forceinline__ int stream_warp(int warp) { return warp < 2 ? warp : warp - 2; }  // 0 .. 9
+__device__ __forceinline__ int lane_warp(int warp) { return warp < 4 ? warp - 2 : warp - 10; }  // 0 .. 5
 constexpr int kMaxGroupHeads = 64;    // Q heads per KV head supported by the tau step
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -85,17 +102,22 @@ struct EstParams {
   uint32_t* mask;
   float* dbg_tau;
   float* rmax;     // [q_rows, nb, 2] scaled band logits' row maxima over j <= i
-  uint32_t* sync;  // [0] queue head, [1 + g] pool items done, [1 + n_groups + g] group ready,
-                   // [1 + 2 n_groups + bh * nchunk + c] score chunk c of (batch, Q head) bh written
+  uint32_t* sync;  // [0] stream queue head, [1] Top-P queue head, [2 + g] pool items done,
+                   // [2 + n_groups + g] group ready,
+                   // [2 + 2 n_groups + bh * nchunk + c] score chunk c of (batch, Q head) bh written
   int hq, hkv, G, n, nb, W, q_rows, n_groups;  // n: tokens per head (the last block may be short)
   int pool_items;      // per group
   int score_items;     // per group
   int topp_items;      // per group
   int pool_item_span;  // pool items per head row
-  int topp_warps;
-  int topp_stride;  // bytes of shared memory per Top-P warp
-  int pool_stages;  // TMA ring depth (<= kMaxPoolStages)
-  int smem_bytes;   // dynamic shared memory of the launch
+  // Top-P warps of each lane: how many take rows, bytes of shared memory
+  // each, and whether a warp holds one logit row (single) or two (the next
+  // one streams in while the current one is ranked)
+  int lane_warps, lane_stride, lane_single;
+  int team_warps, team_stride, team_single;
+  int lane_off;      // byte offset of the Top-P lane's shared memory
+  int stream_bytes;  // dynamic shared memory of the stream lane (pool ring, score operands)
+  int pool_stages;   // TMA ring depth (<= kMaxPoolStages)
   float p;
   int explicit_tau;
   float tau_hi, tau_lo;
@@ -178,12 +200,12 @@ __device__ __forceinline__ float warp_reduce_n(float (&v)[N], int lane) {
 // blocks and the temperatures of its Q heads (reading R1 of the pages: the
 // band's pooled Q x K energy relative to the full spectrum's).
 __device__ __forceinline__ void group_temperatures(const EstParams& P, int g, PoolSmem& sm) {
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int t = stream_tid(threadIdx.x), warp = t >> 5, lane = t & 31;  // the stream lane
   const int bi = g / P.hkv, kv = g - bi * P.hkv;
   for (int slot = 0; slot <= P.G; ++slot) {  // slots 0..G-1: Q heads, G: the KV head
     const int hr = slot < P.G ? bi * P.hq + kv * P.G + slot : P.q_rows + g;
     float s[3] = {0.f, 0.f, 0.f};
-    for (int i = t; i < P.nb; i += kEstThreads) {
+    for (int i = t; i < P.nb; i += kStreamThreads) {
       const float* pp = P.part + ((size_t)hr * P.nb + i) * 4;
       s[0] += pp[0];
       s[1] += pp[1];
@@ -194,13 +216,13 @@ __device__ __forceinline__ void group_temperatures(const EstParams& P, int g, Po
     if (lane == 0)
 #pragma unroll
       for (int e = 0; e < 3; ++e) sm.wred[warp][e] = s[e];
-    __syncthreads();
+    named_barrier(kBarStream, kStreamThreads);
     if (t < 3) {
       float a = 0.f;
-      for (int w = 0; w < kEstThreads / 32; ++w) a += sm.wred[w][t];
+      for (int w = 0; w < kStreamThreads / 32; ++w) a += sm.wred[w][t];
       sm.sums[slot][t] = a;
     }
-    __syncthreads();
+    named_barrier(kBarStream, kStreamThreads);
   }
   if (t < P.G) {
     const int row = bi * P.hq + kv * P.G + t;
@@ -246,71 +268,50 @@ struct PoolState {  // per-role counters of ring stages and items, carried acros
   int pre;  // producer: tiles of the next pool item already streamed into the ring
 };
 
-// Queue order, with PI / SI / TI pool / score / Top-P items per group g of n:
-//   pool(0) | pool(1) score(0) | pool(2) score(1) topp(0) | ... |
-//   pool(n-1) score(n-2) topp(n-3) | score(n-1) topp(n-2) | topp(n-1)
-// so scoring of group g overlaps pooling of group g + 1, and the Top-P items of
-// group g come one group after its score items.  Returns the item kind (0
-// pool, 1 score, 2 Top-P, -1 past the end) and sets (g, y), y the index within
-// the group's items of that kind.
+// Stream queue order, with PI / SI pool / score items per group g of n and a
+// lag of two groups:
+//   pool(0) pool(1) | pool(2) score(0) | pool(3) score(1) | ... | pool(n-1) score(n-3) | score(n-2) score(n-1)
+// so scoring of group g overlaps pooling of group g + 2, by which time the
+// pooling of g has ended and the score items do not wait.  The Top-P queue
+// holds topp(0) | topp(1) | ... | topp(n-1).  Returns the item kind (0 pool,
+// 1 score, 2 Top-P, -1 past the end) and sets (g, y), y the index within the
+// group's items of that kind.
 enum : int { kItemPool = 0, kItemScore = 1, kItemTopp = 2, kItemNone = -1 };
-__device__ __forceinline__ int decode_item(const EstParams& P, int x, int& g, int& y) {
-  const int n = P.n_groups, PI = P.pool_items, SI = P.score_items, TI = P.topp_items;
-  if (x < PI) {
-    g = 0;
-    y = x;
+constexpr int kScoreLag = 2;
+__device__ __forceinline__ int decode_stream(const EstParams& P, int x, int& g, int& y) {
+  const int n = P.n_groups, PI = P.pool_items, SI = P.score_items;
+  const int lag = min(kScoreLag, n), M = n - lag, L = PI + SI;
+  if (x < lag * PI) {
+    g = x / PI;
+    y = x - g * PI;
     return kItemPool;
   }
-  x -= PI;
-  const int first = (n > 1 ? PI : 0) + SI;  // pair 0: pool(1) score(0)
-  if (x < first) {
-    if (n > 1 && x < PI) {
-      g = 1;
-      y = x;
-      return kItemPool;
-    }
-    g = 0;
-    y = x - (n > 1 ? PI : 0);
-    return kItemScore;
-  }
-  x -= first;
-  const int L = PI + SI + TI, M = max(n - 2, 0);  // pairs 1 .. n-2: pool(p+1) score(p) topp(p-1)
-  if (x < M * L) {
-    const int p = 1 + x / L, rem = x - (p - 1) * L;
+  x -= lag * PI;
+  if (x < M * L) {  // pairs p = 0 .. M-1: pool(p + lag) score(p)
+    const int p = x / L, rem = x - p * L;
     if (rem < PI) {
-      g = p + 1;
+      g = p + lag;
       y = rem;
       return kItemPool;
     }
-    if (rem < PI + SI) {
-      g = p;
-      y = rem - PI;
-      return kItemScore;
-    }
-    g = p - 1;
-    y = rem - PI - SI;
-    return kItemTopp;
+    g = p;
+    y = rem - PI;
+    return kItemScore;
   }
   x -= M * L;
-  if (n > 1) {  // pair n-1: score(n-1) topp(n-2)
-    if (x < SI) {
-      g = n - 1;
-      y = x;
-      return kItemScore;
-    }
-    if (x < SI + TI) {
-      g = n - 2;
-      y = x - SI;
-      return kItemTopp;
-    }
-    x -= SI + TI;
-  }
-  if (x < TI) {
-    g = n - 1;
-    y = x;
-    return kItemTopp;
+  if (x < lag * SI) {
+    const int q = x / SI;
+    g = M + q;
+    y = x - q * SI;
+    return kItemScore;
   }
   return kItemNone;
+}
+__device__ __forceinline__ int decode_topp(const EstParams& P, int x, int& g, int& y) {
+  if (x >= P.n_groups * P.topp_items) return kItemNone;
+  g = x / P.topp_items;
+  y = x - g * P.topp_items;
+  return kItemTopp;
 }
 
 // The tiles of pool item (g, y): tensor map ([heads, n, 128]), head, first
@@ -366,7 +367,7 @@ __device__ __forceinline__ void pool_item(const EstParams& P, const CUtensorMap*
     pool_stream(pool_coords(P, tm, g, y), st.pre, nt, sm, ring0, stages, st);
     st.pre = 0;
     int gn, yn;
-    if (decode_item(P, x_next, gn, yn) == kItemPool) {
+    if (decode_stream(P, x_next, gn, yn) == kItemPool) {
       const PoolCoords cn = pool_coords(P, tm, gn, yn);
       st.pre = min(cn.nt, stages);
       pool_stream(cn, 0, st.pre, sm, ring0, stages, st);
@@ -452,20 +453,20 @@ __device__ __forceinline__ void pool_item(const EstParams& P, const CUtensorMap*
     }
   }
   // publish: count the item; the CTA that completes the group computes tau
-  __syncthreads();
+  named_barrier(kBarStream, kStreamThreads);
   if (t == 0) {
     __threadfence();
-    const uint32_t done = atomicAdd(&P.sync[1 + g], 1u);
+    const uint32_t done = atomicAdd(&P.sync[2 + g], 1u);
     sm.flag = (done == (uint32_t)P.pool_items - 1u);
     if (sm.flag) __threadfence();
   }
-  __syncthreads();
+  named_barrier(kBarStream, kStreamThreads);
   if (sm.flag) {
     group_temperatures(P, g, sm);
-    __syncthreads();
+    named_barrier(kBarStream, kStreamThreads);
     if (t == 0) {
       __threadfence();
-      st_release_gpu(&P.sync[1 + P.n_groups + g], 1u);
+      st_release_gpu(&P.sync[2 + P.n_groups + g], 1u);
     }
   }
 }
@@ -821,8 +822,8 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
 // both bands on the tensor cores, accumulators in tensor memory, double
 // buffered; warp roles: warp 0 lane 0 streams the operands (TMA), warp 1
 // lane 0 issues the products, warps 4-11 read the accumulators of a finished
-// chunk, scale them, write the score tiles and keep the row maxima.  Steps
-// (5)-(7) per row follow on all 16 warps.
+// chunk, scale them, write the score tiles and keep the row maxima.  The
+// chunk's rows then wait for a Top-P item (steps 5-7 per row).
 // ---------------------------------------------------------------------------
 struct ScoreState {  // mbarrier parities, carried across items (each role keeps its own)
   uint32_t a, b, free, mma, acc;
@@ -873,7 +874,7 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
   const int units = 3 * ncol;
   const uint32_t idesc = ncolw == 128 ? idesc_bf16_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 64, 0, 0);
   const uint32_t sbase = (smem_u32(smem) + 1023u) & ~1023u;
-  if (sbase - smem_u32(smem) + (uint32_t)gemm_smem_bytes(P.bl.dp) - 1024u > (uint32_t)P.smem_bytes) {
+  if (sbase - smem_u32(smem) + (uint32_t)gemm_smem_bytes(P.bl.dp) - 1024u > (uint32_t)P.stream_bytes) {
     if (t == 0) set_device_error(-6);  // PRISM_ERR_UNSUPPORTED (host sizing makes this unreachable)
     return;
   }
@@ -1012,29 +1013,37 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
         }
     }
   }
-  __syncthreads();  // score tiles and row maxima complete
+  named_barrier(kBarStream, kStreamThreads);  // score tiles and row maxima complete
   // publish: the chunk's row maxima, then "chunk scored" for its Top-P items
-  if (t < 256) {
-    const int rl = t & 127, band = t >> 7, i = i0 + rl;
+  const int st = stream_tid(t);
+  if (st < 256) {
+    const int rl = st & 127, band = st >> 7, i = i0 + rl;
     if (i <= max_i) P.rmax[((size_t)bh * P.nb + i) * 2 + band] = fmaxf(sm.rmax[0][band][rl], sm.rmax[1][band][rl]);
   }
-  __syncthreads();
+  named_barrier(kBarStream, kStreamThreads);
   if (t == 0) {
     __threadfence();
-    st_release_gpu(&P.sync[1 + 2 * P.n_groups + bh * nchunk + chunk], 1u);
+    st_release_gpu(&P.sync[2 + 2 * P.n_groups + bh * nchunk + chunk], 1u);
   }
-  __syncthreads();  // shared memory is reused by the next item
+  named_barrier(kBarStream, kStreamThreads);  // shared memory is reused by the next item
 }
 
 // ---------------------------------------------------------------------------
 // Top-P item: steps (5)-(7) for kToppRows consecutive query blocks of one
 // (batch, Q head): one warp per row at a time, both bands, union, whole mask
-// row.  A warp's tasks are (row, band) pairs; the logits of the next task
-// stream into the other half of a double buffer (cp.async) while the current
-// one is ranked.  The rows' score chunk has been published by its score item.
+// row.  A warp's tasks are (row, band) pairs; with two logit buffers the next
+// task's row streams in (cp.async) while the current one is ranked.  The
+// rows' score chunk has been published by its score item.  Run by a team of
+// nw warps (team-local index lw) with `stride` bytes of shared memory each
+// at `region`.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void topp_item(const EstParams& P, int g, int y, unsigned char* smem) {
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+struct ToppTeam {
+  unsigned char* region;
+  int lw, nw, stride, single;
+};
+
+__device__ __forceinline__ void topp_item(const EstParams& P, int g, int y, const ToppTeam& T) {
+  const int lane = threadIdx.x & 31;
   const int bi = g / P.hkv, kv = g - bi * P.hkv;
   const int nseg = (P.nb + kToppRows - 1) / kToppRows;
   const int seg = nseg - 1 - y / P.G;  // longest rows first
@@ -1043,64 +1052,96 @@ __device__ __forceinline__ void topp_item(const EstParams& P, int g, int y, unsi
   const int max_i = min(P.nb, r0 + kToppRows) - 1;
   const int chunk = r0 / kScoreRows, i0 = chunk * kScoreRows;
   const size_t tri = (size_t)P.nb * (P.nb + 1) / 2;
-  if (warp < P.topp_warps) {
-    unsigned char* wb = smem + (size_t)warp * P.topp_stride;
-    const int nbp = (P.nb + 7) & ~7;
-    ToppScratch S;
-    S.cand = reinterpret_cast<uint16_t*>(wb + (size_t)nbp * 8);
-    S.h = reinterpret_cast<unsigned long long*>(wb + (size_t)nbp * 10);
-    uint32_t* bits = reinterpret_cast<uint32_t*>(wb + (size_t)nbp * 10 + kTopPBins * 8);
-    const int nrows = max_i - r0 - warp >= 0 ? (max_i - r0 - warp) / P.topp_warps + 1 : 0;
-    const int ntasks = 2 * nrows;
-    const float* tiles = score_tile(P, bh, chunk, 0);
-    auto fetch = [&](int task) {  // logits of task -> buffer (task & 1), 16-byte pieces
-      const int i = r0 + warp + (task >> 1) * P.topp_warps;
-      const float* row = tiles + (i - i0) * 128 + (task & 1) * 128 * 128;
-      const uint32_t dst = smem_u32(wb) + (uint32_t)(task & 1) * (uint32_t)nbp * 4u;
-      for (int c = lane; c * 4 <= i; c += 32)
-        cp_async16(dst + (uint32_t)c * 16u, row + (size_t)((c * 4) >> 7) * kTilePair + ((c * 4) & 127));
-      cp_async_commit();
-    };
-    if (ntasks > 0) fetch(0);
-    // row maxima of the warp's first 32 tasks, one per lane, loaded up front
-    float my_rmax = 0.f;
-    if (lane < ntasks) {
-      const int i = r0 + warp + (lane >> 1) * P.topp_warps;
-      my_rmax = P.rmax[((size_t)bh * P.nb + i) * 2 + (lane & 1)];
-    }
-    for (int task = 0; task < ntasks; ++task) {
+  if (T.lw >= T.nw) return;
+  unsigned char* wb = T.region + (size_t)T.lw * T.stride;
+  const int nbp = (P.nb + 7) & ~7;
+  const int nbuf = T.single ? 1 : 2;
+  ToppScratch S;
+  S.cand = reinterpret_cast<uint16_t*>(wb + (size_t)nbp * 4 * nbuf);
+  S.h = reinterpret_cast<unsigned long long*>(wb + (size_t)nbp * (4 * nbuf + 2));
+  uint32_t* bits = reinterpret_cast<uint32_t*>(wb + (size_t)nbp * (4 * nbuf + 2) + kTopPBins * 8);
+  const int nrows = max_i - r0 - T.lw >= 0 ? (max_i - r0 - T.lw) / T.nw + 1 : 0;
+  const int ntasks = 2 * nrows;
+  const float* tiles = score_tile(P, bh, chunk, 0);
+  auto fetch = [&](int task) {  // logits of task -> its buffer, 16-byte pieces
+    const int i = r0 + T.lw + (task >> 1) * T.nw;
+    const float* row = tiles + (i - i0) * 128 + (task & 1) * 128 * 128;
+    const uint32_t dst = smem_u32(wb) + (uint32_t)(task & (nbuf - 1)) * (uint32_t)nbp * 4u;
+    for (int c = lane; c * 4 <= i; c += 32)
+      cp_async16(dst + (uint32_t)c * 16u, row + (size_t)((c * 4) >> 7) * kTilePair + ((c * 4) & 127));
+    cp_async_commit();
+  };
+  if (!T.single && ntasks > 0) fetch(0);
+  // row maxima of the warp's first 32 tasks, one per lane, loaded up front
+  float my_rmax = 0.f;
+  if (lane < ntasks) {
+    const int i = r0 + T.lw + (lane >> 1) * T.nw;
+    my_rmax = P.rmax[((size_t)bh * P.nb + i) * 2 + (lane & 1)];
+  }
+  for (int task = 0; task < ntasks; ++task) {
+    if (T.single) {
+      fetch(task);  // the buffer is free: the last task ended with __syncwarp
+      cp_async_wait<0>();
+    } else {
       if (task + 1 < ntasks)
         fetch(task + 1);
       else
         cp_async_commit();  // an empty group keeps the count of groups in flight uniform
       cp_async_wait<1>();   // this task's pieces have landed
-      __syncwarp();
-      const int i = r0 + warp + (task >> 1) * P.topp_warps, band = task & 1;
-      const int n = i + 1;
-      const float rmax_t = __shfl_sync(0xffffffffu, my_rmax, task & 31);
-      const float rmax = task < 32 ? rmax_t : P.rmax[((size_t)bh * P.nb + i) * 2 + band];
-      S.d = reinterpret_cast<uint32_t*>(wb + (size_t)(task & 1) * nbp * 4);
-      float* dbg = P.dbg_scores ? P.dbg_scores + (size_t)bh * 2 * tri + (size_t)band * tri + (size_t)i * (i + 1) / 2
-                                : nullptr;
-      uint32_t* dst = P.mask + ((size_t)bh * P.nb + i) * P.W;
-      if (band == 0) {
-        for (int w = lane; w < P.W; w += 32) bits[w] = 0u;
-        __syncwarp();
-      }
-      topp_band_row(rmax, n, P.p, S, bits, dbg, lane);
-      if (band == 1) {
-        if (P.force && lane == 0) {  // optional additions to M_high | M_low
-          if (P.force & 1) bits[0] |= 1u;
-          if (P.force & 2) bits[i >> 5] |= 1u << (i & 31);
-        }
-        __syncwarp();
-        for (int w = lane; w < P.W; w += 32) dst[w] = bits[w];
-        __syncwarp();
-      }
     }
-    cp_async_wait<0>();
+    __syncwarp();
+    const int i = r0 + T.lw + (task >> 1) * T.nw, band = task & 1;
+    const int n = i + 1;
+    const float rmax_t = __shfl_sync(0xffffffffu, my_rmax, task & 31);
+    const float rmax = task < 32 ? rmax_t : P.rmax[((size_t)bh * P.nb + i) * 2 + band];
+    S.d = reinterpret_cast<uint32_t*>(wb + (size_t)(task & (nbuf - 1)) * nbp * 4);
+    float* dbg = P.dbg_scores ? P.dbg_scores + (size_t)bh * 2 * tri + (size_t)band * tri + (size_t)i * (i + 1) / 2
+                              : nullptr;
+    uint32_t* dst = P.mask + ((size_t)bh * P.nb + i) * P.W;
+    if (band == 0) {
+      for (int w = lane; w < P.W; w += 32) bits[w] = 0u;
+      __syncwarp();
+    }
+    topp_band_row(rmax, n, P.p, S, bits, dbg, lane);
+    if (band == 1) {
+      if (P.force && lane == 0) {  // optional additions to M_high | M_low
+        if (P.force & 1) bits[0] |= 1u;
+        if (P.force & 2) bits[i >> 5] |= 1u << (i & 31);
+      }
+      __syncwarp();
+      for (int w = lane; w < P.W; w += 32) dst[w] = bits[w];
+      __syncwarp();
+    }
   }
-  __syncthreads();  // shared memory is reused by the next item
+  cp_async_wait<0>();
+}
+
+// A lane's (or the stream team's) loop over the Top-P queue.  `leader` claims
+// each item and waits for its score chunk; every thread of the team passes
+// the team's barrier twice per item.
+__device__ __forceinline__ void topp_loop(const EstParams& P, const ToppTeam& T, bool leader, int bar, int nthreads,
+                                          volatile int* s_item, volatile int* s_ok) {
+  const int nchunk = (P.nb + kScoreRows - 1) / kScoreRows;
+  const int nseg = (P.nb + kToppRows - 1) / kToppRows;
+  for (;;) {
+    if (leader) {
+      const int x = (int)atomicAdd(&P.sync[1], 1u);
+      int g, y, ok = 0;
+      if (decode_topp(P, x, g, y) == kItemTopp) {
+        const int bh = (g / P.hkv) * P.hq + (g % P.hkv) * P.G + y % P.G;
+        const int chunk = (nseg - 1 - y / P.G) * kToppRows / kScoreRows;
+        ok = flag_wait_ns(&P.sync[2 + 2 * P.n_groups + bh * nchunk + chunk], kWaitLimitNs) ? 1 : 0;
+      }
+      *s_item = x;
+      *s_ok = ok;
+    }
+    named_barrier(bar, nthreads);
+    const int x = *s_item, ok = *s_ok;
+    int g, y;
+    if (decode_topp(P, x, g, y) == kItemNone) break;  // no thread passes a barrier after this
+    if (ok) topp_item(P, g, y, T);
+    named_barrier(bar, nthreads);  // the item's shared memory and s_item are reused
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -1110,13 +1151,11 @@ __global__ void __launch_bounds__(kEstThreads, 1)
 estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ TermMaps tms) {
   extern __shared__ __align__(16) unsigned char est_smem[];
   __shared__ PoolSmem psm;
-  __shared__ int s_next;
-  __shared__ int s_ok;
+  __shared__ int s_next, s_ok, s_titem[2], s_tok[2];
   const int stages = P.pool_stages;
   PoolState pst = {0u, 0u, 0u, 0};
   ScoreState ss = {0u, 0u, 0u, 0u, 0u};
   for (int i = threadIdx.x; i < 16 * 32; i += kEstThreads) psm.ones[i] = 0x3F803F80u;  // bf16 1.0 pairs
-  fence_proxy_async_smem();  // read by the tensor cores
   fence_proxy_async_smem();  // read by the tensor cores
   if (threadIdx.x == 0) {
     for (int st = 0; st < stages; ++st) {
@@ -1143,50 +1182,42 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const int total = P.n_groups * (P.pool_items + P.score_items + P.topp_items);
-  // During a pool item thread 0 already claims the CTA's next item (the
-  // claim's latency is hidden, and a following pool item's tiles can start
-  // streaming); a score item, long and not waited for by anyone, claims its
-  // successor only when it is done, so no pool item is held back behind it.
-  // A claimed item only waits for items earlier in the queue, so the schedule
-  // still cannot deadlock.
-  if (threadIdx.x == 0) s_next = (int)atomicAdd(&P.sync[0], 1u);
-  for (;;) {
-    __syncthreads();
-    const int x = s_next;
-    __syncthreads();
-    if (x >= total) break;
-    int g, y;
-    const int kind = decode_item(P, x, g, y);
-    if (kind == kItemPool) {
-      const int x_next = threadIdx.x == 0 ? (int)atomicAdd(&P.sync[0], 1u) : total;
-      if (threadIdx.x == 0) s_next = x_next;  // read by all after the item's last barrier
-      pool_item(P, tms.m, g, y, x_next, psm, est_smem, stages, pst);
-      continue;
-    }
-    // wait until what the item reads is published: the group's pooling and
-    // temperatures (score item), or the score chunk of its rows (Top-P item)
-    if (threadIdx.x == 0) {
-      const uint32_t* ready;
-      if (kind == kItemScore) {
-        ready = &P.sync[1 + P.n_groups + g];
-      } else {
-        const int nseg = (P.nb + kToppRows - 1) / kToppRows;
-        const int bh = (g / P.hkv) * P.hq + (g % P.hkv) * P.G + y % P.G;
-        const int chunk = (nseg - 1 - y / P.G) * kToppRows / kScoreRows;
-        ready = &P.sync[1 + 2 * P.n_groups + bh * ((P.nb + kScoreRows - 1) / kScoreRows) + chunk];
+  const int warp = threadIdx.x >> 5;
+  if (in_stream_lane(warp)) {
+    const int sid = stream_tid(threadIdx.x);
+    const int total = P.n_groups * (P.pool_items + P.score_items);
+    // During a pool item thread 0 already claims the lane's next item (the
+    // claim's latency is hidden, and a following pool item's tiles can start
+    // streaming); a score item claims its successor only when it is done, so
+    // no pool item is held back behind it.  A claimed item only waits for
+    // items earlier in the queue, so the schedule cannot deadlock.
+    if (sid == 0) s_next = (int)atomicAdd(&P.sync[0], 1u);
+    for (;;) {
+      named_barrier(kBarStream, kStreamThreads);
+      const int x = s_next;
+      named_barrier(kBarStream, kStreamThreads);
+      if (x >= total) break;
+      int g, y;
+      const int kind = decode_stream(P, x, g, y);
+      if (kind == kItemPool) {
+        const int x_next = sid == 0 ? (int)atomicAdd(&P.sync[0], 1u) : total;
+        if (sid == 0) s_next = x_next;  // read by all after the item's last barrier
+        pool_item(P, tms.m, g, y, x_next, psm, est_smem, stages, pst);
+        continue;
       }
-      s_ok = flag_wait_ns(ready, kWaitLimitNs) ? 1 : 0;
+      // a score item waits until its group's pooling and temperatures are published
+      if (sid == 0) s_ok = flag_wait_ns(&P.sync[2 + P.n_groups + g], kWaitLimitNs) ? 1 : 0;
+      named_barrier(kBarStream, kStreamThreads);
+      if (s_ok) score_item(P, tms.m, g, y, est_smem, psm, ss);
+      named_barrier(kBarStream, kStreamThreads);
+      if (sid == 0) s_next = (int)atomicAdd(&P.sync[0], 1u);
     }
-    __syncthreads();
-    if (s_ok) {
-      if (kind == kItemScore)
-        score_item(P, tms.m, g, y, est_smem, psm, ss);
-      else
-        topp_item(P, g, y, est_smem);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) s_next = (int)atomicAdd(&P.sync[0], 1u);
+    // the stream queue is empty: the lane's warps join the Top-P queue
+    const ToppTeam T = {est_smem, stream_warp(warp), P.team_warps, P.team_stride, P.team_single};
+    topp_loop(P, T, sid == 0, kBarStream, kStreamThreads, &s_titem[0], &s_tok[0]);
+  } else if (P.lane_warps > 0) {
+    const ToppTeam T = {est_smem + P.lane_off, lane_warp(warp), P.lane_warps, P.lane_stride, P.lane_single};
+    topp_loop(P, T, threadIdx.x == 64, kBarLane, kLaneThreads, &s_titem[1], &s_tok[1]);
   }
   tc_fence_before();
   __syncthreads();

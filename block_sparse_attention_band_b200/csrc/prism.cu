@@ -125,7 +125,7 @@ int validate(const prism_config* cfg, Plan* pl) {
   off = align_up(off + (size_t)P.q_rows * P.nb * P.W * sizeof(uint32_t), 256);
   P.off_sync = off;
   // queue head, per-group counters and ready flags, per (batch, Q head, score chunk) flags
-  P.sync_bytes = (1 + 2 * (size_t)P.kv_rows + (size_t)P.q_rows * nch) * sizeof(uint32_t);
+  P.sync_bytes = (2 + 2 * (size_t)P.kv_rows + (size_t)P.q_rows * nch) * sizeof(uint32_t);
   off = align_up(off + P.sync_bytes, 256);
   P.total = off;
   return PRISM_OK;
@@ -140,29 +140,43 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 int g_dev_state[kMaxDevices];  // 0 unknown, 1 ready, <0 error code
 
-// Shared memory of the persistent estimator: the score items' product tiles,
-// reused by the Top-P warps (each needs 8 bytes per key block + the bitset).
+// Shared memory of the persistent estimator: the stream lane's region (the
+// pool ring or the score items' operands; Top-P rows for its warps once the
+// stream queue is empty) followed by the Top-P lane's region.
 // the widest product layout and the static scratch share one CTA's 227 KB
 static_assert(kGemmSmemBytes + sizeof(PoolSmem) + 256 <= 232448, "estimator shared memory over the per-CTA limit");
+constexpr size_t kEstMaxDyn = 232448 - sizeof(PoolSmem) - 256;
 
 struct EstLaunch {
-  int topp_warps, topp_stride;
-  size_t smem;
+  int lane_warps, lane_stride, lane_single;
+  int team_warps, team_stride, team_single;
+  size_t stream, smem;
+  int stages;
 };
-EstLaunch est_launch_shape(int nb) {
-  const int W = (nb + 31) / 32;
-  const int nbp = (nb + 7) & ~7;
-  EstLaunch L;
-  // two logit rows (double buffer; keys replace the logits in place) + one u16
-  // member list + 256 64-bit bins + one bit row per warp
-  L.topp_stride = (int)align_up((size_t)nbp * 10 + 256 * 8 + (size_t)W * 4, 16);
-  // dynamic shared memory: the product tiles, or as many Top-P warps as fit
-  // next to the static pool scratch (227 KB per CTA in all)
-  const size_t max_dyn = 232448 - sizeof(PoolSmem) - 256;
-  const size_t want = std::min<size_t>((size_t)(kEstThreads / 32) * L.topp_stride, max_dyn);
-  L.smem = std::max<size_t>(kGemmSmemBytes, want);
-  L.topp_warps = (int)std::max<size_t>(1, std::min<size_t>(kEstThreads / 32, L.smem / L.topp_stride));
-  return L;
+// Per Top-P warp: one or two logit rows (keys replace the logits in place), a
+// u16 member list, 256 64-bit bins and one bit row.
+static size_t topp_stride(int nb, bool single) {
+  const size_t W = ((size_t)nb + 31) / 32, nbp = ((size_t)nb + 7) & ~(size_t)7;
+  return align_up(nbp * (single ? 6 : 10) + 256 * 8 + W * 4, 16);
+}
+// Fills L; false if not even one Top-P warp fits beside the product operands.
+bool est_launch_shape(int nb, int dp, EstLaunch& L) {
+  const size_t sd = topp_stride(nb, false), ss = topp_stride(nb, true);
+  const size_t base = (size_t)gemm_smem_bytes(dp);
+  const size_t rest = kEstMaxDyn - base;
+  const int nd = (int)std::min<size_t>(kLaneWarpsMax, rest / sd), ns = (int)std::min<size_t>(kLaneWarpsMax, rest / ss);
+  L.lane_single = ns > nd;
+  L.lane_warps = L.lane_single ? ns : nd;
+  L.lane_stride = (int)(L.lane_single ? ss : sd);
+  const size_t lane_bytes = (size_t)L.lane_warps * L.lane_stride;
+  L.stream = (kEstMaxDyn - lane_bytes) & ~(size_t)15;  // what the lane leaves: more ring stages
+  const int td = (int)std::min<size_t>(kTeamWarpsMax, L.stream / sd);
+  L.team_single = td == 0;
+  L.team_warps = td > 0 ? td : (int)std::min<size_t>(kTeamWarpsMax, L.stream / ss);
+  L.team_stride = (int)(td > 0 ? sd : ss);
+  L.smem = L.stream + lane_bytes;
+  L.stages = (int)std::min<size_t>(kMaxPoolStages, (L.stream - 1024) / kTileBytes);  // 1 KB-aligned ring
+  return L.team_warps > 0;
 }
 
 int g_num_sms[kMaxDevices];
@@ -193,7 +207,7 @@ int ensure_device() {
   if (cudaFuncSetAttribute(attn::sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)attn::kSmemBytes) != cudaSuccess ||
       cudaFuncSetAttribute(estimator_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)(232448 - sizeof(PoolSmem) - 256)) != cudaSuccess ||
+                           (int)kEstMaxDyn) != cudaSuccess ||
       cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return PRISM_ERR_CUDA;
   g_dev_state[dev] = 1;
@@ -302,11 +316,17 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   E.pool_items = (E.G + 1) * E.pool_item_span;
   E.score_items = E.G * ((P.nb + kScoreRows - 1) / kScoreRows);
   E.topp_items = E.G * ((P.nb + kToppRows - 1) / kToppRows);
-  const EstLaunch L = est_launch_shape(P.nb);
-  E.topp_warps = L.topp_warps;
-  E.topp_stride = L.topp_stride;
-  E.pool_stages = (int)std::min<size_t>(kMaxPoolStages, (L.smem - 1024) / kTileBytes);  // 1 KB-aligned ring
-  E.smem_bytes = (int)L.smem;
+  EstLaunch L;
+  if (!est_launch_shape(P.nb, P.bl.dp, L)) return PRISM_ERR_UNSUPPORTED;
+  E.lane_warps = L.lane_warps;
+  E.lane_stride = L.lane_stride;
+  E.lane_single = L.lane_single;
+  E.team_warps = L.team_warps;
+  E.team_stride = L.team_stride;
+  E.team_single = L.team_single;
+  E.lane_off = (int)L.stream;
+  E.stream_bytes = (int)L.stream;
+  E.pool_stages = L.stages;
   E.p = P.p_eff;
   E.explicit_tau = P.explicit_tau;
   E.tau_hi = P.tau_hi;
