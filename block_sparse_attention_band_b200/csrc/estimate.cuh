@@ -53,6 +53,7 @@ constexpr uint32_t kTileBytes = 128 * 128 * 2;
 constexpr int kMaxPoolStages = 6;      // TMA ring depth (32 KB stages)
 constexpr int kPoolN = 16;             // N of a pooling product: block b sums into TMEM columns [16 b, 16 b + 16)
 constexpr int kScoreRows = 128;       // query blocks (of one head) per score item = MMA M
+constexpr int kScorePartBlocks = 512;  // key blocks per score item: longer rows are split into parts
 constexpr int kToppRows = 16;         // query blocks (of one head) per Top-P item
 constexpr uint32_t kOpChunk = 128 * 64 * 2;  // one 64-dim x 128-row bf16 operand chunk (SW128)
 constexpr int kTerms = 3;             // bf16 terms per pooled value
@@ -82,6 +83,7 @@ __device__ __forceinline__ int stream_tid(int t) { return t < 64 ? t : t - 64; }
 __device__ __forceinline__ int stream_warp(int warp) { return warp < 2 ? warp : warp - 2; }  // 0 .. 9
 __device__ __forceinline__ int lane_warp(int warp) { return warp < 4 ? warp - 2 : warp - 10; }  // 0 .. 5
 constexpr int kMaxGroupHeads = 64;    // Q heads per KV head supported by the tau step
+constexpr int kTauBatch = 5;          // head rows whose energy partials the tau step sums at once
 constexpr float kLog2e = 1.4426950408889634f;
 
 // TMA descriptors of the three pooled bf16 terms [rows, dp]: boxes of 64 dims
@@ -101,13 +103,16 @@ struct EstParams {
   float* dbg_scores;  // optional copy in packed lower-triangular rows [q_rows, 2, nb(nb+1)/2]
   uint32_t* mask;
   float* dbg_tau;
-  float* rmax;     // [q_rows, nb, 2] scaled band logits' row maxima over j <= i
+  float* rmax;     // [q_rows, nb, rparts, 2] scaled band logits' row maxima over the key blocks j <= i
+                   // of each part
   uint32_t* sync;  // [0] stream queue head, [1] Top-P queue head, [2 + g] pool items done,
                    // [2 + n_groups + g] group ready,
-                   // [2 + 2 n_groups + bh * nchunk + c] score chunk c of (batch, Q head) bh written
+                   // [2 + 2 n_groups + bh * nchunk + c] parts of score chunk c of (batch, Q head) bh written
   int hq, hkv, G, n, nb, W, q_rows, n_groups;  // n: tokens per head (the last block may be short)
   int pool_items;      // per group
   int score_items;     // per group
+  int score_span;      // score items per head: (row chunk, key-block part) pairs
+  int rparts;          // key-block parts of the longest row chunk
   int topp_items;      // per group
   int pool_item_span;  // pool items per head row
   // Top-P warps of each lane: how many take rows, bytes of shared memory
@@ -133,6 +138,22 @@ __device__ __forceinline__ float* score_tile(const EstParams& P, int bh, int cr,
   return P.scores + ((size_t)bh * pairs + (size_t)cr * (cr + 1) / 2 + cc) * (2 * 128 * 128);
 }
 
+// Score items: row chunk c (kScoreRows query blocks) against the key blocks
+// j <= its last row, in parts of kScorePartBlocks key blocks.
+__host__ __device__ __forceinline__ int score_parts(int chunk) {
+  return (chunk * kScoreRows + kScoreRows + kScorePartBlocks - 1) / kScorePartBlocks;
+}
+// Item z of one head (longest rows first) -> (row chunk, part).
+__device__ __forceinline__ void score_part_of(const EstParams& P, int z, int& chunk, int& part) {
+  const int nchunk = (P.nb + kScoreRows - 1) / kScoreRows;
+  for (chunk = nchunk - 1; chunk > 0; --chunk) {
+    const int np = score_parts(chunk);
+    if (z < np) break;
+    z -= np;
+  }
+  part = z;
+}
+
 // ---------------------------------------------------------------------------
 // warp / ordering helpers
 // ---------------------------------------------------------------------------
@@ -152,6 +173,9 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads) {
 __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+__device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
 // ---------------------------------------------------------------------------
 // static shared memory of the kernel
@@ -163,13 +187,14 @@ struct PoolSmem {
   __align__(1024) uint32_t ones[16 * 32];
   union {                                   // pool and score items never overlap in a CTA
     float rmax[2][2][128];                  // score item: row maxima per column half and band
-    float wred[16][3];                      // temperatures: per-warp partial sums
+    float wred[16][16];                     // temperatures: per-warp partial sums (kTauBatch slots x 3)
     float bpart[kPoolTilesPerItem][4][3];  // pool item: per block and read-out warp: hi, lo, all
   };
   float sums[kMaxGroupHeads + 1][3];
   uint64_t bars[kMaxPoolStages];       // pool ring: stage loaded
   uint64_t bars_free[kMaxPoolStages];  // pool ring: stage multiplied
   uint64_t bar_pool;                   // pool item: every block sum is in tensor memory
+  uint64_t bar_pool_half;              // pool item: the sums of its first 16 blocks are done
   uint64_t bar_a, bar_b[kBSlots], bar_free[kBSlots], bar_mma[2], bar_acc[2];  // score item: operands, slots,
                                                                             // products, accumulators read
   uint32_t tmem;
@@ -202,25 +227,42 @@ __device__ __forceinline__ float warp_reduce_n(float (&v)[N], int lane) {
 __device__ __forceinline__ void group_temperatures(const EstParams& P, int g, PoolSmem& sm) {
   const int t = stream_tid(threadIdx.x), warp = t >> 5, lane = t & 31;  // the stream lane
   const int bi = g / P.hkv, kv = g - bi * P.hkv;
-  for (int slot = 0; slot <= P.G; ++slot) {  // slots 0..G-1: Q heads, G: the KV head
-    const int hr = slot < P.G ? bi * P.hq + kv * P.G + slot : P.q_rows + g;
-    float s[3] = {0.f, 0.f, 0.f};
+  // slots 0..G-1: Q heads, G: the KV head; kTauBatch slots at a time, so the
+  // loads of all of them are in flight together (the partials come from L2)
+  for (int s0 = 0; s0 <= P.G; s0 += kTauBatch) {
+    const int ns = min(kTauBatch, P.G + 1 - s0);
+    float s[kTauBatch][3];
+#pragma unroll
+    for (int q = 0; q < kTauBatch; ++q) s[q][0] = s[q][1] = s[q][2] = 0.f;
+#pragma unroll 2
     for (int i = t; i < P.nb; i += kStreamThreads) {
-      const float* pp = P.part + ((size_t)hr * P.nb + i) * 4;
-      s[0] += pp[0];
-      s[1] += pp[1];
-      s[2] += pp[2];
+      float4 v[kTauBatch];
+#pragma unroll
+      for (int q = 0; q < kTauBatch; ++q) {
+        const int slot = s0 + q;
+        const int hr = slot < P.G ? bi * P.hq + kv * P.G + slot : P.q_rows + g;
+        v[q] = q < ns ? __ldcg(reinterpret_cast<const float4*>(P.part + ((size_t)hr * P.nb + i) * 4))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int q = 0; q < kTauBatch; ++q) {
+        s[q][0] += v[q].x;
+        s[q][1] += v[q].y;
+        s[q][2] += v[q].z;
+      }
     }
 #pragma unroll
-    for (int e = 0; e < 3; ++e) s[e] = warp_sum(s[e]);
-    if (lane == 0)
+    for (int q = 0; q < kTauBatch; ++q)
 #pragma unroll
-      for (int e = 0; e < 3; ++e) sm.wred[warp][e] = s[e];
+      for (int e = 0; e < 3; ++e) {
+        const float r = warp_sum(s[q][e]);
+        if (lane == 0) sm.wred[warp][3 * q + e] = r;
+      }
     named_barrier(kBarStream, kStreamThreads);
-    if (t < 3) {
+    if (t < 3 * ns) {
       float a = 0.f;
       for (int w = 0; w < kStreamThreads / 32; ++w) a += sm.wred[w][t];
-      sm.sums[slot][t] = a;
+      sm.sums[s0 + t / 3][t % 3] = a;
     }
     named_barrier(kBarStream, kStreamThreads);
   }
@@ -264,7 +306,7 @@ __device__ __forceinline__ void group_temperatures(const EstParams& P, int g, Po
 // 4-7 (thread = dim) read the sums, write the means in the band-segment layout
 // as three bf16 terms and the per-block energy partials.
 struct PoolState {  // per-role counters of ring stages and items, carried across items
-  uint32_t prod, cons, done;
+  uint32_t prod, cons, done, half;
   int pre;  // producer: tiles of the next pool item already streamed into the ring
 };
 
@@ -387,18 +429,25 @@ __device__ __forceinline__ void pool_item(const EstParams& P, const CUtensorMap*
         mma_bf16_ss(sm.tmem + (uint32_t)(tt * kPoolN), adesc + (uint64_t)((k * 2048) >> 4), bdesc, idesc,
                     k > 0 ? 1u : 0u);
       mma_commit(smem_u32(&sm.bars_free[s]));
+      if (tt == 15 && nt > 16) mma_commit(smem_u32(&sm.bar_pool_half));  // the read-out can start
     }
     mma_commit(smem_u32(&sm.bar_pool));
   } else if (warp >= 4 && warp < 8) {  // read-out: thread = dim
     const int q4 = warp & 3, d = q4 * 32 + lane;
-    mbar_wait(smem_u32(&sm.bar_pool), st.done & 1u);
-    ++st.done;
-    tc_fence_after();
     const int c = P.bl.col[d];
     const bool ih = c < P.bl.s2, il = c >= P.bl.s1 && c < P.bl.s3;  // c = 255: neither
     const size_t o0 = ((size_t)hr * P.nb + blk0) * P.bl.dp;
     // the item's blocks in groups of 16 (one tensor-memory read of 16 columns each)
     for (int b0 = 0; b0 < nt; b0 += 16) {
+      // the first 16 blocks are read while the products of the others run
+      if (b0 == 0 && nt > 16) {
+        mbar_wait(smem_u32(&sm.bar_pool_half), st.half & 1u);
+        ++st.half;
+      } else {
+        mbar_wait(smem_u32(&sm.bar_pool), st.done & 1u);
+        ++st.done;
+      }
+      tc_fence_after();
       uint32_t v[16];
 #pragma unroll
       for (int b = 0; b < 16; ++b)
@@ -477,8 +526,8 @@ __device__ __forceinline__ void pool_item(const EstParams& P, const CUtensorMap*
 // Shared-memory scratch of one Top-P warp.
 struct ToppScratch {
   uint32_t* d;            // [n] the row's logits, replaced by the rank keys d_j (below)
-  uint16_t* cand;         // [n] members of the crossing bin
-  unsigned long long* h;  // [256] bin masses
+  uint32_t* memw;         // [ceil(n / 32)] members of the crossing bin, one bit per block
+  unsigned long long* h;  // [256] bin masses; then the member records of the exact step
 };
 
 constexpr int kTopPBins = 256;
@@ -506,17 +555,71 @@ __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v)
   return v;
 }
 
-// Exact crossing among `cnt` members (<= 32) listed in S.cand, all ranked
-// behind mass `base`: returns the member c with ahead(c) < target <=
-// ahead(c) + e_c, or -1 if none reaches the target.  The members are sorted
-// across the warp by (d, j) with a bitonic network, then an inclusive scan of
-// their masses in that order finds the crossing.
-__device__ __forceinline__ int topp_exact32(const ToppScratch& S, int cnt, unsigned long long base,
+// Warp-wide exclusive scan of small counts.
+__device__ __forceinline__ int warp_excl_scan(int c, int lane, int& total) {
+  int v = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  total = __shfl_sync(0xffffffffu, v, 31);
+  return v - c;
+}
+
+// A member record of the exact step: key, block, fixed-point mass.
+__device__ __forceinline__ uint4 member_record(const ToppScratch& S, uint32_t j) {
+  const uint32_t d = S.d[j];
+  return make_uint4(d, j, fixmass(key_value(d)), 0u);
+}
+
+// Writes the records of the (at most 32) blocks flagged in S.memw[0 .. nw) to
+// rec[0 .. cnt), in block order.
+__device__ __forceinline__ void list_flagged(const ToppScratch& S, int nw, uint4* rec, int lane) {
+  int base = 0;
+  for (int w0 = 0; w0 < nw; w0 += 32) {
+    uint32_t wv = w0 + lane < nw ? S.memw[w0 + lane] : 0u;
+    int tot;
+    int pos = base + warp_excl_scan(__popc(wv), lane, tot);
+    while (wv) {
+      const int b = __ffs(wv) - 1;
+      wv &= wv - 1u;
+      rec[pos++] = member_record(S, (uint32_t)((w0 + lane) * 32 + b));
+    }
+    base += tot;
+  }
+}
+
+// Writes the records of the (at most 32) blocks whose key lies in [rlo, rhi]
+// to rec[0 .. cnt), in block order (a scan over the row's n keys).
+__device__ __forceinline__ void list_range(const ToppScratch& S, int n, uint32_t rlo, uint32_t rhi, uint4* rec,
+                                           int lane) {
+  const unsigned lt = (1u << lane) - 1u;
+  int base = 0;
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    bool in = false;
+    if (j < n) {
+      const uint32_t d = S.d[j];
+      in = d >= rlo && d <= rhi;
+    }
+    const unsigned mk = __ballot_sync(0xffffffffu, in);
+    if (in) rec[base + __popc(mk & lt)] = member_record(S, (uint32_t)j);
+    base += __popc(mk);
+  }
+}
+
+// Exact crossing among `cnt` (<= 32) member records rec[], all ranked behind
+// mass `base`: returns the member c with ahead(c) < target <= ahead(c) + e_c
+// (ahead in (d, j) order), or -1 if none reaches the target.  The members are
+// sorted across the warp by (d, j) with a bitonic network, then an inclusive
+// scan of their masses in that order finds the crossing.
+__device__ __forceinline__ int topp_exact32(const uint4* rec, int cnt, unsigned long long base,
                                             unsigned long long target, int lane) {
   unsigned long long key = ~0ull;  // (d << 32) | j; absent members sort last
   if (lane < cnt) {
-    const int j = S.cand[lane];
-    key = ((unsigned long long)S.d[j] << 32) | (uint32_t)j;
+    const uint4 r = rec[lane];
+    key = ((unsigned long long)r.x << 32) | r.y;
   }
 #pragma unroll
   for (int k = 2; k <= 32; k <<= 1) {
@@ -585,12 +688,13 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
   const float m = rmax * kLog2e;
   uint32_t* hlo = reinterpret_cast<uint32_t*>(S.h);
   uint32_t* hhi = hlo + kTopPBins;
+  uint4* rec = reinterpret_cast<uint4*>(S.h);  // member records, over the bins once they are read
   // the 2 KB of bins zeroed with 16-byte stores
   for (int q = lane; q < 2 * kTopPBins / 4; q += 32) reinterpret_cast<uint4*>(hlo)[q] = make_uint4(0u, 0u, 0u, 0u);
   __syncwarp();
   // e_j, keys (in place of the logits), exact bin masses; only the
   // ceil(n / 32) slots the row has are visited
-  const int ns = (n + 31) >> 5;
+  const int ns = nw;
   auto hist1 = [&](int j, float x) {
     const float e = fast_exp2(fmaf(x, kLog2e, -m));
     const uint32_t d = rank_key(e);
@@ -642,47 +746,48 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
     xb = 8 * L + ub;
     base = before + __shfl_sync(0xffffffffu, pre - hb, ub);
   }
-  // one pass: keep the earlier bins, list the crossing bin's members; lane u
-  // collects mask word u of each batch
+  // one pass over the keys: blocks of earlier bins (key below the crossing
+  // bin's first key) are kept, the crossing bin's members flagged; lane u
+  // collects the words of slot u of each batch of 32 slots
+  const uint32_t key_lo = (uint32_t)xb << 19;
+  const uint32_t key_hi = xb == kTopPBins - 1 ? 0xffffffffu : ((uint32_t)(xb + 1) << 19);
   int cnt = 0;
   for (int u0 = 0; u0 < ns; u0 += 32) {
     const int u1 = min(u0 + 32, ns);
-    uint32_t myw = 0u;
-    auto sel = [&](int u, int b) {  // b: bin of block 32 u + lane (kTopPBins: none)
-      const unsigned mb = __ballot_sync(0xffffffffu, b < xb);
-      const bool in = b == xb;
-      const unsigned mi = __ballot_sync(0xffffffffu, in);
-      if (in) S.cand[cnt + __popc(mi & lt)] = (uint16_t)(u * 32 + lane);
-      cnt += __popc(mi);
-      if (lane == u - u0) myw = mb;
+    uint32_t myw = 0u, mym = 0u;
+    auto sel = [&](int uu, uint32_t d) {
+      const unsigned kb = __ballot_sync(0xffffffffu, d < key_lo);
+      const unsigned mb = __ballot_sync(0xffffffffu, d < key_hi) & ~kb;
+      if (lane == uu - u0) {
+        myw = kb;
+        mym = mb;
+      }
     };
     const int uf = min(u1, n >> 5);  // whole slots
-    int u = u0;
-#pragma unroll 4
-    for (; u < uf; ++u) sel(u, (int)min(S.d[u * 32 + lane] >> 19, (uint32_t)(kTopPBins - 1)));
-    for (; u < u1; ++u) {
-      const int j = u * 32 + lane;
-      sel(u, j < n ? (int)min(S.d[j] >> 19, (uint32_t)(kTopPBins - 1)) : kTopPBins);
+    int uu = u0;
+#pragma unroll 8
+    for (; uu < uf; ++uu) sel(uu, S.d[uu * 32 + lane]);
+    for (; uu < u1; ++uu) {
+      const int j = uu * 32 + lane;
+      sel(uu, j < n ? S.d[j] : 0xffffffffu);
     }
-    if (lane < u1 - u0) bits[u0 + lane] |= myw;  // slot u holds mask word u
+    if (lane < u1 - u0) {
+      bits[u0 + lane] |= myw;
+      S.memw[u0 + lane] = mym;
+    }
+    cnt += __reduce_add_sync(0xffffffffu, (unsigned)__popc(mym));
   }
   __syncwarp();
   if (cnt <= 32) {
     // member x is kept iff base + (mass of the members ranked ahead of it) <
-    // lim; the members are listed (key, j, mass) over the no longer needed
-    // bins and read back with broadcast loads
-    uint4* memb = reinterpret_cast<uint4*>(S.h);
-    uint4 me = make_uint4(0xffffffffu, 0x7fffffffu, 0u, 0u);
-    if (lane < cnt) {
-      const uint32_t jx = S.cand[lane], dx = S.d[jx];
-      me = make_uint4(dx, jx, fixmass(key_value(dx)), 0u);
-      memb[lane] = me;
-    }
+    // lim; the members' records are read back with broadcast loads
+    list_flagged(S, ns, rec, lane);
     __syncwarp();
+    const uint4 me = lane < cnt ? rec[lane] : make_uint4(0xffffffffu, 0x7fffffffu, 0u, 0u);
     unsigned long long ahead = base;
 #pragma unroll 4
     for (int y = 0; y < cnt; ++y) {
-      const uint4 o = memb[y];
+      const uint4 o = rec[y];
       if (o.x < me.x || (o.x == me.x && o.y < me.y)) ahead += o.z;
     }
     if (lane < cnt && ahead < lim) atomicOr(&bits[me.y >> 5], 1u << (me.y & 31));
@@ -690,9 +795,10 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
     return;
   }
   // refine on lower key bits, 8-bit digits: a regular bin spans 2^19 keys
-  // (digits at shifts 11, 3, 0), the catch-all bin up to 2^30 (22, 14, 6, 0)
+  // (digits at shifts 11, 3, 0), the catch-all bin up to 2^30 (22, 14, 6, 0).
+  // The members are the row's keys in [rlo, rhi], found by scanning the keys.
   int cross = -1;
-  uint32_t lo_key = (uint32_t)xb << 19;
+  uint32_t rlo = key_lo, rhi = key_hi - 1u;
   const bool wide = xb == kTopPBins - 1;
   for (int level = 0;; ++level) {
     const int sh = wide ? (level == 0 ? 22 : level == 1 ? 14 : level == 2 ? 6 : 0)
@@ -702,44 +808,42 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
       hhi[b] = 0u;
     }
     __syncwarp();
-    for (int x0 = 0; x0 < cnt; x0 += 32) {
-      const int x = x0 + lane;
-      if (x < cnt) {
-        const uint32_t d = S.d[S.cand[x]];
-        bin_add(hlo, hhi, (int)min((d - lo_key) >> sh, (uint32_t)(kTopPBins - 1)), fixmass(key_value(d)));
-      }
+    for (int j = lane; j < n; j += 32) {
+      const uint32_t d = S.d[j];
+      if (d >= rlo && d <= rhi)
+        bin_add(hlo, hhi, (int)min((d - rlo) >> sh, (uint32_t)(kTopPBins - 1)), fixmass(key_value(d)));
     }
     __syncwarp();
     unsigned long long h2[8], t2 = 0ull;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      h2[u] = bin_mass(hlo, hhi, lane * 8 + u);
-      t2 += h2[u];
+    for (int q = 0; q < 8; ++q) {
+      h2[q] = bin_mass(hlo, hhi, lane * 8 + q);
+      t2 += h2[q];
     }
     const unsigned long long inc2 = warp_scan_u64(t2, lane);
     unsigned long long run = inc2 - t2;
     int bin2 = -1;
     unsigned long long bb = 0ull;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (bin2 < 0 && base + run + h2[u] >= target && h2[u] > 0ull) {
-        bin2 = lane * 8 + u;
+    for (int q = 0; q < 8; ++q) {
+      if (bin2 < 0 && base + run + h2[q] >= target && h2[q] > 0ull) {
+        bin2 = lane * 8 + q;
         bb = base + run;
       }
-      run += h2[u];
+      run += h2[q];
     }
     const unsigned f2 = __ballot_sync(0xffffffffu, bin2 >= 0);
+    __syncwarp();  // the bins are read before the member records overwrite them
     if (f2 == 0u) {
       // (exact sums make this unreachable) the members' mass stays below
       // the target: all of them are kept -- the cut is the last member
       uint32_t bd = 0u;
       int bj = -1;
-      for (int x = lane; x < cnt; x += 32) {
-        const int jj = S.cand[x];
-        const uint32_t dd = S.d[jj];
-        if (bj < 0 || dd > bd || (dd == bd && jj > bj)) {
+      for (int j = lane; j < n; j += 32) {
+        const uint32_t dd = S.d[j];
+        if (dd >= rlo && dd <= rhi && (bj < 0 || dd > bd || (dd == bd && j > bj))) {
           bd = dd;
-          bj = jj;
+          bj = j;
         }
       }
 #pragma unroll
@@ -757,28 +861,25 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
     const int sl = __ffs(f2) - 1;
     const int xb2 = __shfl_sync(0xffffffffu, bin2, sl);
     base = __shfl_sync(0xffffffffu, bb, sl);
-    const uint32_t blo = lo_key + ((uint32_t)xb2 << sh);
-    const uint32_t bhi = sh == 0 ? blo : blo + ((1u << sh) - 1u);
+    const uint32_t blo = rlo + ((uint32_t)xb2 << sh);
+    // the last digit bin also holds every key above its start
+    const uint32_t bhi = sh == 0 ? blo : (xb2 == kTopPBins - 1 ? rhi : blo + ((1u << sh) - 1u));
     int c2 = 0;
-    for (int x0 = 0; x0 < cnt; x0 += 32) {
-      const int x = x0 + lane;
-      int jj = 0;
+    for (int j0 = 0; j0 < n; j0 += 32) {
+      const int j = j0 + lane;
       bool in = false;
-      if (x < cnt) {
-        jj = S.cand[x];
-        const uint32_t d = S.d[jj];
+      if (j < n) {
+        const uint32_t d = S.d[j];
         in = d >= blo && d <= bhi;
       }
-      const unsigned mk = __ballot_sync(0xffffffffu, in);
-      __syncwarp();
-      if (in) S.cand[c2 + __popc(mk & lt)] = (uint16_t)jj;
-      c2 += __popc(mk);
+      c2 += __popc(__ballot_sync(0xffffffffu, in));
     }
-    __syncwarp();
-    cnt = c2;
-    lo_key = blo;
-    if (cnt <= 32) {
-      cross = topp_exact32(S, cnt, base, target, lane);
+    rlo = blo;
+    rhi = bhi;
+    if (c2 <= 32) {
+      list_range(S, n, rlo, rhi, rec, lane);
+      __syncwarp();
+      cross = topp_exact32(rec, c2, base, target, lane);
       break;
     }
     if (sh == 0) {
@@ -786,14 +887,14 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
       // reaches the target
       const unsigned long long me = (unsigned long long)fixmass(key_value(blo));
       unsigned long long acc = base;
-      for (int x0 = 0; x0 < cnt && cross < 0; x0 += 32) {
-        const int x = x0 + lane;
-        const bool ok = x < cnt;
+      for (int j0 = 0; j0 < n && cross < 0; j0 += 32) {
+        const int j = j0 + lane;
+        const bool ok = j < n && S.d[j] == blo;
         const unsigned mk = __ballot_sync(0xffffffffu, ok);
         const int pos = __popc(mk & lt);
         const bool hit = ok && acc + me * (unsigned long long)(pos + 1) >= target;
         const unsigned hm = __ballot_sync(0xffffffffu, hit);
-        if (hm) cross = __shfl_sync(0xffffffffu, ok ? (int)S.cand[x] : 0, __ffs(hm) - 1);
+        if (hm) cross = __shfl_sync(0xffffffffu, j, __ffs(hm) - 1);
         acc += me * (unsigned long long)__popc(mk);
       }
       break;
@@ -864,13 +965,17 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int bi = g / P.hkv, kv = g - bi * P.hkv;
   const int nchunk = (P.nb + kScoreRows - 1) / kScoreRows;
-  const int chunk = nchunk - 1 - y / P.G;  // longest rows first
+  int chunk, part;
+  score_part_of(P, y / P.G, chunk, part);  // longest rows first
   const int bh = bi * P.hq + kv * P.G + y % P.G;
   const int i0 = chunk * kScoreRows;
   const int max_i = min(P.nb, i0 + kScoreRows) - 1;
   const uint32_t nch = (uint32_t)P.bl.dp / 64;
   const int ncolw = score_cols(P.bl.dp);  // N: key blocks per column chunk
-  const int ncol = max_i / ncolw + 1;
+  // this part's key blocks [j0, j1): column chunks c0 .. c0 + ncol - 1
+  const int j0 = part * kScorePartBlocks, j1 = min(j0 + kScorePartBlocks, max_i + 1);
+  const int c0 = j0 / ncolw;
+  const int ncol = (j1 - 1) / ncolw + 1 - c0;
   const int units = 3 * ncol;
   const uint32_t idesc = ncolw == 128 ? idesc_bf16_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 64, 0, 0);
   const uint32_t sbase = (smem_u32(smem) + 1023u) & ~1023u;
@@ -908,7 +1013,7 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
         mbar_arrive_expect_tx(bar_b(u), slot_bytes);
         for (uint32_t k = 0; k < nch; ++k)
           tma_load_2d(slot_addr(u) + k * (uint32_t)ncolw * 128, &tm[term + (ncolw == 128 ? 0 : 3)],
-                      (int)(64 * k), brow0 + c * ncolw, bar_b(u));
+                      (int)(64 * k), brow0 + (c0 + c) * ncolw, bar_b(u));
       }
       for (int u = max(units - kBSlots, 0); u < units; ++u) {  // the last releases
         mbar_wait(bar_f(u), (ps.free >> (u % kBSlots)) & 1u);
@@ -967,7 +1072,7 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
           tmem_wait_ld_dep16(vl);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const int j = c * ncolw + col0 + 8 * k + cq;  // key block of the first value
+            const int j = (c0 + c) * ncolw + col0 + 8 * k + cq;  // key block of the first value
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
               const int rl = q4 * 32 + lh * 16 + gr + 8 * rr;  // row in the item
@@ -1014,16 +1119,17 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
     }
   }
   named_barrier(kBarStream, kStreamThreads);  // score tiles and row maxima complete
-  // publish: the chunk's row maxima, then "chunk scored" for its Top-P items
+  // publish: the part's row maxima, then count the part for the chunk's Top-P items
   const int st = stream_tid(t);
   if (st < 256) {
     const int rl = st & 127, band = st >> 7, i = i0 + rl;
-    if (i <= max_i) P.rmax[((size_t)bh * P.nb + i) * 2 + band] = fmaxf(sm.rmax[0][band][rl], sm.rmax[1][band][rl]);
+    if (i <= max_i)
+      P.rmax[(((size_t)bh * P.nb + i) * P.rparts + part) * 2 + band] = fmaxf(sm.rmax[0][band][rl], sm.rmax[1][band][rl]);
   }
   named_barrier(kBarStream, kStreamThreads);
   if (t == 0) {
     __threadfence();
-    st_release_gpu(&P.sync[2 + 2 * P.n_groups + bh * nchunk + chunk], 1u);
+    red_release_gpu_add(&P.sync[2 + 2 * P.n_groups + bh * nchunk + chunk], 1u);
   }
   named_barrier(kBarStream, kStreamThreads);  // shared memory is reused by the next item
 }
@@ -1057,9 +1163,10 @@ __device__ __forceinline__ void topp_item(const EstParams& P, int g, int y, cons
   const int nbp = (P.nb + 7) & ~7;
   const int nbuf = T.single ? 1 : 2;
   ToppScratch S;
-  S.cand = reinterpret_cast<uint16_t*>(wb + (size_t)nbp * 4 * nbuf);
-  S.h = reinterpret_cast<unsigned long long*>(wb + (size_t)nbp * (4 * nbuf + 2));
-  uint32_t* bits = reinterpret_cast<uint32_t*>(wb + (size_t)nbp * (4 * nbuf + 2) + kTopPBins * 8);
+  // per warp: nbuf logit rows | bins (2 KB) | member words | bit row
+  S.h = reinterpret_cast<unsigned long long*>(wb + (size_t)nbp * 4 * nbuf);
+  S.memw = reinterpret_cast<uint32_t*>(wb + (size_t)nbp * 4 * nbuf + kTopPBins * 8);
+  uint32_t* bits = S.memw + nbp / 32 + 1;
   const int nrows = max_i - r0 - T.lw >= 0 ? (max_i - r0 - T.lw) / T.nw + 1 : 0;
   const int ntasks = 2 * nrows;
   const float* tiles = score_tile(P, bh, chunk, 0);
@@ -1073,11 +1180,15 @@ __device__ __forceinline__ void topp_item(const EstParams& P, int g, int y, cons
   };
   if (!T.single && ntasks > 0) fetch(0);
   // row maxima of the warp's first 32 tasks, one per lane, loaded up front
+  const int np = score_parts(chunk);
+  auto row_max = [&](int i, int band) {  // over the score parts of the row
+    const float* r = P.rmax + ((size_t)bh * P.nb + i) * P.rparts * 2 + band;
+    float m = r[0];
+    for (int q = 1; q < np; ++q) m = fmaxf(m, r[2 * q]);
+    return m;
+  };
   float my_rmax = 0.f;
-  if (lane < ntasks) {
-    const int i = r0 + T.lw + (lane >> 1) * T.nw;
-    my_rmax = P.rmax[((size_t)bh * P.nb + i) * 2 + (lane & 1)];
-  }
+  if (lane < ntasks) my_rmax = row_max(r0 + T.lw + (lane >> 1) * T.nw, lane & 1);
   for (int task = 0; task < ntasks; ++task) {
     if (T.single) {
       fetch(task);  // the buffer is free: the last task ended with __syncwarp
@@ -1093,7 +1204,7 @@ __device__ __forceinline__ void topp_item(const EstParams& P, int g, int y, cons
     const int i = r0 + T.lw + (task >> 1) * T.nw, band = task & 1;
     const int n = i + 1;
     const float rmax_t = __shfl_sync(0xffffffffu, my_rmax, task & 31);
-    const float rmax = task < 32 ? rmax_t : P.rmax[((size_t)bh * P.nb + i) * 2 + band];
+    const float rmax = task < 32 ? rmax_t : row_max(i, band);
     S.d = reinterpret_cast<uint32_t*>(wb + (size_t)(task & (nbuf - 1)) * nbp * 4);
     float* dbg = P.dbg_scores ? P.dbg_scores + (size_t)bh * 2 * tri + (size_t)band * tri + (size_t)i * (i + 1) / 2
                               : nullptr;
@@ -1130,7 +1241,8 @@ __device__ __forceinline__ void topp_loop(const EstParams& P, const ToppTeam& T,
       if (decode_topp(P, x, g, y) == kItemTopp) {
         const int bh = (g / P.hkv) * P.hq + (g % P.hkv) * P.G + y % P.G;
         const int chunk = (nseg - 1 - y / P.G) * kToppRows / kScoreRows;
-        ok = flag_wait_ns(&P.sync[2 + 2 * P.n_groups + bh * nchunk + chunk], kWaitLimitNs) ? 1 : 0;
+        ok = count_wait_ns(&P.sync[2 + 2 * P.n_groups + bh * nchunk + chunk], (uint32_t)score_parts(chunk),
+                           kWaitLimitNs) ? 1 : 0;
       }
       *s_item = x;
       *s_ok = ok;
@@ -1153,7 +1265,7 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
   __shared__ PoolSmem psm;
   __shared__ int s_next, s_ok, s_titem[2], s_tok[2];
   const int stages = P.pool_stages;
-  PoolState pst = {0u, 0u, 0u, 0};
+  PoolState pst = {0u, 0u, 0u, 0u, 0};
   ScoreState ss = {0u, 0u, 0u, 0u, 0u};
   for (int i = threadIdx.x; i < 16 * 32; i += kEstThreads) psm.ones[i] = 0x3F803F80u;  // bf16 1.0 pairs
   fence_proxy_async_smem();  // read by the tensor cores
@@ -1163,6 +1275,7 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
       mbar_init(smem_u32(&psm.bars_free[st]), 1u);
     }
     mbar_init(smem_u32(&psm.bar_pool), 1u);
+    mbar_init(smem_u32(&psm.bar_pool_half), 1u);
     mbar_init(smem_u32(&psm.bar_a), 1u);
     for (int sl = 0; sl < kBSlots; ++sl) {
       mbar_init(smem_u32(&psm.bar_b[sl]), 1u);

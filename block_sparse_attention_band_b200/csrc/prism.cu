@@ -120,11 +120,11 @@ int validate(const prism_config* cfg, Plan* pl) {
   const size_t nch = ((size_t)P.nb + 127) / 128;
   off = align_up(off + (size_t)P.q_rows * (nch * (nch + 1) / 2) * 2 * 128 * 128 * sizeof(float), 256);
   P.off_rmax = off;
-  off = align_up(off + (size_t)P.q_rows * P.nb * 2 * sizeof(float), 256);
+  off = align_up(off + (size_t)P.q_rows * P.nb * score_parts((int)nch - 1) * 2 * sizeof(float), 256);
   P.off_mask = off;
   off = align_up(off + (size_t)P.q_rows * P.nb * P.W * sizeof(uint32_t), 256);
   P.off_sync = off;
-  // queue head, per-group counters and ready flags, per (batch, Q head, score chunk) flags
+  // queue heads, per-group counters and ready flags, per (batch, Q head, score chunk) part counters
   P.sync_bytes = (2 + 2 * (size_t)P.kv_rows + (size_t)P.q_rows * nch) * sizeof(uint32_t);
   off = align_up(off + P.sync_bytes, 256);
   P.total = off;
@@ -153,11 +153,11 @@ struct EstLaunch {
   size_t stream, smem;
   int stages;
 };
-// Per Top-P warp: one or two logit rows (keys replace the logits in place), a
-// u16 member list, 256 64-bit bins and one bit row.
+// Per Top-P warp: one or two logit rows (keys replace the logits in place),
+// 256 64-bit bins, a member bit row and the mask bit row.
 static size_t topp_stride(int nb, bool single) {
   const size_t W = ((size_t)nb + 31) / 32, nbp = ((size_t)nb + 7) & ~(size_t)7;
-  return align_up(nbp * (single ? 6 : 10) + 256 * 8 + W * 4, 16);
+  return align_up(nbp * 4 * (single ? 1 : 2) + 256 * 8 + (nbp / 32 + 1) * 4 + W * 4, 16);
 }
 // Fills L; false if not even one Top-P warp fits beside the product operands.
 bool est_launch_shape(int nb, int dp, EstLaunch& L) {
@@ -314,7 +314,13 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   E.n_groups = P.kv_rows;
   E.pool_item_span = (P.nb + kPoolTilesPerItem - 1) / kPoolTilesPerItem;
   E.pool_items = (E.G + 1) * E.pool_item_span;
-  E.score_items = E.G * ((P.nb + kScoreRows - 1) / kScoreRows);
+  {
+    const int nchunk = (P.nb + kScoreRows - 1) / kScoreRows;
+    E.score_span = 0;
+    for (int c = 0; c < nchunk; ++c) E.score_span += score_parts(c);
+    E.score_items = E.G * E.score_span;
+    E.rparts = score_parts(nchunk - 1);
+  }
   E.topp_items = E.G * ((P.nb + kToppRows - 1) / kToppRows);
   EstLaunch L;
   if (!est_launch_shape(P.nb, P.bl.dp, L)) return PRISM_ERR_UNSUPPORTED;

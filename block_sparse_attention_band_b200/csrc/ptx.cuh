@@ -94,6 +94,22 @@ __device__ __forceinline__ bool flag_wait_ns(const uint32_t* flag, uint64_t limi
   }
 }
 
+// The same for a counter that must reach `target`.
+__device__ __forceinline__ bool count_wait_ns(const uint32_t* ctr, uint32_t target, uint64_t limit_ns) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+  if (v >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      set_device_error(kDevErrTimeout);
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // fences
 // ---------------------------------------------------------------------------

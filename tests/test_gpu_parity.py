@@ -208,6 +208,50 @@ def test_rope_layout_presets(layout, cuda_device):
     P.check_attention_rows(o, q, k, v, mask, rows, w.hq // w.hkv)
 
 
+def _crowded_inputs(kind: str, nb: int, seed: int):
+    """Q, K (bf16, [1, 2, N, 128] / [1, 1, N, 128]) whose pooled logits tie or
+    crowd into one Top-P bin: every K token of block j is c + s * r_j, so the
+    pooled K rows differ only by s * r_j (s = 0: exact ties in every row);
+    "mixed" keeps random K tokens in the second half of the blocks."""
+    g = torch.Generator("cpu")
+    g.manual_seed(seed)
+    n = nb * 128
+    a_q = torch.randn(2, 1, 128, generator=g)
+    q = (a_q + 0.5 * torch.randn(2, n, 128, generator=g)).to(torch.bfloat16)[None]
+    c = torch.randn(1, 128, generator=g)
+    r = torch.randn(nb, 128, generator=g)
+    s = {"ties": 0.0, "crowded": 0.005, "mixed": 0.005}[kind]
+    kb = c + s * r  # [nb, 128]
+    k = kb.repeat_interleave(128, dim=0)[None]  # [1, N, 128]
+    if kind == "mixed":
+        k[:, n // 2:] = torch.randn(1, n - n // 2, 128, generator=g)
+    return q, k.to(torch.bfloat16)[None]
+
+
+@pytest.mark.parametrize("kind", ["ties", "crowded", "mixed"])
+def test_topp_ties_and_crowded_bins(kind, cuda_device):
+    """Rows whose blocks share (or nearly share) one logit: the crossing bin
+    holds many members, so the exact Top-P refines on lower key bits and, for
+    equal keys, cuts by block index -- the oracle's stable order."""
+    nb, p = 40, 0.91
+    q, k = _crowded_inputs(kind, nb, seed=71 + len(kind))
+    w = gen.small_workload(f"crowd_{kind}", 1, 2, 1, nb * 128, seed=0, p=p)
+    cfg = P.make_cfg(w)
+    mask, sc, tau, _ = P.run_estimate(cfg, q.to(cuda_device), k.to(cuda_device))
+    hi, lo = gen.default_bands()
+    ref = oracle.estimate(q, k, hi, lo, p)
+    P.check_tau(tau, ref)
+    P.check_scores(sc, ref)
+    P.check_mask(mask, ref, p)
+    self_mask, self_cx = P.topp_on_scores(sc, p)
+    near = (np.abs(self_cx[..., 0, :, :] - p) < P.SELF_WINDOW) | (np.abs(self_cx[..., 1, :, :] - p) < P.SELF_WINDOW)
+    assert not np.any((self_mask != mask) & ~near)
+    if kind == "ties":  # every row keeps exactly its first ceil(p (i + 1)) blocks
+        for i in range(nb):
+            keep = int(np.ceil(p * (i + 1) - 1e-9))
+            assert mask[0, 0, i, :keep].all() and not mask[0, 0, i, keep:].any(), i
+
+
 def test_small_p_sparse_rows(cuda_device):
     w = gen.small_workload("sparse_nb48", 1, 2, 1, 48 * 128, seed=35, p=0.3)
     q, k, v, qd, kd, vd = _inputs(w, cuda_device)
