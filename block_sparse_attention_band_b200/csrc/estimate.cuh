@@ -67,21 +67,21 @@ __host__ __device__ constexpr int gemm_smem_bytes(int dp) {
 constexpr int kGemmSmemBytes = gemm_smem_bytes(192);  // the largest layout: 144 + 2 x 24 KB + alignment
 
 // The CTA's warps form two lanes that take items from two queues at once:
-// the stream lane (warps 0, 1, 4-11) runs pool and score items, the Top-P
-// lane (warps 2, 3, 12-15) runs Top-P items, so the Top-P work of earlier
+// the stream lane (warps 0, 1, 4-7) runs pool and score items, the Top-P
+// lane (warps 2, 3, 8-15) runs Top-P items, so the Top-P work of earlier
 // groups proceeds on the CUDA cores while the same SM streams Q and K.  Once
 // the stream queue is empty the stream lane's warps take Top-P items too.
 // Each lane synchronises on its own named barrier (1 is the pool read-out
 // warps' own).
-constexpr int kStreamThreads = 320;  // warps 0, 1, 4-11
-constexpr int kLaneThreads = 192;    // warps 2, 3, 12-15
+constexpr int kStreamThreads = 192;  // warps 0, 1, 4-7
+constexpr int kLaneThreads = 320;    // warps 2, 3, 8-15
 constexpr int kLaneWarpsMax = kLaneThreads / 32;
 constexpr int kTeamWarpsMax = kStreamThreads / 32;
 enum : int { kBarStream = 2, kBarLane = 3 };
-__device__ __forceinline__ bool in_stream_lane(int warp) { return warp < 2 || (warp >= 4 && warp < 12); }
-__device__ __forceinline__ int stream_tid(int t) { return t < 64 ? t : t - 64; }        // 0 .. 319
-__device__ __forceinline__ int stream_warp(int warp) { return warp < 2 ? warp : warp - 2; }  // 0 .. 9
-__device__ __forceinline__ int lane_warp(int warp) { return warp < 4 ? warp - 2 : warp - 10; }  // 0 .. 5
+__device__ __forceinline__ bool in_stream_lane(int warp) { return warp < 2 || (warp >= 4 && warp < 8); }
+__device__ __forceinline__ int stream_tid(int t) { return t < 64 ? t : t - 64; }            // 0 .. 191
+__device__ __forceinline__ int stream_warp(int warp) { return warp < 2 ? warp : warp - 2; }  // 0 .. 5
+__device__ __forceinline__ int lane_warp(int warp) { return warp < 4 ? warp - 2 : warp - 6; }    // 0 .. 9
 constexpr int kMaxGroupHeads = 64;    // Q heads per KV head supported by the tau step
 constexpr int kTauBatch = 5;          // head rows whose energy partials the tau step sums at once
 constexpr float kLog2e = 1.4426950408889634f;
@@ -922,7 +922,7 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
 // chunks of N = 128 (64 for the widest band layout).  Step (5): logits of
 // both bands on the tensor cores, accumulators in tensor memory, double
 // buffered; warp roles: warp 0 lane 0 streams the operands (TMA), warp 1
-// lane 0 issues the products, warps 4-11 read the accumulators of a finished
+// lane 0 issues the products, warps 4-7 read the accumulators of a finished
 // chunk, scale them, write the score tiles and keep the row maxima.  The
 // chunk's rows then wait for a Top-P item (steps 5-7 per row).
 // ---------------------------------------------------------------------------
@@ -1044,15 +1044,14 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
         ps.acc ^= 1u << (c & 1);
       }
     }
-  } else if (warp >= 4 && warp < 12) {
-    // warp w reads TMEM lane quarter w % 4 and column half (w - 4) / 4 in the
-    // 16 x 256-bit shape: four threads share a row, each holding two adjacent
+  } else if (warp >= 4 && warp < 8) {
+    // warp w reads TMEM lane quarter w % 4 in the 16 x 256-bit shape, 32
+    // columns at a time: four threads share a row, each holding two adjacent
     // key blocks, so every store instruction writes eight whole 32-byte
     // sectors of the score tiles.  The row maxima over j <= i are kept too.
     const float sc_hi = P.tau[bh * 4 + 2], sc_lo = P.tau[bh * 4 + 3];
-    const int q4 = warp & 3, h = (warp - 4) >> 2;
+    const int q4 = warp & 3;
     const int gr = lane >> 2, cq = (lane & 3) * 2;
-    const int hw = ncolw / 2;
     float mx[2][2][2];  // [lane half][row of the pair][band]
 #pragma unroll
     for (int a = 0; a < 8; ++a) (&mx[0][0][0])[a] = -INFINITY;
@@ -1062,8 +1061,8 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
       tc_fence_after();
 #pragma unroll
       for (int lh = 0; lh < 2; ++lh) {
-        for (int grp = 0; grp < hw; grp += 32) {
-          const int col0 = h * hw + grp;  // column in the chunk
+#pragma unroll 1
+        for (int col0 = 0; col0 < ncolw; col0 += 32) {  // column in the chunk
           const uint32_t taddr = dacc(c) + ((uint32_t)(q4 * 32 + lh * 16) << 16) + (uint32_t)col0;
           uint32_t vh[16], vl[16];
           tmem_ld_16x256b_x4(taddr, vh);
@@ -1113,16 +1112,16 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
           const int rl = q4 * 32 + lh * 16 + gr + 8 * rr;
-          sm.rmax[h][0][rl] = mx[lh][rr][0];
-          sm.rmax[h][1][rl] = mx[lh][rr][1];
+          sm.rmax[0][0][rl] = sm.rmax[1][0][rl] = mx[lh][rr][0];
+          sm.rmax[0][1][rl] = sm.rmax[1][1][rl] = mx[lh][rr][1];
         }
     }
   }
   named_barrier(kBarStream, kStreamThreads);  // score tiles and row maxima complete
   // publish: the part's row maxima, then count the part for the chunk's Top-P items
   const int st = stream_tid(t);
-  if (st < 256) {
-    const int rl = st & 127, band = st >> 7, i = i0 + rl;
+  for (int q = st; q < 256; q += kStreamThreads) {
+    const int rl = q & 127, band = q >> 7, i = i0 + rl;
     if (i <= max_i)
       P.rmax[(((size_t)bh * P.nb + i) * P.rparts + part) * 2 + band] = fmaxf(sm.rmax[0][band][rl], sm.rmax[1][band][rl]);
   }
@@ -1283,8 +1282,8 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
     }
     mbar_init(smem_u32(&psm.bar_mma[0]), 1u);
     mbar_init(smem_u32(&psm.bar_mma[1]), 1u);
-    mbar_init(smem_u32(&psm.bar_acc[0]), 8u);  // one arrival per read-out warp
-    mbar_init(smem_u32(&psm.bar_acc[1]), 8u);
+    mbar_init(smem_u32(&psm.bar_acc[0]), 4u);  // one arrival per read-out warp
+    mbar_init(smem_u32(&psm.bar_acc[1]), 4u);
     fence_mbar_init();
     for (int m = 0; m < 8; ++m) tma_prefetch_desc(&tms.m[m]);
   }
