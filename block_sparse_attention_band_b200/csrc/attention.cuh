@@ -78,7 +78,7 @@ struct Tile {
   uint32_t last_mask;
   __device__ __forceinline__ uint32_t word(int w) const {
     if (!valid || w > last_word) return 0u;
-    const uint32_t b = mrow[w];
+    const uint32_t b = __ldcg(mrow + w);  // L2: the mask may have been written during this launch
     return w == last_word ? (b & last_mask) : b;
   }
 };
@@ -214,9 +214,10 @@ __device__ __forceinline__ float softmax_p(const uint32_t (&sv)[128], uint32_t t
 
 __global__ void __launch_bounds__(kThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const uint32_t* __restrict__ mask,
+                   const __grid_constant__ CUtensorMap tmV, const uint32_t* mask,
                    __nv_bfloat16* __restrict__ out, int batch, int hq, int hkv, int seqlen, int nb,
-                   float scale_log2) {
+                   float scale_log2, const uint32_t* ready, int ready_rows) {
+  __shared__ int s_masks_ok;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -249,9 +250,22 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tmem_alloc(smem_u32(tmem_holder), kTmemCols);
     tmem_relinquish();
   }
+  if (threadIdx.x == 0) {
+    // launched while the estimator still runs: wait (bounded) until the
+    // estimator has published the mask rows of both tiles
+    int ok = 1;
+    if (ready) {
+      const int nseg = (nb + ready_rows - 1) / ready_rows;
+      for (int x = 0; x < 2; ++x)
+        if (ok && tiles[x].valid)
+          ok = flag_wait_ns(&ready[(size_t)tiles[x].bh * nseg + tiles[x].i / ready_rows], kWaitLimitNs) ? 1 : 0;
+    }
+    s_masks_ok = ok;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (!s_masks_ok) tiles[0].valid = tiles[1].valid = 0;  // (timed out: error recorded, no work)
   const uint32_t tmem = *tmem_holder;
   // Each warpgroup sets its register budget first and then runs only its own
   // roles (no code is shared across the split); warp 1 frees tensor memory

@@ -105,6 +105,7 @@ struct EstParams {
   float* dbg_tau;
   float* rmax;     // [q_rows, nb, rparts, 2] scaled band logits' row maxima over the key blocks j <= i
                    // of each part
+  uint32_t* ready;  // [q_rows, ceil(nb / kToppRows)] mask rows of a Top-P item written
   uint32_t* sync;  // [0] stream queue head, [1] Top-P queue head, [2 + g] pool items done,
                    // [2 + n_groups + g] group ready,
                    // [2 + 2 n_groups + bh * nchunk + c] parts of score chunk c of (batch, Q head) bh written
@@ -1252,6 +1253,11 @@ __device__ __forceinline__ void topp_loop(const EstParams& P, const ToppTeam& T,
     if (decode_topp(P, x, g, y) == kItemNone) break;  // no thread passes a barrier after this
     if (ok) topp_item(P, g, y, T);
     named_barrier(bar, nthreads);  // the item's shared memory and s_item are reused
+    if (leader && ok) {  // the item's mask rows are final: attention may read them
+      const int bh = (g / P.hkv) * P.hq + (g % P.hkv) * P.G + y % P.G;
+      __threadfence();
+      st_release_gpu(&P.ready[(size_t)bh * nseg + (nseg - 1 - y / P.G)], 1u);
+    }
   }
 }
 
@@ -1262,6 +1268,10 @@ __global__ void __launch_bounds__(kEstThreads, 1)
 estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ TermMaps tms) {
   extern __shared__ __align__(16) unsigned char est_smem[];
   __shared__ PoolSmem psm;
+  // a kernel launched after this one with programmatic serialization (the
+  // attention of a prefill) may be scheduled on SMs this grid leaves; it
+  // waits for the mask rows it reads through the `ready` flags
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ int s_next, s_ok, s_titem[2], s_tok[2];
   const int stages = P.pool_stages;
   PoolState pst = {0u, 0u, 0u, 0u, 0};

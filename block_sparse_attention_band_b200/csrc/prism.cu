@@ -124,8 +124,11 @@ int validate(const prism_config* cfg, Plan* pl) {
   P.off_mask = off;
   off = align_up(off + (size_t)P.q_rows * P.nb * P.W * sizeof(uint32_t), 256);
   P.off_sync = off;
-  // queue heads, per-group counters and ready flags, per (batch, Q head, score chunk) part counters
-  P.sync_bytes = (2 + 2 * (size_t)P.kv_rows + (size_t)P.q_rows * nch) * sizeof(uint32_t);
+  // queue heads, per-group counters and ready flags, per (batch, Q head, score chunk) part counters,
+  // per (batch, Q head, Top-P segment) mask-rows-written flags
+  P.sync_bytes = (2 + 2 * (size_t)P.kv_rows + (size_t)P.q_rows * nch +
+                  (size_t)P.q_rows * (((size_t)P.nb + kToppRows - 1) / kToppRows)) *
+                 sizeof(uint32_t);
   off = align_up(off + P.sync_bytes, 256);
   P.total = off;
   return PRISM_OK;
@@ -289,6 +292,12 @@ int launched() { return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR
 // ---------------------------------------------------------------------------
 // launch sequences
 // ---------------------------------------------------------------------------
+// Word offset of the mask-rows-written flags in the estimator's sync region.
+size_t ready_offset(const Plan& P) {
+  const size_t nch = ((size_t)P.nb + 127) / 128;
+  return 2 + 2 * (size_t)P.kv_rows + (size_t)P.q_rows * nch;
+}
+
 int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, unsigned char* ws,
                  cudaStream_t st, float* dbg_scores, float* dbg_tau) {
   EstParams E;
@@ -304,6 +313,7 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   E.dbg_tau = dbg_tau;
   E.rmax = reinterpret_cast<float*>(ws + P.off_rmax);
   E.sync = reinterpret_cast<uint32_t*>(ws + P.off_sync);
+  E.ready = E.sync + ready_offset(P);
   E.hq = P.hq;
   E.hkv = P.hkv;
   E.G = P.hq / P.hkv;
@@ -364,8 +374,11 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   return launched();
 }
 
+// `ready` (nullable): the estimator's per-segment mask flags; then the kernel
+// is launched with programmatic serialization, so it may start on SMs the
+// estimator has left while that still finishes other rows.
 int run_attention(const Plan& P, const void* q, const void* k, const void* v, const uint32_t* mask,
-                  void* o, cudaStream_t st) {
+                  void* o, cudaStream_t st, const uint32_t* ready = nullptr) {
   CUtensorMap mq, mk, mv;
   if (make_map_tokens(&mq, q, (size_t)P.q_rows, (size_t)P.n) != PRISM_OK ||
       make_map_tokens(&mk, k, (size_t)P.kv_rows, (size_t)P.n) != PRISM_OK ||
@@ -373,8 +386,25 @@ int run_attention(const Plan& P, const void* q, const void* k, const void* v, co
     return PRISM_ERR_CUDA;
   const float scale_log2 = P.scale * 1.4426950408889634f;
   const unsigned grid = attn::grid_size(P.b, P.hq, P.hkv, P.nb);
-  attn::sparse_attn_kernel<<<grid, attn::kThreads, attn::kSmemBytes, st>>>(
-      mq, mk, mv, mask, reinterpret_cast<__nv_bfloat16*>(o), P.b, P.hq, P.hkv, P.n, P.nb, scale_log2);
+  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(o);
+  if (!ready) {
+    attn::sparse_attn_kernel<<<grid, attn::kThreads, attn::kSmemBytes, st>>>(
+        mq, mk, mv, mask, out, P.b, P.hq, P.hkv, P.n, P.nb, scale_log2, nullptr, kToppRows);
+    return launched();
+  }
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(grid);
+  lc.blockDim = dim3(attn::kThreads);
+  lc.dynamicSmemBytes = attn::kSmemBytes;
+  lc.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  if (cudaLaunchKernelEx(&lc, attn::sparse_attn_kernel, mq, mk, mv, mask, out, P.b, P.hq, P.hkv, P.n, P.nb,
+                         scale_log2, ready, kToppRows) != cudaSuccess)
+    return PRISM_ERR_CUDA;
   return launched();
 }
 
@@ -484,7 +514,10 @@ int prism_prefill(const prism_config* cfg, const void* q, const void* k, const v
   uint32_t* mask = mask_out ? mask_out : reinterpret_cast<uint32_t*>(ws + P.off_mask);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if ((s = run_estimate(P, q, k, mask, ws, st, nullptr, nullptr)) != PRISM_OK) return s;
-  return run_attention(P, q, k, v, mask, o, st);
+  // the attention starts on query blocks whose masks are final while the
+  // estimator finishes the others
+  const uint32_t* ready = reinterpret_cast<const uint32_t*>(ws + P.off_sync) + ready_offset(P);
+  return run_attention(P, q, k, v, mask, o, st, ready);
 }
 
 // Same estimator as prism_estimate, with the library's built-in scratch array in

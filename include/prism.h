@@ -160,7 +160,15 @@ int prism_sparse_attn(const prism_config* cfg, const void* q, const void* k, con
 /*
  * One prefill layer: prism_estimate followed by prism_sparse_attn on the same
  * stream, no host synchronisation in between.  mask_out may be NULL, in which
- * case the mask lives in the workspace (the size then includes it).
+ * case the mask lives in the workspace (the size then includes it).  The
+ * attention is launched with programmatic serialization: its thread blocks
+ * may start on SMs the estimator has left, each waiting (bounded, then
+ * PRISM_ERR_TIMEOUT through prism_get_last_device_error) until the estimator
+ * has published the mask rows it reads, so attention on finished rows
+ * overlaps the end of the estimator (Prism: Spectral-Aware Block-Sparse
+ * Attention, gist.science Technical Summary, introduction: the cost of
+ * finding the relevant blocks is what such methods must keep small).  The
+ * outputs equal those of the two separate calls.
  */
 int prism_prefill(const prism_config* cfg, const void* q, const void* k, const void* v,
                   uint32_t* mask_out, void* o, void* workspace, size_t workspace_bytes,

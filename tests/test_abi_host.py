@@ -68,7 +68,7 @@ def test_workspace_size_formula():
     nch = 1  # score chunks of 128 query blocks
     expect = 3 * up(rows * nb * dp * 2) + up(rows * nb * 4 * 4) + up(q_rows * 16) \
         + up(q_rows * nch * 2 * 128 * 128 * 4) + up(q_rows * nb * 1 * 2 * 4) + up(q_rows * nb * 1 * 4) \
-        + up((2 + 2 * kv_rows + q_rows * nch) * 4)
+        + up((2 + 2 * kv_rows + q_rows * nch + q_rows * ((nb + 15) // 16)) * 4)
     assert n == expect
 
 

@@ -59,6 +59,13 @@ def test_full_size_sampled_parity(name, cuda_device):
     pb.prism_estimate(cfg, qd, kd, mask2, ws, dbg_scores=scores, dbg_tau=tau)
     torch.cuda.synchronize()
     assert torch.equal(mask2, mask), "estimate and prefill disagree on the mask"
+    # the prefill's attention starts while its estimator still runs: every
+    # output row must equal a separate attention call on the final mask
+    o_sep = torch.empty_like(o)
+    pb.prism_sparse_attn(cfg, qd, kd, vd, mask, o_sep)
+    torch.cuda.synchronize()
+    assert torch.equal(o_sep, o), "overlapped prefill differs from separate calls"
+    del o_sep
     hi, lo = gen.default_bands()
     ref = P.oracle_estimate_streamed(q, k, (hi, lo), w.p, heads=heads)
     sc = P.unpack_tri(scores[0, heads].cpu().double().numpy(), nb)
