@@ -57,6 +57,7 @@ class _Config(ctypes.Structure):
         ("p", ctypes.c_float), ("causal", ctypes.c_int), ("tau_mode", ctypes.c_int),
         ("tau_hi", ctypes.c_float), ("tau_lo", ctypes.c_float), ("softmax_scale", ctypes.c_float),
         ("force_blocks", ctypes.c_int),
+        ("seqlens", ctypes.POINTER(ctypes.c_int32)),
     ]
 
 
@@ -95,13 +96,19 @@ class PrismConfig:
     def __init__(self, batch: int, hq: int, hkv: int, seqlen: int, band_hi: Sequence[int],
                  band_lo: Sequence[int], p: float, head_dim: int = 128, block: int = 128,
                  causal: int = 1, tau_mode: int = PRISM_TAU_RMS, tau_hi: float = 1.0,
-                 tau_lo: float = 1.0, softmax_scale: float = 0.0, force_blocks: int = 0):
+                 tau_lo: float = 1.0, softmax_scale: float = 0.0, force_blocks: int = 0,
+                 seqlens: Optional[Sequence[int]] = None):
+        """``seqlens``: tokens of each batch element when they differ (padded
+        layout of ``seqlen`` tokens; padding zero in q and k, finite in v)."""
         self._hi = (ctypes.c_int32 * max(len(band_hi), 1))(*band_hi)
         self._lo = (ctypes.c_int32 * max(len(band_lo), 1))(*band_lo)
+        self._sl = (ctypes.c_int32 * len(seqlens))(*seqlens) if seqlens is not None else None
         self.c = _Config(batch, hq, hkv, seqlen, head_dim, block,
                          ctypes.cast(self._hi, ctypes.POINTER(ctypes.c_int32)), len(band_hi),
                          ctypes.cast(self._lo, ctypes.POINTER(ctypes.c_int32)), len(band_lo),
-                         p, causal, tau_mode, tau_hi, tau_lo, softmax_scale, force_blocks)
+                         p, causal, tau_mode, tau_hi, tau_lo, softmax_scale, force_blocks,
+                         ctypes.cast(self._sl, ctypes.POINTER(ctypes.c_int32)) if self._sl is not None
+                         else ctypes.POINTER(ctypes.c_int32)())
 
     @property
     def nb(self) -> int:

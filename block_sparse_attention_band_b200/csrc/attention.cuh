@@ -68,11 +68,20 @@ enum : uint32_t {
   kNumBars = 16
 };
 
+// Per-sequence token counts of a batch whose sequences differ in length
+// (varlen = 0: every sequence fills the layout's seqlen).
+constexpr int kMaxSeqs = 256;
+struct SeqLens {
+  int varlen;
+  int n[kMaxSeqs];
+};
+
 // One 128-query tile of a work item.
 struct Tile {
-  int valid;  // 0: the item has a single tile
+  int valid;  // 0: no such tile (past the item's rows or its sequence)
   int i;      // query block
   int bh;     // batch * hq + head
+  int ntok;   // tokens of its sequence
   const uint32_t* mrow;
   int last_word;
   uint32_t last_mask;
@@ -84,11 +93,13 @@ struct Tile {
 };
 
 __device__ __forceinline__ void make_tile(Tile& t, int row, int rows_total, int G, int nb, int kv_global,
-                                          int hq, const uint32_t* mask, int W) {
+                                          int hq, const uint32_t* mask, int W, int seqlen, const SeqLens& lens) {
   t.valid = row < rows_total;
   const int r = t.valid ? row : 0;
   t.i = nb - 1 - r / G;
   const int bi = kv_global / (hq / G);  // batch of this KV head
+  t.ntok = lens.varlen ? lens.n[bi] : seqlen;
+  if (t.i * 128 >= t.ntok) t.valid = 0;  // a query block past its sequence
   const int kv = kv_global - bi * (hq / G);
   const int h = kv * G + r % G;
   t.bh = bi * hq + h;
@@ -216,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const uint32_t* mask,
                    __nv_bfloat16* __restrict__ out, int batch, int hq, int hkv, int seqlen, int nb,
-                   float scale_log2, const uint32_t* ready, int ready_rows) {
+                   float scale_log2, const uint32_t* ready, int ready_rows, const __grid_constant__ SeqLens lens) {
   __shared__ int s_masks_ok;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -236,8 +247,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const int kv_global = (int)(blockIdx.x / items_per_kv);
   const int W = (nb + 31) >> 5;
   Tile tiles[2];
-  make_tile(tiles[0], 2 * m, rows_per_kv, G, nb, kv_global, hq, mask, W);
-  make_tile(tiles[1], 2 * m + 1, rows_per_kv, G, nb, kv_global, hq, mask, W);
+  make_tile(tiles[0], 2 * m, rows_per_kv, G, nb, kv_global, hq, mask, W, seqlen, lens);
+  make_tile(tiles[1], 2 * m + 1, rows_per_kv, G, nb, kv_global, hq, mask, W, seqlen, lens);
 
   if (threadIdx.x == 0) {
     for (uint32_t s = 0; s < kNumBars; ++s)
@@ -438,7 +449,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
     // ------------------------------------------------------------ epilogue
     // query rows past the end of a short last block are computed but not stored
-    const bool row_ok = T.valid && T.i * 128 + r < seqlen;
+    const bool row_ok = T.valid && T.i * 128 + r < T.ntok;
     __nv_bfloat16* orow = row_ok ? out + ((size_t)T.bh * seqlen + (size_t)T.i * 128 + r) * 128 : nullptr;
     if (T.valid && n == 0) {  // (warp-uniform branches: the loads below are warp-collective)
       const uint4 z = make_uint4(0u, 0u, 0u, 0u);

@@ -83,6 +83,7 @@ __device__ __forceinline__ int stream_tid(int t) { return t < 64 ? t : t - 64; }
 __device__ __forceinline__ int stream_warp(int warp) { return warp < 2 ? warp : warp - 2; }  // 0 .. 5
 __device__ __forceinline__ int lane_warp(int warp) { return warp < 4 ? warp - 2 : warp - 6; }    // 0 .. 9
 constexpr int kMaxGroupHeads = 64;    // Q heads per KV head supported by the tau step
+constexpr int kMaxSeqs = 256;         // sequences of a batch with per-sequence lengths
 constexpr int kTauBatch = 5;          // head rows whose energy partials the tau step sums at once
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -129,7 +130,13 @@ struct EstParams {
   float tau_hi, tau_lo;
   int force;  // optional forced blocks: 1 = key block 0, 2 = the diagonal
   BandLayout bl;
+  int varlen;              // 1: batch element b holds seq_n[b] <= n tokens (the rest is padding)
+  int seq_n[kMaxSeqs];
 };
+
+// Tokens and blocks of batch element bi (the layout keeps n tokens, nb blocks per head).
+__device__ __forceinline__ int seq_tokens(const EstParams& P, int bi) { return P.varlen ? P.seq_n[bi] : P.n; }
+__device__ __forceinline__ int seq_blocks(const EstParams& P, int bi) { return (seq_tokens(P, bi) + 127) >> 7; }
 
 // The 128 x 128 score tile (row chunk cr, column chunk cc <= cr) of one
 // (batch, Q head): rows = query blocks 128 cr + r, columns = key blocks 128 cc + c.
@@ -228,6 +235,7 @@ __device__ __forceinline__ float warp_reduce_n(float (&v)[N], int lane) {
 __device__ __forceinline__ void group_temperatures(const EstParams& P, int g, PoolSmem& sm) {
   const int t = stream_tid(threadIdx.x), warp = t >> 5, lane = t & 31;  // the stream lane
   const int bi = g / P.hkv, kv = g - bi * P.hkv;
+  const int nbb = seq_blocks(P, bi);
   // slots 0..G-1: Q heads, G: the KV head; kTauBatch slots at a time, so the
   // loads of all of them are in flight together (the partials come from L2)
   for (int s0 = 0; s0 <= P.G; s0 += kTauBatch) {
@@ -236,7 +244,7 @@ __device__ __forceinline__ void group_temperatures(const EstParams& P, int g, Po
 #pragma unroll
     for (int q = 0; q < kTauBatch; ++q) s[q][0] = s[q][1] = s[q][2] = 0.f;
 #pragma unroll 2
-    for (int i = t; i < P.nb; i += kStreamThreads) {
+    for (int i = t; i < nbb; i += kStreamThreads) {
       float4 v[kTauBatch];
 #pragma unroll
       for (int q = 0; q < kTauBatch; ++q) {
@@ -274,7 +282,7 @@ __device__ __forceinline__ void group_temperatures(const EstParams& P, int g, Po
       th = P.tau_hi;
       tl = P.tau_lo;
     } else {
-      const float n = (float)P.nb;
+      const float n = (float)nbb;
       const float* sq = sm.sums[t];
       const float* sk = sm.sums[P.G];
       const float rq_hi = sqrtf(sq[0] / (n * P.bl.d_hi)), rq_lo = sqrtf(sq[1] / (n * P.bl.d_lo));
@@ -372,7 +380,7 @@ __device__ __forceinline__ PoolCoords pool_coords(const EstParams& P, const CUte
   c.map = &tm[is_q ? 6 : 7];
   c.head = is_q ? bi * P.hq + kv * P.G + slot : g;
   c.tok0 = blk0 * 128;
-  c.nt = min(blk0 + kPoolTilesPerItem, P.nb) - blk0;
+  c.nt = max(min(blk0 + kPoolTilesPerItem, seq_blocks(P, bi)) - blk0, 0);  // 0: past the sequence
   return c;
 }
 
@@ -400,12 +408,15 @@ __device__ __forceinline__ void pool_item(const EstParams& P, const CUtensorMap*
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int slot = y / P.pool_item_span;
   const int blk0 = (y - slot * P.pool_item_span) * kPoolTilesPerItem;
-  const int nt = min(blk0 + kPoolTilesPerItem, P.nb) - blk0;
   const int bi = g / P.hkv, kv = g - bi * P.hkv;
+  const int nbb = seq_blocks(P, bi);
+  const int nt = max(min(blk0 + kPoolTilesPerItem, nbb) - blk0, 0);  // 0: past the sequence, only counted
   const bool is_q = slot < P.G;
   const int hr = is_q ? bi * P.hq + kv * P.G + slot : P.q_rows + g;
   const uint32_t ring0 = (smem_u32(ring) + 1023u) & ~1023u;
-  if (t == 0) {  // producer
+  if (nt == 0) {
+    // nothing to pool (no tile of it was prefetched either)
+  } else if (t == 0) {  // producer
     fence_proxy_async_smem();  // generic writes of the last item before the async ones
     pool_stream(pool_coords(P, tm, g, y), st.pre, nt, sm, ring0, stages, st);
     st.pre = 0;
@@ -459,7 +470,7 @@ __device__ __forceinline__ void pool_item(const EstParams& P, const CUtensorMap*
       for (int b = 0; b < 16; ++b) {
         // block mean: the last block may hold fewer than 128 tokens (zeros past the end)
         const int blk = blk0 + b0 + b;
-        const float inv = blk == P.nb - 1 ? 1.0f / (float)(P.n - 128 * (P.nb - 1)) : (1.0f / 128.0f);
+        const float inv = blk == nbb - 1 ? 1.0f / (float)(seq_tokens(P, bi) - 128 * (nbb - 1)) : (1.0f / 128.0f);
         const float m = __uint_as_float(v[b]) * inv;
         const bool ok = b0 + b < nt;
         if (ok && c != 255) {
@@ -970,7 +981,8 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
   score_part_of(P, y / P.G, chunk, part);  // longest rows first
   const int bh = bi * P.hq + kv * P.G + y % P.G;
   const int i0 = chunk * kScoreRows;
-  const int max_i = min(P.nb, i0 + kScoreRows) - 1;
+  const int nbb = seq_blocks(P, bi);
+  const int max_i = min(nbb, i0 + kScoreRows) - 1;  // < i0: the chunk is past the sequence, only counted
   const uint32_t nch = (uint32_t)P.bl.dp / 64;
   const int ncolw = score_cols(P.bl.dp);  // N: key blocks per column chunk
   // this part's key blocks [j0, j1): column chunks c0 .. c0 + ncol - 1
@@ -994,7 +1006,9 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
   auto bar_e = [&](int c) { return smem_u32(&sm.bar_acc[c & 1]); };
   auto dacc = [&](int c) { return sm.tmem + 256u * (uint32_t)(c & 1); };
 
-  if (warp == 0) {
+  if (max_i < i0) {
+    // past the sequence: no rows, only the part count below
+  } else if (warp == 0) {
     if (lane == 0) {  // operand producer
       const int arow = bh * P.nb + i0;          // pooled rows of the Q head
       const int brow0 = (P.q_rows + g) * P.nb;  // pooled rows of the KV head
@@ -1155,10 +1169,16 @@ __device__ __forceinline__ void topp_item(const EstParams& P, int g, int y, cons
   const int seg = nseg - 1 - y / P.G;  // longest rows first
   const int bh = bi * P.hq + kv * P.G + y % P.G;
   const int r0 = seg * kToppRows;
-  const int max_i = min(P.nb, r0 + kToppRows) - 1;
+  const int nbb = seq_blocks(P, bi);
+  const int max_i = min(nbb, r0 + kToppRows) - 1;
   const int chunk = r0 / kScoreRows, i0 = chunk * kScoreRows;
   const size_t tri = (size_t)P.nb * (P.nb + 1) / 2;
   if (T.lw >= T.nw) return;
+  {  // rows of the layout past the sequence: empty mask rows
+    const int lo = max(r0, nbb), hi = min(P.nb, r0 + kToppRows);
+    for (int x = T.lw * 32 + (threadIdx.x & 31); x < (hi - lo) * P.W; x += T.nw * 32)
+      P.mask[((size_t)bh * P.nb + lo) * P.W + x] = 0u;
+  }
   unsigned char* wb = T.region + (size_t)T.lw * T.stride;
   const int nbp = (P.nb + 7) & ~7;
   const int nbuf = T.single ? 1 : 2;

@@ -33,8 +33,11 @@ struct Plan {
   float tau_hi, tau_lo;
   float scale;
   int force;
+  int varlen;            // per-sequence lengths given
+  int seq_n[kMaxSeqs];   // tokens of each batch element (n when not varlen)
   size_t off_pool[kTerms], off_part, off_tau, off_scores, off_rmax, off_mask, off_sync, sync_bytes, total;
 };
+static_assert(kMaxSeqs == attn::kMaxSeqs, "one sequence limit for both kernels");
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -55,6 +58,11 @@ int validate(const prism_config* cfg, Plan* pl) {
     return PRISM_ERR_TAU;
   if (!(cfg->p > 0.f)) return PRISM_ERR_P;  // also rejects NaN
   if (cfg->force_blocks & ~(PRISM_FORCE_SINK | PRISM_FORCE_DIAG)) return PRISM_ERR_UNSUPPORTED;
+  if (cfg->seqlens) {  // one length per batch element, 1 .. seqlen
+    if (cfg->batch > kMaxSeqs) return PRISM_ERR_UNSUPPORTED;
+    for (int x = 0; x < cfg->batch; ++x)
+      if (cfg->seqlens[x] < 1 || cfg->seqlens[x] > cfg->seqlen) return PRISM_ERR_SHAPE;
+  }
   if (!cfg->band_hi || !cfg->band_lo) return PRISM_ERR_NULL;
   if (cfg->n_hi <= 0 || cfg->n_lo <= 0 || cfg->n_hi > 128 || cfg->n_lo > 128) return PRISM_ERR_BAND;
   bool in_hi[128] = {}, in_lo[128] = {};
@@ -70,6 +78,8 @@ int validate(const prism_config* cfg, Plan* pl) {
   }
   if (!pl) return PRISM_OK;
   Plan& P = *pl;
+  P.varlen = cfg->seqlens != nullptr;
+  for (int x = 0; x < cfg->batch && x < kMaxSeqs; ++x) P.seq_n[x] = P.varlen ? cfg->seqlens[x] : cfg->seqlen;
   P.b = cfg->batch;
   P.hq = cfg->hq;
   P.hkv = cfg->hkv;
@@ -349,6 +359,8 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   E.tau_lo = P.tau_lo;
   E.force = P.force;
   E.bl = P.bl;
+  E.varlen = P.varlen;
+  for (int x = 0; x < kMaxSeqs; ++x) E.seq_n[x] = x < P.b ? P.seq_n[x] : 0;
   int dev = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, estimator_kernel, kEstThreads, L.smem) !=
@@ -387,9 +399,12 @@ int run_attention(const Plan& P, const void* q, const void* k, const void* v, co
   const float scale_log2 = P.scale * 1.4426950408889634f;
   const unsigned grid = attn::grid_size(P.b, P.hq, P.hkv, P.nb);
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(o);
+  attn::SeqLens lens;
+  lens.varlen = P.varlen;
+  for (int x = 0; x < attn::kMaxSeqs; ++x) lens.n[x] = x < P.b ? P.seq_n[x] : 0;
   if (!ready) {
     attn::sparse_attn_kernel<<<grid, attn::kThreads, attn::kSmemBytes, st>>>(
-        mq, mk, mv, mask, out, P.b, P.hq, P.hkv, P.n, P.nb, scale_log2, nullptr, kToppRows);
+        mq, mk, mv, mask, out, P.b, P.hq, P.hkv, P.n, P.nb, scale_log2, nullptr, kToppRows, lens);
     return launched();
   }
   cudaLaunchConfig_t lc = {};
@@ -403,7 +418,7 @@ int run_attention(const Plan& P, const void* q, const void* k, const void* v, co
   lc.attrs = attr;
   lc.numAttrs = 1;
   if (cudaLaunchKernelEx(&lc, attn::sparse_attn_kernel, mq, mk, mv, mask, out, P.b, P.hq, P.hkv, P.n, P.nb,
-                         scale_log2, ready, kToppRows) != cudaSuccess)
+                         scale_log2, ready, kToppRows, lens) != cudaSuccess)
     return PRISM_ERR_CUDA;
   return launched();
 }

@@ -114,6 +114,18 @@ typedef struct prism_config {
                             PRISM_FORCE_SINK keeps key block 0 in every row,
                             PRISM_FORCE_DIAG keeps the diagonal block j = i.
                             Other bits: PRISM_ERR_UNSUPPORTED. */
+  const int32_t* seqlens;  /* NULL: every batch element holds seqlen tokens.
+                            Else a host array of batch lengths, 1 <= seqlens[b]
+                            <= seqlen (batch <= 256, else
+                            PRISM_ERR_UNSUPPORTED; out of range:
+                            PRISM_ERR_SHAPE): batch element b holds seqlens[b]
+                            tokens at positions 0 .. seqlens[b]-1 of the
+                            [.., seqlen, 128] layout, the rest is padding that
+                            must hold zeros in q and k and finite values in v.
+                            Each sequence has its own ceil(seqlens[b] / B)
+                            blocks, pooling, temperatures and Top-P rows; mask
+                            rows past them are written as zeros, o rows past
+                            them are not written.  Read during the call only. */
 } prism_config;
 
 enum { PRISM_FORCE_SINK = 1, PRISM_FORCE_DIAG = 2 };

@@ -90,6 +90,17 @@ def test_bad_config_rejected_on_host(kw, code):
     assert pb.lib.prism_prefill(_cfg(**kw).ptr(), fake, fake, fake, None, fake, fake, 1 << 40, None) == code
 
 
+def test_seqlens_validated_and_layout_sized():
+    base = _ws_size(_cfg())[1]
+    ok = _cfg(batch=3, seqlens=[1024, 1, 500])
+    s, n = _ws_size(ok)
+    assert s == 0 and n == _ws_size(_cfg(batch=3))[1]  # the workspace follows the padded layout
+    for bad in ([0, 5, 5], [1025, 5, 5], [-3, 5, 5]):
+        assert _ws_size(_cfg(batch=3, seqlens=bad))[0] == -2
+    assert _ws_size(_cfg(batch=257, seqlens=[7] * 257))[0] == -6
+    assert base > 0
+
+
 def test_null_pointers_workspace_and_alignment_rejected():
     cfg = _cfg()
     _, ws = _ws_size(cfg)

@@ -252,6 +252,55 @@ def test_topp_ties_and_crowded_bins(kind, cuda_device):
             assert mask[0, 0, i, :keep].all() and not mask[0, 0, i, keep:].any(), i
 
 
+def test_variable_length_batch(cuda_device):
+    """A padded batch of sequences of different lengths (seqlens): every
+    sequence's mask rows and outputs equal those of the same sequence run
+    alone (bit for bit) and match the oracle; rows past a sequence are empty
+    mask rows and unwritten outputs."""
+    lens = [9 * 128 + 77, 700, 129, 128]
+    n_max, hq, hkv = max(lens), 4, 2
+    singles = [gen.small_workload(f"varlen_{n}", 1, hq, hkv, n, seed=80 + x, p=0.9) for x, n in enumerate(lens)]
+    b = len(lens)
+    q = torch.zeros(b, hq, n_max, 128, dtype=torch.bfloat16)
+    k = torch.zeros(b, hkv, n_max, 128, dtype=torch.bfloat16)
+    v = torch.full((b, hkv, n_max, 128), 7.0, dtype=torch.bfloat16)  # finite padding, never used
+    parts = []
+    for x, w in enumerate(singles):
+        qs, ks, vs = gen.make_inputs(w)
+        q[x, :, :w.seqlen], k[x, :, :w.seqlen], v[x, :, :w.seqlen] = qs[0], ks[0], vs[0]
+        parts.append((qs, ks, vs))
+    hi, lo = gen.default_bands()
+    cfg = pb.PrismConfig(b, hq, hkv, n_max, hi, lo, 0.9, seqlens=lens)
+    nb, W = cfg.nb, cfg.words
+    qd, kd, vd = q.to(cuda_device), k.to(cuda_device), v.to(cuda_device)
+    ws = torch.empty(pb.prism_workspace_size(cfg), dtype=torch.uint8, device=cuda_device)
+    mask = torch.full((b, hq, nb, W), 0x5A5A5A5A, dtype=torch.int32, device=cuda_device)
+    o = torch.full_like(qd, 3.0)
+    pb.prism_prefill(cfg, qd, kd, vd, mask, o, ws)
+    torch.cuda.synchronize()
+    assert pb.prism_get_last_device_error() == 0
+    words = mask.cpu().numpy().view(np.uint32)
+    ocpu = o.cpu()
+    for x, w in enumerate(singles):
+        qs, ks, vs = parts[x]
+        nbx = w.nb
+        assert not words[x, :, nbx:].any(), "mask rows past the sequence must be empty"
+        assert torch.all(ocpu[x, :, w.seqlen:] == 3.0), "output rows past the sequence were written"
+        # the same sequence alone
+        cfg1 = P.make_cfg(w)
+        m1, sc1, tau1, w1 = P.run_estimate(cfg1, qs.to(cuda_device), ks.to(cuda_device))
+        assert np.array_equal(words[x, :, :nbx, :cfg1.words], w1[0])
+        o1 = P.run_attention(cfg1, qs.to(cuda_device), ks.to(cuda_device), vs.to(cuda_device),
+                             torch.from_numpy(w1.view(np.int32)).to(cuda_device))
+        assert torch.equal(o[x, :, :w.seqlen].cpu(), o1[0].cpu())
+        # and the oracle on it
+        ref = oracle.estimate(qs, ks, hi, lo, w.p)
+        P.check_tau(tau1, ref)
+        P.check_mask(m1, ref, w.p)
+        rows = [(0, h, i) for h in range(hq) for i in range(nbx)]
+        P.check_attention_rows(o1, qs, ks, vs, m1, rows, hq // hkv)
+
+
 def test_small_p_sparse_rows(cuda_device):
     w = gen.small_workload("sparse_nb48", 1, 2, 1, 48 * 128, seed=35, p=0.3)
     q, k, v, qd, kd, vd = _inputs(w, cuda_device)
