@@ -50,6 +50,7 @@ constexpr uint32_t kOffQ = 0;                    // Q_A, Q_B
 constexpr uint32_t kOffK = 2 * kTileBytes;       // 2 stages
 constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;
 constexpr uint32_t kOffBar = kOffV + 2 * kTileBytes;
+constexpr int kMaxMaskWords = 16384 / 32;  // mask words of one row at the largest nb
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + slack for 1024-byte alignment
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -82,12 +83,12 @@ struct Tile {
   int i;      // query block
   int bh;     // batch * hq + head
   int ntok;   // tokens of its sequence
-  const uint32_t* mrow;
+  const uint32_t* mrow;  // the mask row: in global memory, then its copy in shared memory
   int last_word;
   uint32_t last_mask;
   __device__ __forceinline__ uint32_t word(int w) const {
     if (!valid || w > last_word) return 0u;
-    const uint32_t b = __ldcg(mrow + w);  // L2: the mask may have been written during this launch
+    const uint32_t b = mrow[w];
     return w == last_word ? (b & last_mask) : b;
   }
 };
@@ -229,6 +230,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                    __nv_bfloat16* __restrict__ out, int batch, int hq, int hkv, int seqlen, int nb,
                    float scale_log2, const uint32_t* ready, int ready_rows, const __grid_constant__ SeqLens lens) {
   __shared__ int s_masks_ok;
+  __shared__ uint32_t s_mask[2][kMaxMaskWords];  // the two tiles' mask rows
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -277,6 +279,14 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   __syncthreads();
   tc_fence_after();
   if (!s_masks_ok) tiles[0].valid = tiles[1].valid = 0;  // (timed out: error recorded, no work)
+  // the tiles' mask rows, read once through L2 (they may have been written
+  // during this launch), then from shared memory by every role
+  for (int x = 0; x < 2; ++x)
+    if (tiles[x].valid)
+      for (int w = threadIdx.x; w <= tiles[x].last_word; w += kThreads) s_mask[x][w] = __ldcg(tiles[x].mrow + w);
+  __syncthreads();
+  tiles[0].mrow = s_mask[0];
+  tiles[1].mrow = s_mask[1];
   const uint32_t tmem = *tmem_holder;
   // Each warpgroup sets its register budget first and then runs only its own
   // roles (no code is shared across the split); warp 1 frees tensor memory
