@@ -480,9 +480,15 @@ def main():
     est_gbs = est_bytes / (t_est * 1e-3) / 1e9
 
     # ---------------- end to end: pinned host buffers, copies timed ---------
+    # Every step uploads its Q, K, V from pinned host memory, runs the prefill
+    # through the public API and downloads its whole output O.  Serial: one
+    # step at a time on one stream.  Pipelined (the reported value): two device
+    # buffer sets and three streams, so step s+1's upload and step s-1's
+    # download run beside step s's kernels; timed from the first upload to the
+    # last download, divided by the steps.
     qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
-    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    e2e = []
+    ohs = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(2)]
+    e2e_serial = []
     for it in range(args.steps + 1):
         ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ea.record(stream)
@@ -490,14 +496,49 @@ def main():
         kd.copy_(kh, non_blocking=True)
         vd.copy_(vh, non_blocking=True)
         step()
-        oh.copy_(o, non_blocking=True)
+        ohs[0].copy_(o, non_blocking=True)
         eb.record(stream)
         torch.cuda.synchronize()
         if it > 0:
-            e2e.append(ea.elapsed_time(eb))
-    e2e_ms = reduce_max([statistics.median(e2e)], dist, dev)[0]
+            e2e_serial.append(ea.elapsed_time(eb))
+    e2e_serial_ms = reduce_max([statistics.median(e2e_serial)], dist, dev)[0]
+    sets = [(qd, kd, vd, o), (torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd), torch.empty_like(o))]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def pipelined(n_steps):
+        ev = {}
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(up)
+        for s_ in range(n_steps):
+            qx, kx, vx, ox = sets[s_ % 2]
+            if s_ >= 2:
+                up.wait_event(ev[("done", s_ - 2)])  # step s-2 has read this input set
+            with torch.cuda.stream(up):
+                qx.copy_(qh, non_blocking=True)
+                kx.copy_(kh, non_blocking=True)
+                vx.copy_(vh, non_blocking=True)
+            ev[("in", s_)] = torch.cuda.Event()
+            ev[("in", s_)].record(up)
+            stream.wait_event(ev[("in", s_)])
+            if s_ >= 2:
+                stream.wait_event(ev[("out", s_ - 2)])  # step s-2's output has been downloaded
+            pb.prism_prefill(cfg, qx, kx, vx, mask, ox, ws, stream=stream)
+            ev[("done", s_)] = torch.cuda.Event()
+            ev[("done", s_)].record(stream)
+            down.wait_event(ev[("done", s_)])
+            with torch.cuda.stream(down):
+                ohs[s_ % 2].copy_(ox, non_blocking=True)
+            ev[("out", s_)] = torch.cuda.Event()
+            ev[("out", s_)].record(down)
+        t1.record(down)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / n_steps
+
+    pipelined(2)  # warm-up of the streams and the second buffer set
+    e2e_ms = reduce_max([pipelined(args.steps)], dist, dev)[0]
+    assert pb.prism_get_last_device_error() == 0
     h2d = qh.nbytes + kh.nbytes + vh.nbytes
-    d2h = oh.nbytes
+    d2h = ohs[0].nbytes
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -532,7 +573,9 @@ def main():
                                "peak": peak_hbm, "unit": "GB/s", "frac": est_gbs / peak_hbm,
                                "algorithmic_bytes": est_bytes, "traffic": traffic.get("estimator_kernel"),
                                "peak_source": f"{peak_src} copy bandwidth (of {peak_src})"},
-        "e2e": {"value": job_value(e2e_ms, world), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": job_value(e2e_ms, world), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "mode": "pipelined: step s+1 upload and step s-1 download beside step s (2 buffer sets, 3 streams)",
+                "serial_value": job_value(e2e_serial_ms, world)},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
