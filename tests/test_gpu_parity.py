@@ -189,6 +189,23 @@ def test_irregular_bands(seed, n_hi, n_lo, cuda_device):
     P.check_mask(mask, ref, w.p)
 
 
+def test_long_rows_in_parts_with_the_widest_layout(cuda_device):
+    """Rows longer than one score part (512 key blocks) with band sets whose
+    pooled layout is 192 columns wide (64-block column chunks): the parts'
+    row maxima and counters combine to the oracle's scores and masks."""
+    w = gen.small_workload("parts_dp192_nb600", 1, 1, 1, 600 * 128, seed=90, p=0.9)
+    q, k, _ = gen.make_inputs(w, with_v=False)
+    rng = np.random.default_rng(42)  # 60 / 90 dims: a 192-column pooled layout
+    hi = sorted(rng.choice(128, 60, replace=False).tolist())
+    lo = sorted(rng.choice(128, 90, replace=False).tolist())
+    cfg = P.make_cfg(w, bands=(hi, lo))
+    mask, sc, tau, _ = P.run_estimate(cfg, q.to(cuda_device), k.to(cuda_device))
+    ref = oracle.estimate(q, k, hi, lo, w.p)
+    P.check_tau(tau, ref)
+    P.check_scores(sc, ref)
+    P.check_mask(mask, ref, w.p)
+
+
 @pytest.mark.parametrize("layout", ["interleaved", "half_split"])
 def test_rope_layout_presets(layout, cuda_device):
     """Inputs rotated in either RoPE layout, bands from the matching preset:
