@@ -308,6 +308,59 @@ def run_table(args):
         torch.cuda.empty_cache()
 
 
+def causal_mask_words(nb: int, words: int) -> torch.Tensor:
+    """[nb, words] int32 rows keeping every causal block (p >= 1)."""
+    full = torch.zeros(nb, words, dtype=torch.int64)
+    for i in range(nb):
+        for wd in range(i // 32 + 1):
+            lo = wd * 32
+            full[i, wd] = (1 << 32) - 1 if lo + 32 <= i + 1 else (1 << (i + 1 - lo)) - 1
+    return full.to(torch.int32)
+
+
+def run_sweep_p(args):
+    """Prefill time against the kept-block density: one line per Top-P
+    threshold p on one workload, with the same kernel on every causal block
+    (dense) as the reference point."""
+    import block_sparse_attention_band_b200 as pb
+    dev = torch.device("cuda:0")
+    w = gen.WORKLOADS[args.workload]
+    q, k, v = gen.make_inputs(w)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    hi, lo = gen.default_bands()
+    o = torch.empty_like(qd)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn, reps):
+        fn()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    cfg1 = pb.PrismConfig(w.batch, w.hq, w.hkv, w.seqlen, hi, lo, 1.0)
+    dense_mask = causal_mask_words(w.nb, cfg1.words).expand(w.batch, w.hq, w.nb, cfg1.words).contiguous().to(dev)
+    t_dense = timed(lambda: pb.prism_sparse_attn(cfg1, qd, kd, vd, dense_mask, o, stream=stream), args.steps)
+    del dense_mask
+    causal_tiles = w.batch * w.hq * w.nb * (w.nb + 1) // 2
+    for p in [float(x) for x in args.sweep_p.split(",")]:
+        cfg = pb.PrismConfig(w.batch, w.hq, w.hkv, w.seqlen, hi, lo, p)
+        ws = torch.empty(pb.prism_workspace_size(cfg), dtype=torch.uint8, device=dev)
+        mask = torch.empty(w.batch, w.hq, w.nb, cfg.words, dtype=torch.int32, device=dev)
+        t_pre = timed(lambda: pb.prism_prefill(cfg, qd, kd, vd, mask, o, ws, stream=stream), args.steps)
+        assert pb.prism_get_last_device_error() == 0
+        kept = int(np.unpackbits(mask.cpu().numpy().view(np.uint8)).sum())
+        print(json.dumps({"sweep_p": p, "workload": w.name, "density": kept / causal_tiles, "prefill_ms": t_pre,
+                          "dense_attention_ms": t_dense, "speedup_vs_dense": t_dense / t_pre,
+                          "timing": f"CUDA events, median of {args.steps}"}), flush=True)
+        del ws, mask
+
+
 def run_compare_plain(args):
     """Prism's estimator against the plain mean-pooling estimator (one band of
     all dims, no temperature) on one workload: density, estimator time, and the
@@ -386,9 +439,14 @@ def main():
                     help="Prism vs the plain mean-pooling estimator on one workload (attention error vs dense)")
     ap.add_argument("--table", default=None,
                     help="'all' or a comma list of workloads: per-configuration lines instead of the headline")
+    ap.add_argument("--sweep-p", default=None,
+                    help="comma list of Top-P thresholds: prefill time and density per p on --workload, vs dense")
     args = ap.parse_args()
     if args.table:
         run_table(args)
+        return
+    if args.sweep_p:
+        run_sweep_p(args)
         return
     if args.compare_plain:
         run_compare_plain(args)
@@ -462,6 +520,20 @@ def main():
         attn_ms.append(e[1].elapsed_time(e[2]))
     t_est = statistics.median(est_ms)
     t_attn = statistics.median(attn_ms)
+    # the same attention kernel on every causal block (p = 1): the dense
+    # prefill the method is set against (context for the speed-up, not timed
+    # in the step)
+    dense_mask = causal_mask_words(w.nb, cfg.words).expand(w.batch, w.hq, w.nb, cfg.words).contiguous().to(dev)
+    dense_ms = []
+    for _ in range(3):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record(stream)
+        pb.prism_sparse_attn(cfg, qd, kd, vd, dense_mask, o, stream=stream)
+        e[1].record(stream)
+        torch.cuda.synchronize()
+        dense_ms.append(e[0].elapsed_time(e[1]))
+    t_dense = statistics.median(dense_ms)
+    del dense_mask
 
     words = mask.cpu().numpy().view(np.uint32)
     nb = w.nb
@@ -564,7 +636,8 @@ def main():
                    "density": density, "kept_tiles": kept, "causal_tiles": causal_tiles,
                    "attention_tflops": attn_tflops, "effective_tflops_vs_dense":
                        causal_tiles * flops_tile / (ms_step * 1e-3) / 1e12,
-                   "estimator_gbs": est_gbs, "estimator_hbm_frac": est_gbs / peak_hbm},
+                   "estimator_gbs": est_gbs, "estimator_hbm_frac": est_gbs / peak_hbm,
+                   "dense_attention_ms": t_dense, "speedup_vs_dense": t_dense / ms_step},
         "roofline": {"kernel": "sparse_attn_kernel", "bound": "tensor", "achieved": attn_tflops,
                      "peak": peak_tensor, "unit": "TFLOP/s", "frac": attn_tflops / peak_tensor,
                      "traffic": traffic.get("sparse_attn_kernel"),
