@@ -5,10 +5,12 @@
 // attention blocks; here the subset is the estimator's mask M (one bit per
 // (query block i, key block j)), token-causal inside the diagonal block.
 //
-// Work item = two 128-query tiles that read the same KV head (for GQA, two Q
-// heads of one group at the same query block), so every K/V tile fetched by
-// TMA serves both.  The key blocks visited are the union of the two tiles'
-// kept sets; each tile computes only its own kept blocks.
+// Work item = two 128-query tiles of one Q head, adjacent query blocks i and
+// i - 1: they read the same KV head, so every K/V tile fetched by TMA serves
+// both, and their kept key blocks overlap most (a step that feeds only one
+// tile leaves the other tile's softmax nothing to overlap).  The key blocks
+// visited are the union of the two tiles' kept sets; each tile computes only
+// its own kept blocks.
 //
 // 384 threads (12 warps; registers re-split per warpgroup: warps 0-3 keep 72,
 // the two softmax warpgroups get 216 so a whole S row stays in registers):
@@ -93,16 +95,16 @@ struct Tile {
   }
 };
 
-__device__ __forceinline__ void make_tile(Tile& t, int row, int rows_total, int G, int nb, int kv_global,
-                                          int hq, const uint32_t* mask, int W, int seqlen, const SeqLens& lens) {
-  t.valid = row < rows_total;
-  const int r = t.valid ? row : 0;
-  t.i = nb - 1 - r / G;
+// Tile of query block i (< 0: none) of Q head hg (within its KV group).
+__device__ __forceinline__ void make_tile(Tile& t, int i, int hg, int G, int nb, int kv_global, int hq,
+                                          const uint32_t* mask, int W, int seqlen, const SeqLens& lens) {
+  t.valid = i >= 0;
+  t.i = t.valid ? i : 0;
   const int bi = kv_global / (hq / G);  // batch of this KV head
   t.ntok = lens.varlen ? lens.n[bi] : seqlen;
   if (t.i * 128 >= t.ntok) t.valid = 0;  // a query block past its sequence
   const int kv = kv_global - bi * (hq / G);
-  const int h = kv * G + r % G;
+  const int h = kv * G + hg;
   t.bh = bi * hq + h;
   t.mrow = mask + ((size_t)t.bh * nb + t.i) * W;
   t.last_word = t.i >> 5;
@@ -241,16 +243,18 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = hq / hkv;
-  const int rows_per_kv = G * nb;
-  const int items_per_kv = (rows_per_kv + 1) >> 1;
+  const int items_per_kv = G * ((nb + 1) >> 1);
   // KV-head-major order: the CTAs running at any time share one KV head, whose
-  // K/V (2 N x 256 bytes) then stays in L2 for all its query blocks
+  // K/V (2 N x 256 bytes) then stays in L2 for all its query blocks.  A CTA
+  // takes two adjacent query blocks of one Q head (their kept key blocks
+  // overlap most, so most steps feed both tiles), longest rows first.
   const int m = (int)(blockIdx.x % items_per_kv);
   const int kv_global = (int)(blockIdx.x / items_per_kv);
   const int W = (nb + 31) >> 5;
+  const int pair = m / G, hg = m - pair * G;
   Tile tiles[2];
-  make_tile(tiles[0], 2 * m, rows_per_kv, G, nb, kv_global, hq, mask, W, seqlen, lens);
-  make_tile(tiles[1], 2 * m + 1, rows_per_kv, G, nb, kv_global, hq, mask, W, seqlen, lens);
+  make_tile(tiles[0], nb - 1 - 2 * pair, hg, G, nb, kv_global, hq, mask, W, seqlen, lens);
+  make_tile(tiles[1], nb - 2 - 2 * pair, hg, G, nb, kv_global, hq, mask, W, seqlen, lens);
 
   if (threadIdx.x == 0) {
     for (uint32_t s = 0; s < kNumBars; ++s)
@@ -493,7 +497,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 // Number of work items (CTAs) for a problem.
 __host__ __forceinline__ unsigned grid_size(int batch, int hq, int hkv, int nb) {
   const int G = hq / hkv;
-  return (unsigned)batch * hkv * (unsigned)((G * nb + 1) / 2);
+  return (unsigned)batch * hkv * (unsigned)(G * ((nb + 1) / 2));
 }
 
 }  // namespace attn
