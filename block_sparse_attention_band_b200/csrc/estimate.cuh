@@ -4,26 +4,30 @@
 // each pooled band, temperatures tau_z, dual-band pooled softmax, Top-P per
 // query-block row and band, union of the two masks.
 //
-// One persistent kernel.  CTAs take work items from a device queue in a fixed
-// order that interleaves the two kinds of work per KV group g (the Q heads
-// that share one KV head):
+// One persistent kernel, one CTA per SM.  Its warps form two lanes with a
+// device queue each, working at the same time:
 //
-//   pool(0), pool(1), score(0), pool(2), score(1), ..., pool(n-1), score(n-2), score(n-1)
+// * the stream lane takes pool and score items, per KV group g (the Q heads
+//   that share one KV head) in the order
+//     pool(0), pool(1), pool(2), score(0), pool(3), score(1), ..., score(n-2), score(n-1)
+//   pool items (HBM-bound) stream 128x128 bf16 tiles of Q and K once (TMA into
+//   a ring of shared-memory stages, several tiles in flight); the block sums
+//   are products on the tensor cores (the tile, read transposed, times a
+//   column of ones: D[dim] += sum over the block's tokens), so the CUDA cores
+//   only turn the sums into the fp32 block means (steps 1-2) and per-block
+//   energy partials (step 3); the CTA that finishes the last pool item of a
+//   group computes the group's temperatures (steps 3-4) and publishes "group
+//   ready".  score items wait for their group and compute both bands' pooled
+//   logits on the tensor cores (step 5; tcgen05 on a three-term bf16 split,
+//   fp32 accuracy), in row chunks of 128 query blocks and parts of at most 512
+//   key blocks, keeping the row maxima;
+// * the Top-P lane takes Top-P items (16 query-block rows of one head) once
+//   their score chunk is complete: softmax + Top-P + union per row (steps
+//   5-7), on the CUDA cores, beside the stream lane's pooling.  When the
+//   stream queue is empty its warps take Top-P items too.
 //
-// pool items (HBM-bound) stream 128x128 bf16 tiles of Q and K once (TMA into
-// a ring of shared-memory stages, several tiles in flight); the block sums are
-// products on the tensor cores (the tile, read transposed, times a column of
-// ones: D[dim] += sum over the block's tokens), so the CUDA cores only turn
-// the sums into the fp32 block means (steps 1-2) and per-block energy partials
-// (step 3);
-// the CTA that finishes the last pool item of a group also computes the
-// group's temperatures (steps 3-4) and publishes "group ready".  score items
-// wait for their group, compute both bands' pooled logits on the tensor cores
-// (step 5; tcgen05 on a three-term bf16 split, fp32 accuracy) and run
-// softmax + Top-P + union per row (steps 5-7).  Scoring of
-// group g overlaps pooling of group g+1.  An
-// item only ever waits for items earlier in the queue, which running CTAs
-// hold and which never wait, so the schedule cannot deadlock; the wait is
+// An item only ever waits for items that running lanes hold and that never
+// wait on the other lane, so the schedule cannot deadlock; every wait is
 // bounded all the same.
 //
 // Band slicing is folded into the pooled layout: the pool items write each
