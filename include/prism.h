@@ -21,8 +21,9 @@
  *   synchronises, and enqueues all work on the caller's `stream` (0 = the
  *   legacy default stream).  Calls are asynchronous: a 0 return means the work
  *   was enqueued, not that it finished.
- * - Layouts (b = batch, hq / hkv = query / key-value heads, N = seqlen,
- *   D = head_dim = 128, nb = N / 128, W = ceil(nb / 32)):
+ * - Layouts (b = batch, hq / hkv = query / key-value heads, N = seqlen (the
+ *   padded length when per-sequence lengths are given), D = head_dim = 128,
+ *   nb = ceil(N / 128), W = ceil(nb / 32)):
  *     q, o        bf16 [b, hq,  N, D]     (Q after RoPE; output O)
  *     k, v        bf16 [b, hkv, N, D]     (K after RoPE)
  *     mask        uint32 [b, hq, nb, W]:  bit (j % 32) of word j / 32 of row i
