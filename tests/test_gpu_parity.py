@@ -318,6 +318,23 @@ def test_variable_length_batch(cuda_device):
         P.check_attention_rows(o1, qs, ks, vs, m1, rows, hq // hkv)
 
 
+def test_widest_gqa_group(cuda_device):
+    """64 Q heads on one KV head (the largest group the temperature step
+    takes): estimator and attention match the oracle."""
+    w = gen.small_workload("gqa64_nb5", 1, 64, 1, 5 * 128 + 40, seed=91, p=0.9)
+    q, k, v, qd, kd, vd = _inputs(w, cuda_device)
+    hi, lo = gen.default_bands()
+    cfg = P.make_cfg(w)
+    mask, sc, tau, words = P.run_estimate(cfg, qd, kd)
+    ref = oracle.estimate(q, k, hi, lo, w.p)
+    P.check_tau(tau, ref)
+    P.check_scores(sc, ref)
+    P.check_mask(mask, ref, w.p)
+    o = P.run_attention(cfg, qd, kd, vd, torch.from_numpy(words.view(np.int32)).to(cuda_device))
+    rows = [(0, h, i) for h in (0, 1, 31, 62, 63) for i in range(w.nb)]
+    P.check_attention_rows(o, q, k, v, mask, rows, 64)
+
+
 def test_small_p_sparse_rows(cuda_device):
     w = gen.small_workload("sparse_nb48", 1, 2, 1, 48 * 128, seed=35, p=0.3)
     q, k, v, qd, kd, vd = _inputs(w, cuda_device)
