@@ -335,6 +335,42 @@ def test_widest_gqa_group(cuda_device):
     P.check_attention_rows(o, q, k, v, mask, rows, 64)
 
 
+@pytest.mark.parametrize("shape", [(1, 2, 1, 128, None), (1, 3, 1, 2 * 128, None), (2, 4, 2, 3 * 128 - 5, None),
+                                   (1, 2, 2, 17 * 128, None), (3, 2, 1, 9 * 128 + 3, [9 * 128 + 3, 1, 300])],
+                         ids=["nb1", "nb2", "nb3_short", "nb17", "varlen"])
+def test_outputs_stay_inside_their_buffers(shape, cuda_device):
+    """The caller's mask and output sit between guard regions filled with a
+    pattern; a prefill over odd shapes (1, 2, 3, 17 blocks, a short last block,
+    a padded batch) writes inside them only, and its mask matches a separate
+    estimate."""
+    b, hq, hkv, n, lens = shape
+    w = gen.small_workload("guard", b, hq, hkv, n, seed=95, p=0.9)
+    q, k, v, qd, kd, vd = _inputs(w, cuda_device)
+    if lens is not None:  # padded batch: zero q, k past each sequence
+        for x, nx in enumerate(lens):
+            qd[x, :, nx:] = 0
+            kd[x, :, nx:] = 0
+    hi, lo = gen.default_bands()
+    cfg = pb.PrismConfig(b, hq, hkv, n, hi, lo, w.p, seqlens=lens)
+    nb, W = cfg.nb, cfg.words
+    guard = 4096
+    m_n, o_n = b * hq * nb * W, b * hq * n * 128
+    m_full = torch.full((guard + m_n + guard,), 0x7E57C0DE, dtype=torch.int32, device=cuda_device)
+    o_full = torch.full((guard + o_n + guard,), 1234.0, dtype=torch.bfloat16, device=cuda_device)
+    mask = m_full[guard:guard + m_n].view(b, hq, nb, W)
+    o = o_full[guard:guard + o_n].view(b, hq, n, 128)
+    ws = torch.empty(pb.prism_workspace_size(cfg), dtype=torch.uint8, device=cuda_device)
+    pb.prism_prefill(cfg, qd, kd, vd, mask, o, ws)
+    torch.cuda.synchronize()
+    assert pb.prism_get_last_device_error() == 0
+    assert torch.all(m_full[:guard] == 0x7E57C0DE) and torch.all(m_full[guard + m_n:] == 0x7E57C0DE)
+    assert torch.all(o_full[:guard] == 1234.0) and torch.all(o_full[guard + o_n:] == 1234.0)
+    mask2 = torch.empty_like(mask)
+    pb.prism_estimate(cfg, qd, kd, mask2, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(mask, mask2)
+
+
 def test_small_p_sparse_rows(cuda_device):
     w = gen.small_workload("sparse_nb48", 1, 2, 1, 48 * 128, seed=35, p=0.3)
     q, k, v, qd, kd, vd = _inputs(w, cuda_device)
