@@ -310,12 +310,11 @@ def run_table(args):
 
 def causal_mask_words(nb: int, words: int) -> torch.Tensor:
     """[nb, words] int32 rows keeping every causal block (p >= 1)."""
-    full = torch.zeros(nb, words, dtype=torch.int64)
-    for i in range(nb):
-        for wd in range(i // 32 + 1):
-            lo = wd * 32
-            full[i, wd] = (1 << 32) - 1 if lo + 32 <= i + 1 else (1 << (i + 1 - lo)) - 1
-    return full.to(torch.int32)
+    i = np.arange(nb, dtype=np.int64)[:, None]
+    lo = 32 * np.arange(words, dtype=np.int64)[None, :]
+    kept = np.clip(i + 1 - lo, 0, 32)  # blocks j <= i in word [lo, lo + 32)
+    bits = np.where(kept == 32, np.int64(0xFFFFFFFF), (np.int64(1) << kept) - 1)
+    return torch.from_numpy(bits.astype(np.uint32).view(np.int32))
 
 
 def run_sweep_p(args):
