@@ -220,6 +220,27 @@ def test_band_choice_matters():
                            r["logits"][:, :, 1][np.isfinite(r["logits"][:, :, 1])])
 
 
+def test_gqa_mapping_equals_repeated_kv_heads():
+    """Q head h reads KV head h // (hq / hkv): with every KV head repeated for
+    its group, the same problem as multi-head attention (one KV head per Q
+    head) gives identical temperatures, logits and masks.  A mapping by
+    h % hkv would pair heads differently and fail."""
+    w = gen.small_workload("gqa_pin", 1, 4, 2, 8 * 128, seed=12)
+    q, k, _ = gen.make_inputs(w, with_v=False)
+    q, k = q.double().numpy(), k.double().numpy()
+    hi, lo = gen.default_bands()
+    g = oracle.estimate(q, k, hi, lo, 0.9)
+    m = oracle.estimate(q, np.repeat(k, 2, axis=1), hi, lo, 0.9)
+    np.testing.assert_array_equal(g["tau"], m["tau"])
+    f = np.isfinite(g["logits"])
+    np.testing.assert_array_equal(g["logits"][f], m["logits"][f])
+    np.testing.assert_array_equal(g["mask"], m["mask"])
+    # and it is not the same as pairing Q head h with KV head h % hkv
+    swapped = np.stack([k[:, 0], k[:, 1], k[:, 0], k[:, 1]], axis=1)
+    s_ = oracle.estimate(q, swapped, hi, lo, 0.9)
+    assert not np.allclose(g["tau"], s_["tau"])
+
+
 # ----------------------------------------------------------------------------
 # softmax rows
 # ----------------------------------------------------------------------------
