@@ -220,6 +220,26 @@ def test_band_choice_matters():
                            r["logits"][:, :, 1][np.isfinite(r["logits"][:, :, 1])])
 
 
+def test_batch_elements_are_independent_problems():
+    """Each batch element is estimated on its own: a batch of two equals the
+    two single-element runs (temperatures, logits, masks), and a change to
+    one element leaves the other's results untouched."""
+    w = gen.small_workload("batch_pin", 2, 2, 1, 6 * 128, seed=13)
+    q, k, _ = gen.make_inputs(w, with_v=False)
+    q, k = q.double().numpy(), k.double().numpy()
+    hi, lo = gen.default_bands()
+    both = oracle.estimate(q, k, hi, lo, 0.9)
+    for b in range(2):
+        one = oracle.estimate(q[b:b + 1], k[b:b + 1], hi, lo, 0.9)
+        np.testing.assert_array_equal(both["tau"][b], one["tau"][0])
+        np.testing.assert_array_equal(both["mask"][b], one["mask"][0])
+    q2 = q.copy()
+    q2[1] *= -1.0
+    other = oracle.estimate(q2, k, hi, lo, 0.9)
+    np.testing.assert_array_equal(other["mask"][0], both["mask"][0])
+    assert not np.array_equal(other["mask"][1], both["mask"][1])
+
+
 def test_gqa_mapping_equals_repeated_kv_heads():
     """Q head h reads KV head h // (hq / hkv): with every KV head repeated for
     its group, the same problem as multi-head attention (one KV head per Q
