@@ -6,10 +6,14 @@ heads, head_dim 128) at N = 131072, seeded synthetic post-RoPE inputs.
 
     python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl prism|reference]
 
-Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent
-layer (weak scaling, no data-path collective); rank 0 prints the job-wide
-ms/layer = max-over-ranks step time / N.  ``--impl reference`` times the fp64
-CPU oracle on a bounded sample of the same layer (rank 0 only).
+Multi-GPU (torchrun, one rank per GPU): the one layer is split across the ranks
+by (batch, KV group) units (block_sparse_attention_band_b200.shard: every unit's
+estimator and attention need only its own heads), with no data-path collective;
+each step every rank runs its share, the step time is the max over ranks and
+``value`` is ms per whole layer (strong scaling).  ``--impl reference`` times
+the fp64 CPU oracle on a bounded sample of the same layer (rank 0 only).
+``--record-traffic CSV`` turns an ncu capture of the DRAM-byte counters into
+``gpurun_out/dram_traffic.json`` keyed by the hash of the CUDA sources.
 """
 from __future__ import annotations
 
@@ -35,7 +39,7 @@ from tests import gen  # noqa: E402
 METRIC = "Prism prefill ms/layer @128K (estimate+sparse attn); estimator overhead %"
 UNIT = "ms/layer"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_llama3_8b_128k.md")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
 KERNEL_SOURCES = ("estimate.cuh", "attention.cuh", "ptx.cuh", "prism.cu")
 KERNELS_PER_STEP = 2  # estimator_kernel + sparse_attn_kernel (the queue reset is a memset)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -60,23 +64,62 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes per launch from the committed ncu summary, keyed by kernel;
-    empty when the summary is missing or the kernels changed since it was taken."""
+def profiled_traffic(workload: str):
+    """DRAM bytes (read + write) per launch of each kernel for ``workload``,
+    from the committed ncu record: the captured workload's bytes per launch
+    times the recorded scale factor (the ratio of units the two workloads
+    process).  Empty when the record is missing, has no factor for the
+    workload, or the CUDA sources differ from the ones profiled."""
     try:
-        text = open(TRAFFIC_FILE).read()
-    except OSError:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
         return {}
-    vals, sha = {}, None
-    for line in text.splitlines():
-        line = line.strip().strip("`")
-        if line.startswith("source_sha256_16:"):
-            sha = line.split(":", 1)[1].strip()
-        elif line.startswith("dram_bytes_per_launch:"):
-            for kv in line.split(":", 1)[1].split():
-                k, v = kv.split("=")
-                vals[k] = float(v)
-    return vals if sha == kernel_source_hash() else {}
+    if rec.get("source_sha256_16") != kernel_source_hash():
+        return {}
+    out = {}
+    for kern, d in rec.get("kernels", {}).items():
+        scale = d.get("scale_to", {}).get(workload, 1.0 if workload == rec.get("workload") else None)
+        if scale is not None:
+            out[kern] = (d["dram_read_bytes_per_launch"] + d["dram_write_bytes_per_launch"]) * scale
+    return out
+
+
+def record_traffic(csv_paths, workload: str, scales, out_path: str):
+    """Parse ncu --csv --print-units base captures of dram__bytes_read.sum /
+    dram__bytes_write.sum and write the per-kernel bytes per launch, with the
+    hash of the current CUDA sources, to ``out_path``."""
+    import csv
+    per = {}
+    for path in csv_paths:
+        with open(path) as f:
+            lines = [ln for ln in f if ln.startswith('"')]
+        for row in csv.DictReader(lines):
+            name = row.get("Kernel Name", "")
+            kern = "estimator_kernel" if "estimator" in name else ("sparse_attn_kernel" if "sparse_attn" in name else None)
+            metric = row.get("Metric Name", "")
+            if kern is None or metric not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+                continue
+            unit = (row.get("Metric Unit") or "byte").lower()
+            mult = {"byte": 1, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9}.get(unit, 1)
+            val = float(str(row["Metric Value"]).replace(",", "")) * mult
+            d = per.setdefault(kern, {}).setdefault(row["ID"], {})
+            d[metric] = val
+    kernels = {}
+    for kern, launches in per.items():
+        rd = [x["dram__bytes_read.sum"] for x in launches.values() if len(x) == 2]
+        wr = [x["dram__bytes_write.sum"] for x in launches.values() if len(x) == 2]
+        if not rd:
+            continue
+        kernels[kern] = {"launches": len(rd), "dram_read_bytes_per_launch": sum(rd) / len(rd),
+                         "dram_write_bytes_per_launch": sum(wr) / len(wr),
+                         "scale_to": {k: v for k, v in scales.items()}}
+    rec = {"source_sha256_16": kernel_source_hash(), "workload": workload, "kernels": kernels,
+           "note": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --print-units base; "
+                   "scale_to: bytes of a launch on another workload = bytes per launch here x factor"}
+    with open(out_path, "w") as f:
+        json.dump(rec, f, indent=1)
+    print(json.dumps(rec))
 
 
 def dist_env():
@@ -146,38 +189,58 @@ class ClockSampler:
                 "power_w_max": max((num(r[3]) or 0.0) for r in rows), "reasons": reasons}
 
 
-def cpu_oracle_sample(q, k, v, mask_words, w, n_heads=1, n_rows=2, seed=0):
+def sample_heads_and_blocks(w, seed: int, n_heads: int = 4, n_blocks: int = 16):
+    """The oracle's sample of a layer: one Q head from each of ``n_heads`` KV
+    groups spread over the layer (the seed picks the head within its group),
+    and query blocks {0, 1, nb/2, nb-1} plus seeded random ones."""
+    rng = np.random.default_rng(seed)
+    g = w.hq // w.hkv
+    n_heads = min(n_heads, w.hkv)
+    groups = sorted({round(x * (w.hkv - 1) / max(n_heads - 1, 1)) for x in range(n_heads)})
+    heads = [kv * g + int(rng.integers(g)) for kv in groups]
+    fixed = sorted({0, min(1, w.nb - 1), w.nb // 2, w.nb - 1})[:n_blocks]
+    blocks = set(fixed)
+    while len(blocks) < min(n_blocks, w.nb):
+        blocks.add(int(rng.integers(w.nb)))
+    return heads, sorted(blocks)
+
+
+def cpu_oracle_sample(q, k, v, mask_words, w, n_heads=4, n_blocks=16, seed=0):
     """Time the fp64 oracle on a bounded sample of the layer and extrapolate to
-    a full layer: estimator on ``n_heads`` Q heads (x Hq / n_heads), attention
-    on ``n_rows`` (head, query block) rows (x total kept tiles / sampled kept tiles)."""
+    a full layer: the estimator on ``n_heads`` Q heads (x Hq / n_heads), the
+    attention on those heads x ``n_blocks`` query blocks (x total kept tiles /
+    sampled kept tiles).  The numbers are extrapolations, labelled so."""
     import oracle
     hi, lo = gen.default_bands()
     g = w.hq // w.hkv
-    rng = np.random.default_rng(seed)
-    heads = sorted(rng.choice(w.hq, n_heads, replace=False).tolist())
+    heads, blocks = sample_heads_and_blocks(w, seed, n_heads, n_blocks)
     t0 = time.perf_counter()
+    own = {}
     for h in heads:
-        oracle.estimate(q[:, h:h + 1], k[:, h // g:h // g + 1], hi, lo, w.p, keep_dense=False)
-    t_est = (time.perf_counter() - t0) * w.hq / n_heads
-    m = oracle.unpack_mask(mask_words, w.nb)[0]
+        r = oracle.estimate(q[:, h:h + 1], k[:, h // g:h // g + 1], hi, lo, w.p, keep_dense=False)
+        own[h] = r["mask"][0, 0]
+    t_est = (time.perf_counter() - t0) * w.hq / len(heads)
     causal = np.tril(np.ones((w.nb, w.nb), dtype=bool))
-    kept_total = int((m & causal).sum())
-    rows = [(int(rng.integers(w.hq)), int(rng.integers(w.nb // 2, w.nb))) for _ in range(n_rows)]
+    if mask_words is not None:  # the layer's mask (all heads): its kept tiles
+        m = oracle.unpack_mask(mask_words, w.nb)[0]
+        kept_total = int((m & causal).sum())
+        rows_of = {h: m[h] for h in heads}
+    else:  # the sampled heads' own oracle masks, their mean kept count x Hq
+        rows_of = own
+        kept_total = int(round(sum(int((own[h] & causal).sum()) for h in heads) * w.hq / len(heads)))
     t0 = time.perf_counter()
     kept_sample = 0
-    for (h, i) in rows:
-        oracle.sparse_attention_block(q, k, v, m[h, i], 0, h, i, g)
-        kept_sample += int(m[h, i, : i + 1].sum())
+    for h in heads:
+        for i in blocks:
+            oracle.sparse_attention_block(q, k, v, rows_of[h][i], 0, h, i, g)
+            kept_sample += int(rows_of[h][i, : i + 1].sum())
     t_attn = (time.perf_counter() - t0) * kept_total / max(kept_sample, 1)
-    sample = (f"estimator on {n_heads} of {w.hq} Q heads x{w.hq / n_heads:g}; attention on {n_rows} "
-              f"(head, query-block) rows ({kept_sample} kept tiles) x{kept_total / max(kept_sample, 1):.0f} "
-              f"(kept-tile ratio); extrapolated to one {w.seqlen}-token layer")
+    sample = (f"extrapolated: estimator on {len(heads)} of {w.hq} Q heads x{w.hq / len(heads):g}; attention on "
+              f"{len(heads)} heads x {len(blocks)} query blocks ({kept_sample} kept tiles) "
+              f"x{kept_total / max(kept_sample, 1):.0f} (kept-tile ratio"
+              f"{'' if mask_words is not None else ', layer kept tiles from the sampled heads'}); "
+              f"one {w.seqlen}-token layer")
     return (t_est + t_attn) * 1e3, t_est * 1e3, t_attn * 1e3, sample
-
-
-def layer_workload(w, rank: int):
-    """Rank r times its own independent layer: the workload with seed + r."""
-    return gen.Workload(**{**w.__dict__, "seed": w.seed + rank})
 
 
 def reduce_max(values, dist, device):
@@ -189,9 +252,13 @@ def reduce_max(values, dist, device):
     return [float(x) for x in t.tolist()]
 
 
-def job_value(ms_step_max: float, world: int) -> float:
-    """Job-wide ms per layer: every rank finishes one layer per step."""
-    return ms_step_max / world
+def reduce_sum(values, dist, device):
+    """Sum over ranks of each value (counts: kept tiles, bytes copied, launches)."""
+    if dist is None:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t.tolist()]
 
 
 def blas_threads():
@@ -204,36 +271,32 @@ def blas_threads():
 
 
 def run_reference(args, w, rank, world):
-    """The oracle timed on the host cores (rank 0 only; other ranks exit)."""
+    """The oracle timed on the host cores (rank 0 only; other ranks exit).
+    Each timed step runs the oracle on a fresh sample of the layer (estimator
+    on 4 Q heads, attention on those heads x 16 query blocks, with the
+    sampled heads' own oracle masks) and extrapolates to the whole layer; the
+    warm-up steps run a minimal sample (1 head, 1 block)."""
     if rank != 0:
         return
     q, k, v = gen.make_inputs(w)
-    # the oracle's own mask for the sampled attention rows (estimator on all heads is
-    # what a CPU run would do; here the mask of the full layer is needed only to
-    # count kept tiles, so it comes from the oracle at p on every head)
-    import oracle
-    hi, lo = gen.default_bands()
-    masks = []
-    g = w.hq // w.hkv
-    for h in range(w.hq):
-        r = oracle.estimate(q[:, h:h + 1], k[:, h // g:h // g + 1], hi, lo, w.p, keep_dense=False)
-        masks.append(r["mask"][0, 0])
-    words = oracle.pack_mask(np.stack(masks)[None])
     vals = []
     sample = ""
     for step in range(args.warmup + args.steps):
-        tot, _, _, sample = cpu_oracle_sample(q, k, v, words, w, n_heads=1, n_rows=1, seed=step)
-        if step >= args.warmup:
+        timed = step >= args.warmup
+        tot, _, _, smp = cpu_oracle_sample(q, k, v, None, w, n_heads=4 if timed else 1,
+                                           n_blocks=16 if timed else 1, seed=step)
+        if timed:
             vals.append(tot)
+            sample = smp
     val = statistics.median(vals)
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": val, "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "scaling": "strong", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "seq_len": w.seqlen,
                    "head_dim": w.head_dim, "block": w.block, "p": w.p},
         "cpu_baseline": {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                         "sample": sample},
+                         "sample": f"median over {args.steps} steps of a fresh sample each; " + sample},
         "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -434,13 +497,24 @@ def main():
     ap.add_argument("--impl", default="prism", choices=["prism", "reference"])
     ap.add_argument("--workload", default="llama3_8b_128k", choices=sorted(gen.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end passes (profiling runs)")
     ap.add_argument("--compare-plain", default=None, choices=sorted(gen.WORKLOADS),
                     help="Prism vs the plain mean-pooling estimator on one workload (attention error vs dense)")
     ap.add_argument("--table", default=None,
                     help="'all' or a comma list of workloads: per-configuration lines instead of the headline")
     ap.add_argument("--sweep-p", default=None,
                     help="comma list of Top-P thresholds: prefill time and density per p on --workload, vs dense")
+    ap.add_argument("--record-traffic", default=None,
+                    help="comma list of ncu CSV files (dram__bytes_*.sum, --print-units base) of --workload")
+    ap.add_argument("--traffic-scale", default="",
+                    help="with --record-traffic: comma list workload=factor (bytes per launch there / here)")
     args = ap.parse_args()
+    if args.record_traffic:
+        scales = dict((kv.split("=")[0], float(kv.split("=")[1])) for kv in args.traffic_scale.split(",") if kv)
+        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+        record_traffic(args.record_traffic.split(","), args.workload, scales,
+                       os.path.join(ROOT, "gpurun_out", "dram_traffic.json"))
+        return
     if args.table:
         run_table(args)
         return
@@ -457,6 +531,7 @@ def main():
         return
 
     import block_sparse_attention_band_b200 as pb
+    from block_sparse_attention_band_b200 import shard
 
     dist = None
     if world > 1:
@@ -467,19 +542,27 @@ def main():
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
 
-    # inputs: rank r runs the layer seeded seed + r (independent layers)
-    wr = layer_workload(w, rank)
-    q, k, v = gen.make_inputs(wr)
-    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    # the one layer, generated identically on every rank; each rank uploads
+    # and runs its share: runs of whole KV groups (shard.shard_runs)
+    q, k, v = gen.make_inputs(w)
+    g = w.hq // w.hkv
     hi, lo = gen.default_bands()
-    cfg = pb.PrismConfig(w.batch, w.hq, w.hkv, w.seqlen, hi, lo, w.p)
-    ws = torch.empty(pb.prism_workspace_size(cfg), dtype=torch.uint8, device=dev)
-    mask = torch.empty(w.batch, w.hq, w.nb, cfg.words, dtype=torch.int32, device=dev)
-    o = torch.empty_like(qd)
+    runs = shard.shard_runs(w.batch, w.hkv, world, rank)
+    parts = []
+    for r in runs:
+        qs, ks, vs, _, _ = shard.run_views(r, g, q, k, v, None, None)
+        cfg = pb.PrismConfig(1, qs.shape[1], ks.shape[1], w.seqlen, hi, lo, w.p)
+        part = {"run": r, "cfg": cfg, "qh": qs.contiguous(), "kh": ks.contiguous(), "vh": vs.contiguous()}
+        part["q"], part["k"], part["v"] = part["qh"].to(dev), part["kh"].to(dev), part["vh"].to(dev)
+        part["ws"] = torch.empty(pb.prism_workspace_size(cfg), dtype=torch.uint8, device=dev)
+        part["mask"] = torch.empty(1, qs.shape[1], w.nb, cfg.words, dtype=torch.int32, device=dev)
+        part["o"] = torch.empty_like(part["q"])
+        parts.append(part)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        pb.prism_prefill(cfg, qd, kd, vd, mask, o, ws, stream=stream)
+        for x in parts:
+            pb.prism_prefill(x["cfg"], x["q"], x["k"], x["v"], x["mask"], x["o"], x["ws"], stream=stream)
 
     def barrier():
         if dist is not None:
@@ -510,45 +593,53 @@ def main():
     for _ in range(args.steps):
         e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         e[0].record(stream)
-        pb.prism_estimate(cfg, qd, kd, mask, ws, stream=stream)
+        for x in parts:
+            pb.prism_estimate(x["cfg"], x["q"], x["k"], x["mask"], x["ws"], stream=stream)
         e[1].record(stream)
-        pb.prism_sparse_attn(cfg, qd, kd, vd, mask, o, stream=stream)
+        for x in parts:
+            pb.prism_sparse_attn(x["cfg"], x["q"], x["k"], x["v"], x["mask"], x["o"], stream=stream)
         e[2].record(stream)
         torch.cuda.synchronize()
         est_ms.append(e[0].elapsed_time(e[1]))
         attn_ms.append(e[1].elapsed_time(e[2]))
-    t_est = statistics.median(est_ms)
-    t_attn = statistics.median(attn_ms)
+    t_est_own, t_attn_own = statistics.median(est_ms), statistics.median(attn_ms)
+    t_est, t_attn = reduce_max([t_est_own, t_attn_own], dist, dev)
     # the same attention kernel on every causal block (p = 1): the dense
     # prefill the method is set against (context for the speed-up, not timed
     # in the step)
-    dense_mask = causal_mask_words(w.nb, cfg.words).expand(w.batch, w.hq, w.nb, cfg.words).contiguous().to(dev)
     dense_ms = []
+    dense_masks = [causal_mask_words(w.nb, x["cfg"].words).expand(1, x["q"].shape[1], w.nb, x["cfg"].words)
+                   .contiguous().to(dev) for x in parts]
     for _ in range(3):
         e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         e[0].record(stream)
-        pb.prism_sparse_attn(cfg, qd, kd, vd, dense_mask, o, stream=stream)
+        for x, dm in zip(parts, dense_masks):
+            pb.prism_sparse_attn(x["cfg"], x["q"], x["k"], x["v"], dm, x["o"], stream=stream)
         e[1].record(stream)
         torch.cuda.synchronize()
         dense_ms.append(e[0].elapsed_time(e[1]))
-    t_dense = statistics.median(dense_ms)
-    del dense_mask
+    t_dense = reduce_max([statistics.median(dense_ms)], dist, dev)[0]
+    del dense_masks
 
-    words = mask.cpu().numpy().view(np.uint32)
+    words_parts = [x["mask"].cpu().numpy().view(np.uint32) for x in parts]
     nb = w.nb
-    causal_tiles = w.batch * w.hq * nb * (nb + 1) // 2
-    kept = int(np.unpackbits(words.view(np.uint8)).sum())  # bits j > i are 0 by contract
-    density = kept / causal_tiles
+    kept_own = sum(int(np.unpackbits(wp.view(np.uint8)).sum()) for wp in words_parts)  # bits j > i are 0
+    own_heads = sum(x["q"].shape[1] for x in parts)
     flops_tile = 4 * 128 * 128 * 128
-    attn_flops = kept * flops_tile
-    attn_tflops = attn_flops / (t_attn * 1e-3) / 1e12
-    est_bytes = (w.hq + w.hkv) * w.batch * w.seqlen * 128 * 2 + words.nbytes
+    est_bytes_own = sum((x["q"].shape[1] + x["k"].shape[1]) * w.seqlen * 128 * 2 for x in parts) + \
+        sum(wp.nbytes for wp in words_parts)
+    kept, est_bytes = reduce_sum([kept_own, est_bytes_own], dist, dev)
+    kept = int(kept)
+    causal_tiles = w.batch * w.hq * nb * (nb + 1) // 2
+    density = kept / causal_tiles
+    # per-GPU roofline of this rank's kernels (rank 0 prints its own)
+    attn_tflops = kept_own * flops_tile / (t_attn_own * 1e-3) / 1e12 if kept_own else 0.0
+    est_gbs = est_bytes_own / (t_est_own * 1e-3) / 1e9 if parts else 0.0
 
     peaks, peak_src = load_peaks()
-    traffic = profiled_traffic() if w.name == "llama3_8b_128k" else {}
+    traffic = profiled_traffic(w.name) if world == 1 else {}
     peak_tensor = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     peak_hbm = peaks["hbm_gbs"]
-    est_gbs = est_bytes / (t_est * 1e-3) / 1e9
 
     # ---------------- end to end: pinned host buffers, copies timed ---------
     # Every step uploads its Q, K, V from pinned host memory, runs the prefill
@@ -556,99 +647,113 @@ def main():
     # step at a time on one stream.  Pipelined (the reported value): two device
     # buffer sets and three streams, so step s+1's upload and step s-1's
     # download run beside step s's kernels; timed from the first upload to the
-    # last download, divided by the steps.
-    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
-    ohs = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(2)]
-    e2e_serial = []
-    for it in range(args.steps + 1):
-        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ea.record(stream)
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        step()
-        ohs[0].copy_(o, non_blocking=True)
-        eb.record(stream)
-        torch.cuda.synchronize()
-        if it > 0:
-            e2e_serial.append(ea.elapsed_time(eb))
-    e2e_serial_ms = reduce_max([statistics.median(e2e_serial)], dist, dev)[0]
-    sets = [(qd, kd, vd, o), (torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd), torch.empty_like(o))]
-    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    # last download, divided by the steps.  Each rank moves its own share.
+    e2e = None
+    if not args.no_e2e:
+        for x in parts:
+            x["qp"], x["kp"], x["vp"] = x["qh"].pin_memory(), x["kh"].pin_memory(), x["vh"].pin_memory()
+            x["op"] = [torch.empty(x["o"].shape, dtype=x["o"].dtype).pin_memory() for _ in range(2)]
+        e2e_serial = []
+        for it in range(args.steps + 1):
+            ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ea.record(stream)
+            for x in parts:
+                x["q"].copy_(x["qp"], non_blocking=True)
+                x["k"].copy_(x["kp"], non_blocking=True)
+                x["v"].copy_(x["vp"], non_blocking=True)
+            step()
+            for x in parts:
+                x["op"][0].copy_(x["o"], non_blocking=True)
+            eb.record(stream)
+            torch.cuda.synchronize()
+            if it > 0:
+                e2e_serial.append(ea.elapsed_time(eb))
+        e2e_serial_ms = reduce_max([statistics.median(e2e_serial)], dist, dev)[0]
+        for x in parts:
+            x["sets"] = [(x["q"], x["k"], x["v"], x["o"]), (torch.empty_like(x["q"]), torch.empty_like(x["k"]),
+                                                           torch.empty_like(x["v"]), torch.empty_like(x["o"]))]
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def pipelined(n_steps):
-        ev = {}
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        t0.record(up)
-        for s_ in range(n_steps):
-            qx, kx, vx, ox = sets[s_ % 2]
-            if s_ >= 2:
-                up.wait_event(ev[("done", s_ - 2)])  # step s-2 has read this input set
-            with torch.cuda.stream(up):
-                qx.copy_(qh, non_blocking=True)
-                kx.copy_(kh, non_blocking=True)
-                vx.copy_(vh, non_blocking=True)
-            ev[("in", s_)] = torch.cuda.Event()
-            ev[("in", s_)].record(up)
-            stream.wait_event(ev[("in", s_)])
-            if s_ >= 2:
-                stream.wait_event(ev[("out", s_ - 2)])  # step s-2's output has been downloaded
-            pb.prism_prefill(cfg, qx, kx, vx, mask, ox, ws, stream=stream)
-            ev[("done", s_)] = torch.cuda.Event()
-            ev[("done", s_)].record(stream)
-            down.wait_event(ev[("done", s_)])
-            with torch.cuda.stream(down):
-                ohs[s_ % 2].copy_(ox, non_blocking=True)
-            ev[("out", s_)] = torch.cuda.Event()
-            ev[("out", s_)].record(down)
-        t1.record(down)
-        torch.cuda.synchronize()
-        return t0.elapsed_time(t1) / n_steps
+        def pipelined(n_steps):
+            ev = {}
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(up)
+            for s_ in range(n_steps):
+                if s_ >= 2:
+                    up.wait_event(ev[("done", s_ - 2)])  # step s-2 has read this input set
+                with torch.cuda.stream(up):
+                    for x in parts:
+                        qx, kx, vx, _ = x["sets"][s_ % 2]
+                        qx.copy_(x["qp"], non_blocking=True)
+                        kx.copy_(x["kp"], non_blocking=True)
+                        vx.copy_(x["vp"], non_blocking=True)
+                ev[("in", s_)] = torch.cuda.Event()
+                ev[("in", s_)].record(up)
+                stream.wait_event(ev[("in", s_)])
+                if s_ >= 2:
+                    stream.wait_event(ev[("out", s_ - 2)])  # step s-2's output has been downloaded
+                for x in parts:
+                    qx, kx, vx, ox = x["sets"][s_ % 2]
+                    pb.prism_prefill(x["cfg"], qx, kx, vx, x["mask"], ox, x["ws"], stream=stream)
+                ev[("done", s_)] = torch.cuda.Event()
+                ev[("done", s_)].record(stream)
+                down.wait_event(ev[("done", s_)])
+                with torch.cuda.stream(down):
+                    for x in parts:
+                        x["op"][s_ % 2].copy_(x["sets"][s_ % 2][3], non_blocking=True)
+                ev[("out", s_)] = torch.cuda.Event()
+                ev[("out", s_)].record(down)
+            t1.record(down)
+            torch.cuda.synchronize()
+            return t0.elapsed_time(t1) / n_steps
 
-    pipelined(2)  # warm-up of the streams and the second buffer set
-    e2e_ms = reduce_max([pipelined(args.steps)], dist, dev)[0]
-    assert pb.prism_get_last_device_error() == 0
-    h2d = qh.nbytes + kh.nbytes + vh.nbytes
-    d2h = ohs[0].nbytes
+        pipelined(2)  # warm-up of the streams and the second buffer set
+        e2e_ms = reduce_max([pipelined(args.steps)], dist, dev)[0]
+        assert pb.prism_get_last_device_error() == 0
+        h2d, d2h = reduce_sum([sum(x["qp"].nbytes + x["kp"].nbytes + x["vp"].nbytes for x in parts),
+                               sum(x["op"][0].nbytes for x in parts)], dist, dev)
+        e2e = {"value": e2e_ms, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "mode": "pipelined: step s+1 upload and step s-1 download beside step s (2 buffer sets, 3 streams)",
+               "serial_value": e2e_serial_ms}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tot, ce, ca, sample = cpu_oracle_sample(q, k, v, words, w, n_heads=2, n_rows=2)
+        tot, ce, ca, sample = cpu_oracle_sample(q, k, v, words_parts[0], w, n_heads=4, n_blocks=16)
         cpu = {"value": tot, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample,
                "estimator_ms": ce, "attention_ms": ca}
 
+    launches = reduce_sum([KERNELS_PER_STEP * len(parts) * args.steps], dist, dev)[0]
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
         return
-    value = job_value(ms_step, world)
+    per_rank = [sum(x.kv1 - x.kv0 for x in shard.shard_runs(w.batch, w.hkv, world, r_)) for r_ in range(world)]
+    share = f"{world} rank(s), KV groups per rank {per_rank}"
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
+        "metric": METRIC, "value": ms_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "strong",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "seq_len": w.seqlen,
                    "head_dim": w.head_dim, "block": w.block, "p": w.p,
                    "l2": "inputs (Q+K+V 1.6 GB) larger than L2; no flush",
-                   "parallelism": f"{world} independent layers (one per GPU)"},
+                   "parallelism": f"one layer split by KV group over {world} GPU(s), no data-path collective"},
         "estimator_overhead_pct": 100.0 * t_est / (t_est + t_attn),
         "stages": {"estimate_ms": t_est, "attention_ms": t_attn, "prefill_ms": ms_step,
                    "density": density, "kept_tiles": kept, "causal_tiles": causal_tiles,
-                   "attention_tflops": attn_tflops, "effective_tflops_vs_dense":
-                       causal_tiles * flops_tile / (ms_step * 1e-3) / 1e12,
-                   "estimator_gbs": est_gbs, "estimator_hbm_frac": est_gbs / peak_hbm,
-                   "dense_attention_ms": t_dense, "speedup_vs_dense": t_dense / ms_step},
+                   "effective_tflops_vs_dense": causal_tiles * flops_tile / (ms_step * 1e-3) / 1e12,
+                   "dense_attention_ms": t_dense, "speedup_vs_dense": t_dense / ms_step,
+                   "shards": share},
         "roofline": {"kernel": "sparse_attn_kernel", "bound": "tensor", "achieved": attn_tflops,
                      "peak": peak_tensor, "unit": "TFLOP/s", "frac": attn_tflops / peak_tensor,
                      "traffic": traffic.get("sparse_attn_kernel"),
-                     "peak_source": f"{peak_src} bf16 sustained (of {peak_src})"},
+                     "algorithmic_flops": kept_own * flops_tile,
+                     "peak_source": f"bf16 sustained (of {peak_src})", "scope": "rank 0's kernels"},
         "estimator_roofline": {"kernel": "estimator_kernel", "bound": "hbm", "achieved": est_gbs,
                                "peak": peak_hbm, "unit": "GB/s", "frac": est_gbs / peak_hbm,
-                               "algorithmic_bytes": est_bytes, "traffic": traffic.get("estimator_kernel"),
-                               "peak_source": f"{peak_src} copy bandwidth (of {peak_src})"},
-        "e2e": {"value": job_value(e2e_ms, world), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "mode": "pipelined: step s+1 upload and step s-1 download beside step s (2 buffer sets, 3 streams)",
-                "serial_value": job_value(e2e_serial_ms, world)},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+                               "algorithmic_bytes": est_bytes_own, "traffic": traffic.get("estimator_kernel"),
+                               "peak_source": f"copy bandwidth (of {peak_src})", "scope": "rank 0's kernels"},
+        "e2e": e2e,
+        "gpu_launches": int(launches),
         "clocks": clocks,
         "cpu_baseline": cpu,
     }

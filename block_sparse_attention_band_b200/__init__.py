@@ -61,6 +61,11 @@ class _Config(ctypes.Structure):
     ]
 
 
+class _Debug(ctypes.Structure):
+    _fields_ = [("scores", ctypes.c_void_p), ("weights", ctypes.c_void_p), ("tau", ctypes.c_void_p),
+                ("pooled", ctypes.c_void_p)]
+
+
 _vp = ctypes.c_void_p
 _cfgp = ctypes.POINTER(_Config)
 lib.prism_version.restype = ctypes.c_int
@@ -69,7 +74,7 @@ lib.prism_status_str.argtypes = [ctypes.c_int]
 lib.prism_workspace_size.restype = ctypes.c_int
 lib.prism_workspace_size.argtypes = [_cfgp, ctypes.POINTER(ctypes.c_size_t)]
 lib.prism_estimate.restype = ctypes.c_int
-lib.prism_estimate.argtypes = [_cfgp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp, _vp, _vp]
+lib.prism_estimate.argtypes = [_cfgp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp, ctypes.POINTER(_Debug)]
 lib.prism_sparse_attn.restype = ctypes.c_int
 lib.prism_sparse_attn.argtypes = [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.prism_prefill.restype = ctypes.c_int
@@ -203,10 +208,15 @@ def prism_workspace_size(cfg: PrismConfig) -> int:
 
 
 def prism_estimate(cfg: PrismConfig, q, k, mask, workspace, stream=None, dbg_scores=None,
-                   dbg_tau=None) -> None:
+                   dbg_tau=None, dbg_weights=None, dbg_pooled=None) -> None:
+    """The estimator; the ``dbg_*`` tensors (optional, fp32 on the device)
+    receive the members of ``prism_debug`` (include/prism.h)."""
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    dbg = None
+    if any(x is not None for x in (dbg_scores, dbg_tau, dbg_weights, dbg_pooled)):
+        dbg = ctypes.byref(_Debug(_addr(dbg_scores), _addr(dbg_weights), _addr(dbg_tau), _addr(dbg_pooled)))
     _check(lib.prism_estimate(cfg.ptr(), _addr(q), _addr(k), _addr(mask), _addr(workspace), ws_bytes,
-                              _stream(stream), _addr(dbg_scores), _addr(dbg_tau)), "prism_estimate")
+                              _stream(stream), dbg), "prism_estimate")
 
 
 def prism_sparse_attn(cfg: PrismConfig, q, k, v, mask, o, stream=None) -> None:

@@ -105,9 +105,11 @@ struct EstParams {
   float* part;    // [q_rows + kv_rows, nb, 4] sum(mean^2): hi, lo, all
   float* tau;     // [q_rows, 4]: tau_hi, tau_lo, 1/(tau_hi sqrt d_hi), 1/(tau_lo sqrt d_lo)
   float* scores;      // scaled band logits in 128 x 128 tiles: [q_rows][tile (cr, cc), cc <= cr][band][128][128]
-  float* dbg_scores;  // optional copy in packed lower-triangular rows [q_rows, 2, nb(nb+1)/2]
+  float* dbg_scores;   // optional copy in packed lower-triangular rows [q_rows, 2, nb(nb+1)/2]
+  float* dbg_weights;  // optional: the Top-P's softmax weights e_j, same packing
   uint32_t* mask;
   float* dbg_tau;
+  float* dbg_pooled;   // optional: block means [q_rows + kv_rows, nb, 128], all dims
   float* rmax;     // [q_rows, nb, rparts, 2] scaled band logits' row maxima over the key blocks j <= i
                    // of each part
   uint32_t* ready;  // [q_rows, ceil(nb / kToppRows)] mask rows of a Top-P item written
@@ -472,6 +474,7 @@ __device__ __forceinline__ void pool_item(const EstParams& P, const CUtensorMap*
         const float inv = blk == nbb - 1 ? 1.0f / (float)(seq_tokens(P, bi) - 128 * (nbb - 1)) : (1.0f / 128.0f);
         const float m = __uint_as_float(v[b]) * inv;
         const bool ok = b0 + b < nt;
+        if (ok && P.dbg_pooled) P.dbg_pooled[((size_t)hr * P.nb + blk) * 128 + d] = m;
         if (ok && c != 255) {
           const __nv_bfloat16 th = __float2bfloat16_rn(m);
           const float r1 = m - __bfloat162float(th);
@@ -676,7 +679,7 @@ __device__ __forceinline__ unsigned long long bin_mass(const uint32_t* lo, const
 constexpr size_t kTilePair = 2 * 128 * 128;  // floats per score tile pair (both bands)
 
 __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const ToppScratch& S, uint32_t* bits,
-                                              float* dbg, int lane) {
+                                              float* dbg, float* dbgw, int lane) {
   const unsigned lt = (1u << lane) - 1u;
   const float* row = reinterpret_cast<const float*>(S.d);
   if (dbg)
@@ -796,6 +799,8 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
       if (o.x < me.x || (o.x == me.x && o.y < me.y)) ahead += o.z;
     }
     if (lane < cnt && ahead < lim) atomicOr(&bits[me.y >> 5], 1u << (me.y & 31));
+    if (dbgw)
+      for (int j = lane; j < n; j += 32) dbgw[j] = key_value(S.d[j]);
     __syncwarp();
     return;
   }
@@ -906,6 +911,9 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
     }
   }
   __syncwarp();
+  // the weights e_j as ranked and summed (debug output)
+  if (dbgw)
+    for (int j = lane; j < n; j += 32) dbgw[j] = key_value(S.d[j]);
   // every block ranked at or ahead of the crossing
   const uint32_t dc = cross >= 0 ? S.d[cross] : 0xffffffffu;
   for (int j0 = 0; j0 < n; j0 += 32) {
@@ -1219,14 +1227,15 @@ __device__ __forceinline__ void topp_item(const EstParams& P, int g, int y, cons
     const float rmax_t = __shfl_sync(0xffffffffu, my_rmax, task & 31);
     const float rmax = task < 32 ? rmax_t : row_max(i, band);
     S.d = reinterpret_cast<uint32_t*>(wb + (size_t)(task & (nbuf - 1)) * nbp * 4);
-    float* dbg = P.dbg_scores ? P.dbg_scores + (size_t)bh * 2 * tri + (size_t)band * tri + (size_t)i * (i + 1) / 2
-                              : nullptr;
+    const size_t drow = (size_t)bh * 2 * tri + (size_t)band * tri + (size_t)i * (i + 1) / 2;
+    float* dbg = P.dbg_scores ? P.dbg_scores + drow : nullptr;
+    float* dbgw = P.dbg_weights ? P.dbg_weights + drow : nullptr;
     uint32_t* dst = P.mask + ((size_t)bh * P.nb + i) * P.W;
     if (band == 0) {
       for (int w = lane; w < P.W; w += 32) bits[w] = 0u;
       __syncwarp();
     }
-    topp_band_row(rmax, n, P.p, S, bits, dbg, lane);
+    topp_band_row(rmax, n, P.p, S, bits, dbg, dbgw, lane);
     if (band == 1) {
       if (P.force && lane == 0) {  // optional additions to M_high | M_low
         if (P.force & 1) bits[0] |= 1u;

@@ -309,7 +309,7 @@ size_t ready_offset(const Plan& P) {
 }
 
 int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, unsigned char* ws,
-                 cudaStream_t st, float* dbg_scores, float* dbg_tau) {
+                 cudaStream_t st, const prism_debug* dbg) {
   EstParams E;
   E.q = reinterpret_cast<const __nv_bfloat16*>(q);
   E.k = reinterpret_cast<const __nv_bfloat16*>(k);
@@ -318,9 +318,11 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   E.part = reinterpret_cast<float*>(ws + P.off_part);
   E.tau = reinterpret_cast<float*>(ws + P.off_tau);
   E.scores = reinterpret_cast<float*>(ws + P.off_scores);
-  E.dbg_scores = dbg_scores;
+  E.dbg_scores = dbg ? dbg->scores : nullptr;
+  E.dbg_weights = dbg ? dbg->weights : nullptr;
+  E.dbg_tau = dbg ? dbg->tau : nullptr;
+  E.dbg_pooled = dbg ? dbg->pooled : nullptr;
   E.mask = mask;
-  E.dbg_tau = dbg_tau;
   E.rmax = reinterpret_cast<float*>(ws + P.off_rmax);
   E.sync = reinterpret_cast<uint32_t*>(ws + P.off_sync);
   E.ready = E.sync + ready_offset(P);
@@ -486,19 +488,20 @@ int prism_workspace_size(const prism_config* cfg, size_t* bytes) {
 }
 
 int prism_estimate(const prism_config* cfg, const void* q, const void* k, uint32_t* mask,
-                   void* workspace, size_t workspace_bytes, prism_stream_t stream, float* dbg_scores,
-                   float* dbg_tau) {
+                   void* workspace, size_t workspace_bytes, prism_stream_t stream, const prism_debug* dbg) {
   Plan P;
   int s = validate(cfg, &P);
   if (s != PRISM_OK) return s;
   if (!q || !k || !mask) return PRISM_ERR_NULL;
   if (!workspace || workspace_bytes < P.total) return PRISM_ERR_WORKSPACE;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(mask, 16) || !aligned(workspace, 256) ||
-      (dbg_scores && !aligned(dbg_scores, 16)) || (dbg_tau && !aligned(dbg_tau, 4)))
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(mask, 16) || !aligned(workspace, 256))
+    return PRISM_ERR_ALIGN;
+  if (dbg && ((dbg->scores && !aligned(dbg->scores, 16)) || (dbg->weights && !aligned(dbg->weights, 16)) ||
+              (dbg->tau && !aligned(dbg->tau, 4)) || (dbg->pooled && !aligned(dbg->pooled, 16))))
     return PRISM_ERR_ALIGN;
   if ((s = ensure_device()) != PRISM_OK) return s;
   return run_estimate(P, q, k, mask, static_cast<unsigned char*>(workspace),
-                      reinterpret_cast<cudaStream_t>(stream), dbg_scores, dbg_tau);
+                      reinterpret_cast<cudaStream_t>(stream), dbg);
 }
 
 int prism_sparse_attn(const prism_config* cfg, const void* q, const void* k, const void* v,
@@ -528,7 +531,7 @@ int prism_prefill(const prism_config* cfg, const void* q, const void* k, const v
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   uint32_t* mask = mask_out ? mask_out : reinterpret_cast<uint32_t*>(ws + P.off_mask);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if ((s = run_estimate(P, q, k, mask, ws, st, nullptr, nullptr)) != PRISM_OK) return s;
+  if ((s = run_estimate(P, q, k, mask, ws, st, nullptr)) != PRISM_OK) return s;
   // the attention starts on query blocks whose masks are final while the
   // estimator finishes the others
   const uint32_t* ready = reinterpret_cast<const uint32_t*>(ws + P.off_sync) + ready_offset(P);
@@ -552,7 +555,7 @@ int prism_estimate_noalloc(const prism_config* cfg, const void* q, const void* k
   void* scratch = nullptr;
   if ((s = static_scratch(&scratch)) != PRISM_OK) return s;
   return run_estimate(P, q, k, mask, static_cast<unsigned char*>(scratch),
-                      reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr);
+                      reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
 
 size_t prism_noalloc_scratch_bytes(void) { return kStaticScratchBytes; }

@@ -144,20 +144,46 @@ enum { PRISM_FORCE_SINK = 1, PRISM_FORCE_DIAG = 2 };
 int prism_workspace_size(const prism_config* cfg, size_t* bytes);
 
 /*
+ * Optional copies of the estimator's intermediate values, for checking each
+ * step on its own (the paper has no counterpart: these are test outputs).
+ * Every member may be NULL (not written); all are DEVICE pointers, fp32,
+ * owned by the caller, 16-byte aligned (tau: 4-byte).  nb(nb+1)/2 = T.
+ *   scores   [b, hq, 2 (hi, lo), T]: the scaled band logits of step (5),
+ *            L_z[i][j] = Qbar_z[i] . Kbar_z[j] / (tau_z sqrt(d_z)), in packed
+ *            lower-triangular rows (row i starts at i(i+1)/2, j = 0..i).
+ *   weights  [b, hq, 2, T], same packing: the unnormalised softmax weights
+ *            e_j = 2^((L_j - max_k L_k) log2 e) in (0, 1] exactly as the Top-P
+ *            step ranks and sums them (step (6): block j is kept iff the sum
+ *            of round(e_k 2^31) over the blocks ranked ahead of it, by (-e, k),
+ *            is below max(floor(p Z), 1), Z the row's sum of round(e_k 2^31)).
+ *            Written only when p < 1.
+ *   tau      [b, hq, 2] = (tau_hi, tau_lo) of step (4).
+ *   pooled   [b hq + b hkv, nb, 128]: the block means of step (2) over all
+ *            128 dims (rows: the b hq query heads batch-major, then the b hkv
+ *            key heads batch-major); a short last block is the mean over its
+ *            tokens; blocks past a sequence (per-sequence lengths) are not
+ *            written.
+ */
+typedef struct prism_debug {
+  float* scores;
+  float* weights;
+  float* tau;
+  float* pooled;
+} prism_debug;
+
+/*
  * Estimator, steps (1)-(7) of [review:method]: band slicing and mean pooling
  * per block of B = 128 tokens, RMS energy of each pooled band, temperatures,
  * dual-band pooled softmax scores, Top-P per query-block row and band, union.
  *   q, k        inputs (layouts above)
  *   mask        output, uint32 [b, hq, nb, W]; every word written
  *   workspace   >= prism_workspace_size(cfg) bytes, 256-byte aligned
- *   dbg_scores  optional (NULL: unused) fp32 output holding the scaled band
- *               scores L_z in packed lower-triangular rows:
- *               [b, hq, 2 (hi, lo), nb(nb+1)/2], row i starting at i(i+1)/2
- *   dbg_tau     optional fp32 output [b, hq, 2] = (tau_hi, tau_lo)
+ *   dbg         optional (NULL: none) debug outputs, see prism_debug; the
+ *               struct is read during the call only
  */
 int prism_estimate(const prism_config* cfg, const void* q, const void* k, uint32_t* mask,
                    void* workspace, size_t workspace_bytes, prism_stream_t stream,
-                   float* dbg_scores, float* dbg_tau);
+                   const prism_debug* dbg);
 
 /*
  * Causal block-sparse attention ([summary:1]: only the selected blocks are

@@ -55,21 +55,23 @@ def _ws_size(cfg):
     return pb.lib.prism_workspace_size(cfg.ptr(), ctypes.byref(n)), n.value
 
 
-def test_workspace_size_formula():
-    s, n = _ws_size(_cfg())
-    assert s == 0
-    nb, rows, q_rows = 8, 6, 4
-    # scores: one 128 x 128 tile pair (row chunk 0, column chunk 0) per Q row
-
-    def up(x):
-        return (x + 255) // 256 * 256
-    kv_rows = rows - q_rows
-    dp = 128  # default bands: 32 high-only + 32 shared + 64 low-only padded columns
-    nch = 1  # score chunks of 128 query blocks
-    expect = 3 * up(rows * nb * dp * 2) + up(rows * nb * 4 * 4) + up(q_rows * 16) \
-        + up(q_rows * nch * 2 * 128 * 128 * 4) + up(q_rows * nb * 1 * 2 * 4) + up(q_rows * nb * 1 * 4) \
-        + up((2 + 2 * kv_rows + q_rows * nch + q_rows * ((nb + 15) // 16)) * 4)
-    assert n == expect
+def test_workspace_size_properties():
+    """The workspace grows with the sequence, the heads and the batch, and a
+    call with one byte less than the reported size is refused before anything
+    is enqueued."""
+    s, base = _ws_size(_cfg())
+    assert s == 0 and base > 0 and base % 256 == 0
+    sizes_n = [_ws_size(_cfg(seqlen=n))[1] for n in (128, 1024, 4096, 32768, 131072)]
+    assert all(a < b for a, b in zip(sizes_n, sizes_n[1:])), sizes_n
+    sizes_h = [_ws_size(_cfg(hq=hq, hkv=hkv))[1] for hq, hkv in ((1, 1), (2, 1), (4, 2), (8, 2), (32, 8))]
+    assert all(a < b for a, b in zip(sizes_h, sizes_h[1:])), sizes_h
+    assert _ws_size(_cfg(batch=2))[1] > base
+    # every pooled value needs at least 3 x 2 bytes per kept dim: a floor that any layout meets
+    assert base >= 6 * (4 + 2) * 8 * 128
+    a = 1 << 20
+    cfg = _cfg()
+    assert pb.lib.prism_estimate(cfg.ptr(), a, a, a, a, base - 1, None, None) == -7
+    assert pb.lib.prism_prefill(cfg.ptr(), a, a, a, a, a, a, base - 1, None) == -7
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -85,7 +87,7 @@ def test_bad_config_rejected_on_host(kw, code):
     assert s == code, pb.prism_status_str(s)
     # the compute entry points reject the same config before any CUDA call
     fake = 1 << 20
-    assert pb.lib.prism_estimate(_cfg(**kw).ptr(), fake, fake, fake, fake, 1 << 40, None, None, None) == code
+    assert pb.lib.prism_estimate(_cfg(**kw).ptr(), fake, fake, fake, fake, 1 << 40, None, None) == code
     assert pb.lib.prism_sparse_attn(_cfg(**kw).ptr(), fake, fake, fake, fake, fake, None) == code
     assert pb.lib.prism_prefill(_cfg(**kw).ptr(), fake, fake, fake, None, fake, fake, 1 << 40, None) == code
 
@@ -107,12 +109,12 @@ def test_null_pointers_workspace_and_alignment_rejected():
     a = 1 << 20
     assert pb.lib.prism_workspace_size(None, ctypes.byref(ctypes.c_size_t())) == -1
     assert pb.lib.prism_workspace_size(cfg.ptr(), None) == -1
-    assert pb.lib.prism_estimate(cfg.ptr(), None, a, a, a, ws, None, None, None) == -1
-    assert pb.lib.prism_estimate(cfg.ptr(), a, a, None, a, ws, None, None, None) == -1
-    assert pb.lib.prism_estimate(cfg.ptr(), a, a, a, None, ws, None, None, None) == -7
-    assert pb.lib.prism_estimate(cfg.ptr(), a, a, a, a, ws - 1, None, None, None) == -7
-    assert pb.lib.prism_estimate(cfg.ptr(), a + 8, a, a, a, ws, None, None, None) == -3
-    assert pb.lib.prism_estimate(cfg.ptr(), a, a, a, a + 16, ws, None, None, None) == -3
+    assert pb.lib.prism_estimate(cfg.ptr(), None, a, a, a, ws, None, None) == -1
+    assert pb.lib.prism_estimate(cfg.ptr(), a, a, None, a, ws, None, None) == -1
+    assert pb.lib.prism_estimate(cfg.ptr(), a, a, a, None, ws, None, None) == -7
+    assert pb.lib.prism_estimate(cfg.ptr(), a, a, a, a, ws - 1, None, None) == -7
+    assert pb.lib.prism_estimate(cfg.ptr(), a + 8, a, a, a, ws, None, None) == -3
+    assert pb.lib.prism_estimate(cfg.ptr(), a, a, a, a + 16, ws, None, None) == -3
     assert pb.lib.prism_sparse_attn(cfg.ptr(), a, a, a, a, None, None) == -1
     assert pb.lib.prism_sparse_attn(cfg.ptr(), a, a, a + 2, a, a, None) == -3
     assert pb.lib.prism_prefill(cfg.ptr(), a, a, a, None, a, None, ws, None) == -7

@@ -1,6 +1,7 @@
 """Full-size workloads in the launch configuration bench.py times
 (prism_prefill, workspace, mask out), checked on samples the oracle can
-compute one by one, plus properties that hold at any size.
+compute one by one, plus properties that hold at any size.  Every length of
+the long-context sweep (8K, 16K, 64K, 128K, 256K) is checked.
 
 Sampling: the estimator oracle runs on 4 Q heads (one from each of 4 KV
 groups, the seed picks the head within the group); the attention oracle on
@@ -19,7 +20,8 @@ from tests import parity as P
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
-FULL = ["llama3_8b_32k", "llama3_8b_128k", "qwen3_8b_64k_planted", "sweep_8k", "sweep_256k"]
+FULL = ["llama3_8b_32k", "llama3_8b_128k", "qwen3_8b_64k_planted",
+        "sweep_8k", "sweep_16k", "sweep_64k", "sweep_128k", "sweep_256k"]
 
 
 def _sample_heads(w, rng):
@@ -54,11 +56,24 @@ def test_full_size_sampled_parity(name, cuda_device):
     heads = _sample_heads(w, rng)
     tri = nb * (nb + 1) // 2
     scores = torch.empty(w.batch, w.hq, 2, tri, dtype=torch.float32, device=cuda_device)
+    weights = torch.empty(w.batch, w.hq, 2, tri, dtype=torch.float32, device=cuda_device)
     tau = torch.empty(w.batch, w.hq, 2, dtype=torch.float32, device=cuda_device)
+    pooled = torch.empty(w.batch * (w.hq + w.hkv), nb, 128, dtype=torch.float32, device=cuda_device)
     mask2 = torch.empty_like(mask)
-    pb.prism_estimate(cfg, qd, kd, mask2, ws, dbg_scores=scores, dbg_tau=tau)
+    pb.prism_estimate(cfg, qd, kd, mask2, ws, dbg_scores=scores, dbg_tau=tau, dbg_weights=weights,
+                      dbg_pooled=pooled)
     torch.cuda.synchronize()
     assert torch.equal(mask2, mask), "estimate and prefill disagree on the mask"
+    # pooled means of the sampled Q heads and their KV heads, element by element
+    g = w.hq // w.hkv
+    prow = heads + sorted({w.hq + h // g for h in heads})
+    P.check_pooled(pooled[prow].cpu().double().numpy(), q, k, only=prow)
+    del pooled
+    # Top-P of the sampled heads restated in fixed point on the GPU's own weights: bit-exact
+    wt = P.unpack_tri(weights[0, heads].cpu().double().numpy(), nb)
+    wt[~np.isfinite(wt)] = np.nan
+    P.check_topp_exact(mb[0, heads], wt, w.p)
+    del weights, wt
     # the prefill's attention starts while its estimator still runs: every
     # output row must equal a separate attention call on the final mask
     o_sep = torch.empty_like(o)
@@ -72,7 +87,9 @@ def test_full_size_sampled_parity(name, cuda_device):
     P.check_tau(tau[0, heads].cpu().double().numpy(), ref)
     P.check_scores(sc, ref)
     n_diff, n_exempt = P.check_mask(mb[0, heads], ref, w.p)
-    print(f"{name}: density {P.density(mb):.4f}, sampled-head mask mismatches {n_diff} (all exempt: {n_exempt})")
+    n_window = int(sum((np.abs(ref["c_excl"][:, z] - w.p) < P.MASK_WINDOW).sum() for z in range(2)))
+    print(f"{name}: density {P.density(mb):.4f}, sampled-head mask mismatches {n_diff} (all exempt: {n_exempt}; "
+          f"blocks in the 1e-4 window: {n_window})")
 
     # attention on sampled (head, query block) rows with the GPU's mask
     blocks = sorted({0, 1, nb // 2, nb - 1} | set(rng.integers(0, nb, 2).tolist()))

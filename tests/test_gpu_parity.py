@@ -3,6 +3,8 @@
 Sizes span several 64-wide score tiles, several 32-bit mask words and a ragged
 tail (nb = 1, 2, 3, 17, 33, 70), GQA 1:1 / 2:1 / 4:1, batch 2.
 """
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -40,19 +42,24 @@ CASES = [
 def test_estimator_parity(w, cuda_device):
     q, k, v, qd, kd, vd = _inputs(w, cuda_device)
     cfg = P.make_cfg(w)
-    mask, sc, tau, _ = P.run_estimate(cfg, qd, kd)
+    ex = {}
+    mask, sc, tau, _ = P.run_estimate(cfg, qd, kd, extras=ex)
     hi, lo = gen.default_bands()
     ref = oracle.estimate(q, k, hi, lo, w.p)
+    P.check_pooled(ex["pooled"], q, k)
     P.check_tau(tau, ref)
     P.check_scores(sc, ref)
     n_diff, n_exempt = P.check_mask(mask, ref, w.p)
-    # Top-P on the GPU's own scores: the oracle's selection must agree exactly
-    # except where fp32 vs fp64 softmax can flip a decision right at p
+    # Top-P on the GPU's own weights, restated in fixed point: bit-exact
+    P.check_topp_exact(mask, ex["weights"], w.p)
+    # the oracle's fp64 Top-P on the GPU's own scores: exact except where the
+    # fp32 weights' rounding can flip a decision right at p
     self_mask, self_cx = P.topp_on_scores(sc, w.p)
     diff = self_mask != mask
     near = (np.abs(self_cx[..., 0, :, :] - w.p) < P.SELF_WINDOW) | (np.abs(self_cx[..., 1, :, :] - w.p) < P.SELF_WINDOW)
     assert not np.any(diff & ~near), f"{np.sum(diff & ~near)} bits differ from Top-P on the GPU scores"
-    print(f"{w.name}: density {P.density(mask):.3f} mismatches {n_diff} (exempt {n_exempt})")
+    print(f"{w.name}: density {P.density(mask):.3f} mismatches {n_diff} (exempt {n_exempt}); "
+          f"oracle Top-P on GPU scores: {int(diff.sum())} bits in the {P.SELF_WINDOW} window")
 
 
 @pytest.mark.parametrize("w", CASES[:4] + CASES[6:7] + CASES[8:], ids=lambda w: w.name)
@@ -80,11 +87,14 @@ def test_short_last_block(w, cuda_device):
     q, k, v, qd, kd, vd = _inputs(w, cuda_device)
     hi, lo = gen.default_bands()
     cfg = P.make_cfg(w)
-    mask, sc, tau, words = P.run_estimate(cfg, qd, kd)
+    ex = {}
+    mask, sc, tau, words = P.run_estimate(cfg, qd, kd, extras=ex)
     ref = oracle.estimate(q, k, hi, lo, w.p)
+    P.check_pooled(ex["pooled"], q, k)  # the short last block divides by its own token count
     P.check_tau(tau, ref)
     P.check_scores(sc, ref)
     P.check_mask(mask, ref, w.p)
+    P.check_topp_exact(mask, ex["weights"], w.p)
     o = P.run_attention(cfg, qd, kd, vd, torch.from_numpy(words.view(np.int32)).to(cuda_device))
     rows = [(b, h, i) for b in range(w.batch) for h in range(w.hq) for i in range(w.nb)]
     P.check_attention_rows(o, q, k, v, mask, rows, w.hq // w.hkv)
@@ -145,9 +155,11 @@ def test_forced_blocks(force, cuda_device):
     q, k, v, qd, kd, vd = _inputs(w, cuda_device)
     hi, lo = gen.default_bands()
     cfg = P.make_cfg(w, force_blocks=force)
-    mask, _, _, words = P.run_estimate(cfg, qd, kd)
+    ex = {}
+    mask, _, _, words = P.run_estimate(cfg, qd, kd, extras=ex)
     ref = oracle.estimate(q, k, hi, lo, w.p, force_sink=bool(force & 1), force_diag=bool(force & 2))
     P.check_mask(mask, ref, w.p)
+    P.check_topp_exact(mask, ex["weights"], w.p, force_sink=bool(force & 1), force_diag=bool(force & 2))
     nb = w.nb
     if force & 1:
         assert mask[..., 0].all()
@@ -254,12 +266,14 @@ def test_topp_ties_and_crowded_bins(kind, cuda_device):
     q, k = _crowded_inputs(kind, nb, seed=71 + len(kind))
     w = gen.small_workload(f"crowd_{kind}", 1, 2, 1, nb * 128, seed=0, p=p)
     cfg = P.make_cfg(w)
-    mask, sc, tau, _ = P.run_estimate(cfg, q.to(cuda_device), k.to(cuda_device))
+    ex = {}
+    mask, sc, tau, _ = P.run_estimate(cfg, q.to(cuda_device), k.to(cuda_device), extras=ex)
     hi, lo = gen.default_bands()
     ref = oracle.estimate(q, k, hi, lo, p)
     P.check_tau(tau, ref)
     P.check_scores(sc, ref)
     P.check_mask(mask, ref, p)
+    P.check_topp_exact(mask, ex["weights"], p)  # the refinement and equal-key paths, bit-exact
     self_mask, self_cx = P.topp_on_scores(sc, p)
     near = (np.abs(self_cx[..., 0, :, :] - p) < P.SELF_WINDOW) | (np.abs(self_cx[..., 1, :, :] - p) < P.SELF_WINDOW)
     assert not np.any((self_mask != mask) & ~near)
@@ -298,6 +312,10 @@ def test_variable_length_batch(cuda_device):
     assert pb.prism_get_last_device_error() == 0
     words = mask.cpu().numpy().view(np.uint32)
     ocpu = o.cpu()
+    # the padded batch's pooled means: each sequence's blocks over its own tokens
+    ex = {}
+    P.run_estimate(cfg, qd, kd, with_scores=False, extras=ex)
+    P.check_pooled(ex["pooled"], q, k, seq_tokens=lens)
     for x, w in enumerate(singles):
         qs, ks, vs = parts[x]
         nbx = w.nb
@@ -420,3 +438,44 @@ def test_softmax_scale_argument(cuda_device):
     o = P.run_attention(cfg, qd, kd, vd, torch.from_numpy(words.view(np.int32)).to(cuda_device))
     rows = [(0, h, i) for h in range(2) for i in range(nb)]
     P.check_attention_rows(o, q, k, v, m, rows, 2, scale=0.05)
+
+
+@pytest.mark.parametrize("base,nb", [(5e5, 6), (1e6, 5)])
+def test_pooled_rope_attenuation_on_gpu(base, nb, cuda_device):
+    """The pooling-attenuation closed form (paper.rainbus.top review, novelty
+    paragraph: a RoPE pair pooled over B positions keeps the fraction
+    lambda_j(B) ~ sinc(B theta_j / 2 pi) of its length) on the kernel's pooled
+    means.  Input: one constant pre-RoPE vector per head, rotated at
+    positions 0..N-1 and rounded to bf16.  Every block's pooled pair j has
+    length |a_j| |sin(B theta_j / 2) / (B sin(theta_j / 2))| (the Dirichlet
+    form; the block's start only rotates it).  bf16 rounding moves each
+    coordinate by <= 2^-9 of the pair length, so the measured ratio is within
+    sqrt(2) 2^-9 of the exact form; fp32 pooling adds < 2^-18.  The
+    normalised sinc is within 6.2e-4 of the exact form (oracle pin)."""
+    d, half, B = 128, 64, 128
+    n = nb * B
+    g = torch.Generator("cpu")
+    g.manual_seed(int(base) % 1000 + nb)
+    a = torch.randn(2, d, generator=g, dtype=torch.float64)  # one vector per head (Q head, KV head)
+    cos, sin = gen.rope_tables(n, d, base)
+    x = gen.apply_rope(a[:, None, :].expand(2, n, d), cos, sin).to(torch.bfloat16)
+    q, k = x[0][None, None].contiguous(), x[1][None, None].contiguous()
+    w = gen.small_workload("sinc_pin", 1, 1, 1, n, seed=0, p=0.9)
+    ex = {}
+    P.run_estimate(P.make_cfg(w), q.to(cuda_device), k.to(cuda_device), with_scores=False, extras=ex)
+    pooled = ex["pooled"]  # [2, nb, 128]: the Q head, then the KV head
+    P.check_pooled(pooled, q, k)
+    theta = np.array(gen.rope_theta(d, base))
+    exact = np.abs(np.sin(B * theta / 2) / (B * np.sin(theta / 2)))
+    sinc = np.abs(np.sinc(B * theta / (2 * np.pi)))  # numpy's sinc is the normalised one
+    bound = math.sqrt(2) * 2.0 ** -9 + 2.0 ** -17
+    for r in range(2):
+        a_len = np.hypot(a[r, :half].numpy(), a[r, half:].numpy())
+        for blk in range(nb):
+            pair_len = np.hypot(pooled[r, blk, :half], pooled[r, blk, half:])
+            lam = pair_len / a_len
+            assert np.all(np.abs(lam - exact) <= bound), (r, blk, np.abs(lam - exact).max())
+            assert np.all(np.abs(lam - sinc) <= bound + 6.2e-4), (r, blk, np.abs(lam - sinc).max())
+            # the dead zone (B theta_j >= 2 pi) is attenuated to < 0.13
+            dead = B * theta >= 2 * np.pi
+            assert np.all(lam[dead] < 0.13 + bound)
