@@ -494,7 +494,7 @@ int prism_estimate(const prism_config* cfg, const void* q, const void* k, uint32
   if (s != PRISM_OK) return s;
   if (!q || !k || !mask) return PRISM_ERR_NULL;
   if (!workspace || workspace_bytes < P.total) return PRISM_ERR_WORKSPACE;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(mask, 16) || !aligned(workspace, 256))
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(mask, 4) || !aligned(workspace, 256))
     return PRISM_ERR_ALIGN;
   if (dbg && ((dbg->scores && !aligned(dbg->scores, 16)) || (dbg->weights && !aligned(dbg->weights, 16)) ||
               (dbg->tau && !aligned(dbg->tau, 4)) || (dbg->pooled && !aligned(dbg->pooled, 16))))
@@ -525,7 +525,7 @@ int prism_prefill(const prism_config* cfg, const void* q, const void* k, const v
   if (!q || !k || !v || !o) return PRISM_ERR_NULL;
   if (!workspace || workspace_bytes < P.total) return PRISM_ERR_WORKSPACE;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
-      !aligned(workspace, 256) || (mask_out && !aligned(mask_out, 16)))
+      !aligned(workspace, 256) || (mask_out && !aligned(mask_out, 4)))
     return PRISM_ERR_ALIGN;
   if ((s = ensure_device()) != PRISM_OK) return s;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
@@ -550,7 +550,7 @@ int prism_estimate_noalloc(const prism_config* cfg, const void* q, const void* k
   if (s != PRISM_OK) return s;
   if (!q || !k || !mask) return PRISM_ERR_NULL;
   if (P.total > kStaticScratchBytes) return PRISM_ERR_SCRATCH_LIMIT;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(mask, 16)) return PRISM_ERR_ALIGN;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(mask, 4)) return PRISM_ERR_ALIGN;
   if ((s = ensure_device()) != PRISM_OK) return s;
   void* scratch = nullptr;
   if ((s = static_scratch(&scratch)) != PRISM_OK) return s;

@@ -17,9 +17,10 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  * - All tensor arguments are DEVICE pointers owned by the caller, contiguous,
- *   16-byte aligned.  The library never allocates device memory, never
- *   synchronises, and enqueues all work on the caller's `stream` (0 = the
- *   legacy default stream).  Calls are asynchronous: a 0 return means the work
+ *   16-byte aligned (the mask: 4-byte aligned, so the rows of any group of
+ *   heads can be addressed inside a larger mask).  The library never
+ *   allocates device memory, never synchronises, and enqueues all work on
+ *   the caller's `stream` (0 = the legacy default stream).  Calls are asynchronous: a 0 return means the work
  *   was enqueued, not that it finished.
  * - Layouts (b = batch, hq / hkv = query / key-value heads, N = seqlen (the
  *   padded length when per-sequence lengths are given), D = head_dim = 128,
@@ -51,7 +52,7 @@ enum {
   PRISM_ERR_NULL = -1,        /* a required pointer is NULL                        */
   PRISM_ERR_SHAPE = -2,       /* batch/heads/seqlen non-positive, hq % hkv != 0,
                                  or sizes overflow                                 */
-  PRISM_ERR_ALIGN = -3,       /* a tensor pointer is not 16-byte aligned           */
+  PRISM_ERR_ALIGN = -3,       /* a tensor pointer is not 16-byte aligned (mask: 4)  */
   PRISM_ERR_BAND = -4,        /* band index out of [0, head_dim), duplicated, or an
                                  empty band                                        */
   PRISM_ERR_P = -5,           /* p is not in (0, 1] (p > 1 is treated as 1), or NaN */

@@ -90,7 +90,8 @@ def topp_fixed_point(weights: np.ndarray, p: float) -> np.ndarray:
     """The GPU's Top-P decision restated on its own weights.
 
     weights [..., nb, nb]: the e_j of each causal row (NaN above the
-    diagonal).  Per row: masses m_j = round-half-even(e_j 2^31) (exact: e_j is
+    diagonal; 0 where the exponential underflowed; the maximum 1 up to one
+    rounding).  Per row: masses m_j = round-half-even(e_j 2^31) (exact: e_j is
     an fp32 value and the product a power-of-two scaling), Z = sum m_j,
     lim = max(floor(p Z), 1) with p the fp32 value the library uses and the
     product formed in fp64; blocks ranked by (-e_j, j); block j kept iff the
@@ -102,7 +103,10 @@ def topp_fixed_point(weights: np.ndarray, p: float) -> np.ndarray:
     for r in range(flat.shape[0]):
         for i in range(nb):
             e = flat[r, i, :i + 1]
-            assert np.all(np.isfinite(e)) and np.all(e > 0) and np.all(e <= 1), "weights must lie in (0, 1]"
+            # the row maximum's weight is 1 up to the rounding of the shifted
+            # argument; the hardware exponential flushes results below 2^-126 to 0
+            assert np.all(np.isfinite(e)) and np.all(e >= 0) and np.all(e < 2) and abs(e.max() - 1.0) < 1e-6, \
+                "weights must lie in [0, 2) with the row maximum at 1"
             m = np.rint(e * 2.0 ** 31).astype(np.int64)
             z = int(m.sum())
             lim = max(int(np.float64(pf) * np.float64(z)), 1)

@@ -118,7 +118,7 @@ def test_null_pointers_workspace_and_alignment_rejected():
     assert pb.lib.prism_sparse_attn(cfg.ptr(), a, a, a, a, None, None) == -1
     assert pb.lib.prism_sparse_attn(cfg.ptr(), a, a, a + 2, a, a, None) == -3
     assert pb.lib.prism_prefill(cfg.ptr(), a, a, a, None, a, None, ws, None) == -7
-    assert pb.lib.prism_prefill(cfg.ptr(), a, a, a, a + 4, a, a, ws, None) == -3
+    assert pb.lib.prism_prefill(cfg.ptr(), a, a, a, a + 2, a, a, ws, None) == -3  # masks: 4-byte words
 
 
 def test_python_binding_rejects_host_tensors():

@@ -448,10 +448,11 @@ def test_pooled_rope_attenuation_on_gpu(base, nb, cuda_device):
     means.  Input: one constant pre-RoPE vector per head, rotated at
     positions 0..N-1 and rounded to bf16.  Every block's pooled pair j has
     length |a_j| |sin(B theta_j / 2) / (B sin(theta_j / 2))| (the Dirichlet
-    form; the block's start only rotates it).  bf16 rounding moves each
-    coordinate by <= 2^-9 of the pair length, so the measured ratio is within
-    sqrt(2) 2^-9 of the exact form; fp32 pooling adds < 2^-18.  The
-    normalised sinc is within 6.2e-4 of the exact form (oracle pin)."""
+    form; the block's start only rotates it).  bf16 rounding (an 8-bit
+    significand: unit roundoff 2^-8) moves each coordinate by <= 2^-8 of the
+    pair length, so the measured ratio is within sqrt(2) 2^-8 of the exact
+    form; fp32 pooling adds < 2^-18.  The normalised sinc is within 6.2e-4 of
+    the exact form (oracle pin)."""
     d, half, B = 128, 64, 128
     n = nb * B
     g = torch.Generator("cpu")
@@ -468,7 +469,7 @@ def test_pooled_rope_attenuation_on_gpu(base, nb, cuda_device):
     theta = np.array(gen.rope_theta(d, base))
     exact = np.abs(np.sin(B * theta / 2) / (B * np.sin(theta / 2)))
     sinc = np.abs(np.sinc(B * theta / (2 * np.pi)))  # numpy's sinc is the normalised one
-    bound = math.sqrt(2) * 2.0 ** -9 + 2.0 ** -17
+    bound = math.sqrt(2) * 2.0 ** -8 + 2.0 ** -17
     for r in range(2):
         a_len = np.hypot(a[r, :half].numpy(), a[r, half:].numpy())
         for blk in range(nb):
@@ -476,6 +477,8 @@ def test_pooled_rope_attenuation_on_gpu(base, nb, cuda_device):
             lam = pair_len / a_len
             assert np.all(np.abs(lam - exact) <= bound), (r, blk, np.abs(lam - exact).max())
             assert np.all(np.abs(lam - sinc) <= bound + 6.2e-4), (r, blk, np.abs(lam - sinc).max())
-            # the dead zone (B theta_j >= 2 pi) is attenuated to < 0.13
+            # the dead zone (B theta_j >= 2 pi) stays under the first side-lobe
+            # peak of |sinc| (0.2172...); the slow pairs pass almost unattenuated
             dead = B * theta >= 2 * np.pi
-            assert np.all(lam[dead] < 0.13 + bound)
+            assert np.all(lam[dead] < 0.2173 + 6.2e-4 + bound)
+            assert np.all(lam[32:] > 0.99 - bound)
