@@ -269,13 +269,16 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   }
   if (threadIdx.x == 0) {
     // launched while the estimator still runs: wait (bounded) until the
-    // estimator has published the mask rows of both tiles
+    // estimator has counted every mask row of the segments of both tiles
     int ok = 1;
     if (ready) {
       const int nseg = (nb + ready_rows - 1) / ready_rows;
       for (int x = 0; x < 2; ++x)
-        if (ok && tiles[x].valid)
-          ok = flag_wait_ns(&ready[(size_t)tiles[x].bh * nseg + tiles[x].i / ready_rows], kWaitLimitNs) ? 1 : 0;
+        if (ok && tiles[x].valid) {
+          const int sg = tiles[x].i / ready_rows;
+          const uint32_t rows = (uint32_t)min(ready_rows, nb - sg * ready_rows);
+          ok = count_wait_ns(&ready[(size_t)tiles[x].bh * nseg + sg], rows, kWaitLimitNs) ? 1 : 0;
+        }
     }
     s_masks_ok = ok;
   }

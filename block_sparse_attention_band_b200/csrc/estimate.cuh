@@ -58,7 +58,8 @@ constexpr int kMaxPoolStages = 6;      // TMA ring depth (32 KB stages)
 constexpr int kPoolN = 16;             // N of a pooling product: block b sums into TMEM columns [16 b, 16 b + 16)
 constexpr int kScoreRows = 128;       // query blocks (of one head) per score item = MMA M
 constexpr int kScorePartBlocks = 512;  // key blocks per score item: longer rows are split into parts
-constexpr int kToppRows = 16;         // query blocks (of one head) per Top-P item
+constexpr int kScorePartFine = 128;    // the same for the last groups' items (spread over every SM)
+constexpr int kToppRows = 16;         // mask rows per ready counter (what the attention of a prefill waits on)
 constexpr uint32_t kOpChunk = 128 * 64 * 2;  // one 64-dim x 128-row bf16 operand chunk (SW128)
 constexpr int kTerms = 3;             // bf16 terms per pooled value
 // product operands: A (3 terms x dp/64 chunks of 128 rows) once, B one term at
@@ -110,24 +111,23 @@ struct EstParams {
   uint32_t* mask;
   float* dbg_tau;
   float* dbg_pooled;   // optional: block means [q_rows + kv_rows, nb, 128], all dims
-  float* rmax;     // [q_rows, nb, rparts, 2] scaled band logits' row maxima over the key blocks j <= i
-                   // of each part
-  uint32_t* ready;  // [q_rows, ceil(nb / kToppRows)] mask rows of a Top-P item written
+  uint32_t* ready;  // [q_rows, ceil(nb / kToppRows)] mask rows written, per kToppRows-row segment
+  uint32_t* rmax;   // [q_rows, nb, 2] the scaled band logits' row maxima over j <= i, order-preserving
+                    // encoding (max_enc), combined over the score parts with atomicMax from 0
   uint32_t* sync;  // [0] stream queue head, [1] Top-P queue head, [2 + g] pool items done,
                    // [2 + n_groups + g] group ready,
                    // [2 + 2 n_groups + bh * nchunk + c] parts of score chunk c of (batch, Q head) bh written
   int hq, hkv, G, n, nb, W, q_rows, n_groups;  // n: tokens per head (the last block may be short)
   int pool_items;      // per group
-  int score_items;     // per group
+  int score_items;     // per group (kScorePartBlocks parts)
   int score_span;      // score items per head: (row chunk, key-block part) pairs
-  int rparts;          // key-block parts of the longest row chunk
-  int topp_items;      // per group
+  int score_items_fine, score_span_fine;  // the same with kScorePartFine parts (the last kScoreLag groups)
+  int topp_rows;       // Top-P queue entries per group: nchunk x G x kScoreRows (rows past nb skipped)
   int pool_item_span;  // pool items per head row
-  // Top-P warps of each lane: how many take rows, bytes of shared memory
-  // each, and whether a warp holds one logit row (single) or two (the next
-  // one streams in while the current one is ranked)
-  int lane_warps, lane_stride, lane_single;
-  int team_warps, team_stride, team_single;
+  // Top-P warps of each lane: how many take rows and bytes of shared memory
+  // each (topp_scratch)
+  int lane_warps, lane_stride;
+  int team_warps, team_stride;
   int lane_off;      // byte offset of the Top-P lane's shared memory
   int stream_bytes;  // dynamic shared memory of the stream lane (pool ring, score operands)
   int pool_stages;   // TMA ring depth (<= kMaxPoolStages)
@@ -153,15 +153,21 @@ __device__ __forceinline__ float* score_tile(const EstParams& P, int bh, int cr,
 }
 
 // Score items: row chunk c (kScoreRows query blocks) against the key blocks
-// j <= its last row, in parts of kScorePartBlocks key blocks.
-__host__ __device__ __forceinline__ int score_parts(int chunk) {
-  return (chunk * kScoreRows + kScoreRows + kScorePartBlocks - 1) / kScorePartBlocks;
+// j <= its last row, in parts of `pb` key blocks: kScorePartBlocks, or
+// kScorePartFine for the groups scored last, whose items then spread over
+// every SM instead of ending the launch on a few long ones.
+__host__ __device__ __forceinline__ int score_parts(int chunk, int pb) {
+  return (chunk * kScoreRows + kScoreRows + pb - 1) / pb;
+}
+constexpr int kScoreLag = 2;  // scoring of group g follows pooling of group g + kScoreLag
+__device__ __forceinline__ int score_part_blocks(const EstParams& P, int g) {
+  return g >= P.n_groups - min(kScoreLag, P.n_groups) ? kScorePartFine : kScorePartBlocks;
 }
 // Item z of one head (longest rows first) -> (row chunk, part).
-__device__ __forceinline__ void score_part_of(const EstParams& P, int z, int& chunk, int& part) {
+__device__ __forceinline__ void score_part_of(const EstParams& P, int z, int pb, int& chunk, int& part) {
   const int nchunk = (P.nb + kScoreRows - 1) / kScoreRows;
   for (chunk = nchunk - 1; chunk > 0; --chunk) {
-    const int np = score_parts(chunk);
+    const int np = score_parts(chunk, pb);
     if (z < np) break;
     z -= np;
   }
@@ -185,6 +191,15 @@ __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
 __device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// An order-preserving map of floats to unsigned words (larger float, larger
+// word; 0 lies below every float), so maxima combine with integer atomicMax.
+__device__ __forceinline__ uint32_t max_enc(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float max_dec(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
 
 // ---------------------------------------------------------------------------
 // static shared memory of the kernel
@@ -195,7 +210,6 @@ struct PoolSmem {
   // swizzle does not matter)
   __align__(1024) uint32_t ones[16 * 32];
   union {                                   // pool and score items never overlap in a CTA
-    float rmax[2][2][128];                  // score item: row maxima per column half and band
     float wred[16][16];                     // temperatures: per-warp partial sums (kTauBatch slots x 3)
     float bpart[kPoolTilesPerItem][4][3];  // pool item: per block and read-out warp: hi, lo, all
   };
@@ -321,15 +335,14 @@ struct PoolState {  // per-role counters of ring stages and items, carried acros
 };
 
 // Stream queue order, with PI / SI pool / score items per group g of n and a
-// lag of two groups:
+// lag of two groups (the last two groups' score items, SF each, have finer
+// parts):
 //   pool(0) pool(1) | pool(2) score(0) | pool(3) score(1) | ... | pool(n-1) score(n-3) | score(n-2) score(n-1)
 // so scoring of group g overlaps pooling of group g + 2, by which time the
-// pooling of g has ended and the score items do not wait.  The Top-P queue
-// holds topp(0) | topp(1) | ... | topp(n-1).  Returns the item kind (0 pool,
-// 1 score, 2 Top-P, -1 past the end) and sets (g, y), y the index within the
-// group's items of that kind.
-enum : int { kItemPool = 0, kItemScore = 1, kItemTopp = 2, kItemNone = -1 };
-constexpr int kScoreLag = 2;
+// pooling of g has ended and the score items do not wait.  Returns the item
+// kind (0 pool, 1 score, -1 past the end) and sets (g, y), y the index within
+// the group's items of that kind.
+enum : int { kItemPool = 0, kItemScore = 1, kItemNone = -1 };
 __device__ __forceinline__ int decode_stream(const EstParams& P, int x, int& g, int& y) {
   const int n = P.n_groups, PI = P.pool_items, SI = P.score_items;
   const int lag = min(kScoreLag, n), M = n - lag, L = PI + SI;
@@ -351,21 +364,15 @@ __device__ __forceinline__ int decode_stream(const EstParams& P, int x, int& g, 
     return kItemScore;
   }
   x -= M * L;
-  if (x < lag * SI) {
-    const int q = x / SI;
+  const int SF = P.score_items_fine;  // the last lag groups: finer parts
+  if (x < lag * SF) {
+    const int q = x / SF;
     g = M + q;
-    y = x - q * SI;
+    y = x - q * SF;
     return kItemScore;
   }
   return kItemNone;
 }
-__device__ __forceinline__ int decode_topp(const EstParams& P, int x, int& g, int& y) {
-  if (x >= P.n_groups * P.topp_items) return kItemNone;
-  g = x / P.topp_items;
-  y = x - g * P.topp_items;
-  return kItemTopp;
-}
-
 // The tiles of pool item (g, y): tensor map ([heads, n, 128]), head, first
 // token, tile count.
 struct PoolCoords {
@@ -394,8 +401,11 @@ __device__ __forceinline__ void pool_stream(const PoolCoords& c, int t0, int t1,
       mbar_wait(smem_u32(&sm.bars_free[s]), (st.prod / (uint32_t)stages - 1u) & 1u);
     const uint32_t dst = ring0 + s * kTileBytes, bar = smem_u32(&sm.bars[s]);
     mbar_arrive_expect_tx(bar, kTileBytes);
-    tma_load_3d(dst, c.map, 0, c.tok0 + tt * 128, c.head, bar);
-    tma_load_3d(dst + kTileBytes / 2, c.map, 64, c.tok0 + tt * 128, c.head, bar);
+    // read once: first out of L2, so the score tiles the Top-P rows read
+    // back stay resident
+    const uint64_t pol = l2_policy_evict_first();
+    tma_load_3d_hint(dst, c.map, 0, c.tok0 + tt * 128, c.head, bar, pol);
+    tma_load_3d_hint(dst + kTileBytes / 2, c.map, 64, c.tok0 + tt * 128, c.head, bar, pol);
   }
 }
 
@@ -539,8 +549,7 @@ __device__ __forceinline__ void pool_item(const EstParams& P, const CUtensorMap*
 // ---------------------------------------------------------------------------
 // Shared-memory scratch of one Top-P warp.
 struct ToppScratch {
-  uint32_t* d;            // [n] the row's logits, replaced by the rank keys d_j (below)
-  uint32_t* memw;         // [ceil(n / 32)] members of the crossing bin, one bit per block
+  uint32_t* d;            // [n] the row's rank keys d_j (below)
   unsigned long long* h;  // [256] bin masses; then the member records of the exact step
 };
 
@@ -579,23 +588,6 @@ __device__ __forceinline__ int warp_excl_scan(int c, int lane, int& total) {
 __device__ __forceinline__ uint4 member_record(const ToppScratch& S, uint32_t j) {
   const uint32_t d = S.d[j];
   return make_uint4(d, j, fixmass(key_value(d)), 0u);
-}
-
-// Writes the records of the (at most 32) blocks flagged in S.memw[0 .. nw) to
-// rec[0 .. cnt), in block order.
-__device__ __forceinline__ void list_flagged(const ToppScratch& S, int nw, uint4* rec, int lane) {
-  int base = 0;
-  for (int w0 = 0; w0 < nw; w0 += 32) {
-    uint32_t wv = w0 + lane < nw ? S.memw[w0 + lane] : 0u;
-    int tot;
-    int pos = base + warp_excl_scan(__popc(wv), lane, tot);
-    while (wv) {
-      const int b = __ffs(wv) - 1;
-      wv &= wv - 1u;
-      rec[pos++] = member_record(S, (uint32_t)((w0 + lane) * 32 + b));
-    }
-    base += tot;
-  }
 }
 
 // Writes the records of the (at most 32) blocks whose key lies in [rlo, rhi]
@@ -647,24 +639,25 @@ __device__ __forceinline__ int topp_exact32(const uint4* rec, int cnt, unsigned 
 }
 
 // A bin's 64-bit mass is kept as two 32-bit sums, of the low 16 bits and of
-// the high 16 bits of each added value, so a bin mass is hi * 2^16 + lo.
-// Neither sum can wrap (at most 2^14 values of < 2^16 each), so the adds need
-// no carry and no result: fire-and-forget shared-memory reductions, exact and
-// independent of the order of the adds.
-// (No "memory" clobber: the bins are read only after a __syncwarp, and
-// leaving the compiler free to move other loads across the reductions keeps
-// several blocks' arithmetic in flight.)
-__device__ __forceinline__ void bin_add(uint32_t* lo, uint32_t* hi, int b, uint32_t x) {
+// the high 16 bits of each added value, so a bin mass is hi * 2^16 + lo
+// (kTopPBins words of each, low sums first).  Neither sum can wrap (at most
+// 2^14 values of < 2^16 each), so the adds need no carry and no result:
+// fire-and-forget 32-bit shared-memory reductions (faster here than 64-bit
+// ones), exact and independent of the order of the adds.  (No "memory"
+// clobber: the bins are read only after a __syncwarp, and leaving the
+// compiler free to move other loads across the reductions keeps several
+// blocks' arithmetic in flight.)
+__device__ __forceinline__ void bin_add(unsigned long long* bins, int b, uint32_t x) {
+  uint32_t* lo = reinterpret_cast<uint32_t*>(bins);
   asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(smem_u32(lo + b)), "r"(x & 0xFFFFu));
-  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(smem_u32(hi + b)), "r"(x >> 16));
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(smem_u32(lo + kTopPBins + b)), "r"(x >> 16));
 }
-__device__ __forceinline__ unsigned long long bin_mass(const uint32_t* lo, const uint32_t* hi, int b) {
-  return ((unsigned long long)hi[b] << 16) + lo[b];
+__device__ __forceinline__ unsigned long long bin_mass(const unsigned long long* bins, int b) {
+  const uint32_t* lo = reinterpret_cast<const uint32_t*>(bins);
+  return ((unsigned long long)lo[kTopPBins + b] << 16) + lo[b];
 }
 
-// Softmax (step 5) + Top-P (step 6) of one band row of n scaled logits, held
-// in shared memory at S.d (as floats); ORs the kept blocks into bits[].  rmax
-// is the row's maximum.
+// Softmax (step 5) + Top-P (step 6) of one band row of n scaled logits:
 //
 // e_j = 2^((L_j - max) log2 e); blocks ranked by (-e_j, j) == (d_j, j) with
 // the exact order-reversing key d_j.  Radix selection on the keys: bins of 16
@@ -675,135 +668,155 @@ __device__ __forceinline__ unsigned long long bin_mass(const uint32_t* lo, const
 // A member x of the crossing bin is kept iff the mass ranked strictly ahead
 // of it is below the target p Z (the top block always): with <= 32 members
 // every member sums the masses of the members ahead of it directly, else the
-// bin is refined on the lower key bits the same way.
+// bin is refined on the lower key bits the same way.  The histogram pass of
+// a Top-P row leaves the keys at S.d and the bin masses in S.h; topp_select
+// does the rest.
 constexpr size_t kTilePair = 2 * 128 * 128;  // floats per score tile pair (both bands)
 
-__device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const ToppScratch& S, uint32_t* bits,
-                                              float* dbg, float* dbgw, int lane) {
-  const unsigned lt = (1u << lane) - 1u;
-  const float* row = reinterpret_cast<const float*>(S.d);
-  if (dbg)
-    for (int j = lane; j < n; j += 32) dbg[j] = row[j];
+// Zeroes the warp's 2 KB of bins (16-byte stores).
+__device__ __forceinline__ void topp_zero_bins(const ToppScratch& S, int lane) {
+  uint4* h = reinterpret_cast<uint4*>(S.h);
+  for (int q = lane; q < 2 * kTopPBins / 4; q += 32) h[q] = make_uint4(0u, 0u, 0u, 0u);
+  __syncwarp();
+}
+
+// e_j, rank key and exact bin mass of one block (the key stored at S.d[j]).
+__device__ __forceinline__ void topp_hist1(const ToppScratch& S, int j, float x, float m) {
+  const float e = fast_exp2(fmaf(x, kLog2e, -m));
+  const uint32_t d = rank_key(e);
+  S.d[j] = d;
+  bin_add(S.h, (int)min(d >> 19, (uint32_t)(kTopPBins - 1)), fixmass(e));
+}
+
+// Every causal block of a row (p >= 1).
+__device__ __forceinline__ void topp_keep_all(int n, uint32_t* bits, int lane) {
   const int nw = (n + 31) >> 5;
-  if (p >= 1.0f) {  // every causal block is kept
-    for (int w = lane; w < nw; w += 32) {
-      const int lo = w * 32;
-      bits[w] |= lo + 32 <= n ? 0xffffffffu : ((1u << (n - lo)) - 1u);
-    }
-    __syncwarp();
-    return;
-  }
-  const float m = rmax * kLog2e;
-  uint32_t* hlo = reinterpret_cast<uint32_t*>(S.h);
-  uint32_t* hhi = hlo + kTopPBins;
-  uint4* rec = reinterpret_cast<uint4*>(S.h);  // member records, over the bins once they are read
-  // the 2 KB of bins zeroed with 16-byte stores
-  for (int q = lane; q < 2 * kTopPBins / 4; q += 32) reinterpret_cast<uint4*>(hlo)[q] = make_uint4(0u, 0u, 0u, 0u);
-  __syncwarp();
-  // e_j, keys (in place of the logits), exact bin masses; only the
-  // ceil(n / 32) slots the row has are visited
-  const int ns = nw;
-  auto hist1 = [&](int j, float x) {
-    const float e = fast_exp2(fmaf(x, kLog2e, -m));
-    const uint32_t d = rank_key(e);
-    S.d[j] = d;
-    bin_add(hlo, hhi, (int)min(d >> 19, (uint32_t)(kTopPBins - 1)), fixmass(e));
-  };
-  int u = 0;
-  for (; u + 4 <= (n >> 5); u += 4) {  // four whole slots: loads first, then their arithmetic
-    float x[4];
-#pragma unroll
-    for (int v = 0; v < 4; ++v) x[v] = row[(u + v) * 32 + lane];
-#pragma unroll
-    for (int v = 0; v < 4; ++v) hist1((u + v) * 32 + lane, x[v]);
-  }
-  for (; u < ns; ++u) {
-    const int j = u * 32 + lane;
-    if (j < n) hist1(j, row[j]);
+  for (int w = lane; w < nw; w += 32) {
+    const int lo = w * 32;
+    bits[w] |= lo + 32 <= n ? 0xffffffffu : ((1u << (n - lo)) - 1u);
   }
   __syncwarp();
-  // lane l's 8 bins: its total (the two 32-bit half sums cannot wrap)
-  unsigned long long tot;
-  {
-    const uint4 l0 = reinterpret_cast<const uint4*>(hlo)[2 * lane], l1 = reinterpret_cast<const uint4*>(hlo)[2 * lane + 1];
-    const uint4 h0 = reinterpret_cast<const uint4*>(hhi)[2 * lane], h1 = reinterpret_cast<const uint4*>(hhi)[2 * lane + 1];
-    const uint32_t sl = (l0.x + l0.y) + (l0.z + l0.w) + (l1.x + l1.y) + (l1.z + l1.w);
-    const uint32_t sh = (h0.x + h0.y) + (h0.z + h0.w) + (h1.x + h1.y) + (h1.z + h1.w);
-    tot = ((unsigned long long)sh << 16) + sl;
-  }
-  const unsigned long long incl = warp_scan_u64(tot, lane);
-  const unsigned long long Z = __shfl_sync(0xffffffffu, incl, 31);
-  const unsigned long long target = (unsigned long long)((double)p * (double)Z);
-  const unsigned long long lim = target > 0ull ? target : 1ull;
-  // crossing bin: the first whose cumulative mass reaches lim (it holds mass;
-  // lim <= Z, so it exists).  Its lane is found by a ballot over the lanes'
-  // inclusive sums, then lanes 0-7 scan that lane's 8 bins.
+}
+
+// The crossing bin of a band row from its bin masses (after a histogram
+// pass): lim = max(floor(p Z), 1) and the first bin whose cumulative mass
+// reaches it, with the mass ranked before that bin.  Each lane sums the two
+// halves of its 8 bins, the two sums are scanned across the warp side by
+// side, and each lane then walks its own 8 bins, so only the lane holding the
+// crossing bin finds it.
+struct ToppCross {
+  unsigned long long target, lim, base;
   int xb;
-  unsigned long long base;
-  {
-    const int L = __ffs(__ballot_sync(0xffffffffu, incl >= lim)) - 1;
-    const unsigned long long before = __shfl_sync(0xffffffffu, incl - tot, L);
-    const unsigned long long hb = lane < 8 ? bin_mass(hlo, hhi, 8 * L + lane) : 0ull;
-    unsigned long long pre = hb;
+};
+__device__ __forceinline__ ToppCross topp_cross_bin(float p, const ToppScratch& S, int lane) {
+  const uint32_t* hlo = reinterpret_cast<const uint32_t*>(S.h);
+  const uint32_t* hhi = hlo + kTopPBins;
+  const uint4 l0 = reinterpret_cast<const uint4*>(hlo)[2 * lane], l1 = reinterpret_cast<const uint4*>(hlo)[2 * lane + 1];
+  const uint4 h0 = reinterpret_cast<const uint4*>(hhi)[2 * lane], h1 = reinterpret_cast<const uint4*>(hhi)[2 * lane + 1];
+  const uint32_t bl[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+  const uint32_t bh[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+  // the warp's sums of the low halves (< 2^30) and of the high halves fit 32 bits
+  const uint32_t sl = (bl[0] + bl[1]) + (bl[2] + bl[3]) + (bl[4] + bl[5]) + (bl[6] + bl[7]);
+  const uint32_t sh = (bh[0] + bh[1]) + (bh[2] + bh[3]) + (bh[4] + bh[5]) + (bh[6] + bh[7]);
+  uint32_t il = sl, ih = sh;
 #pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-      const unsigned long long v = __shfl_up_sync(0xffffffffu, pre, o);
-      if (lane >= o) pre += v;
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t ul = __shfl_up_sync(0xffffffffu, il, o), uh = __shfl_up_sync(0xffffffffu, ih, o);
+    if (lane >= o) {
+      il += ul;
+      ih += uh;
     }
-    const int ub = __ffs(__ballot_sync(0xffffffffu, lane < 8 && before + pre >= lim)) - 1;
-    xb = 8 * L + ub;
-    base = before + __shfl_sync(0xffffffffu, pre - hb, ub);
   }
-  // one pass over the keys: blocks of earlier bins (key below the crossing
-  // bin's first key) are kept, the crossing bin's members flagged; lane u
-  // collects the words of slot u of each batch of 32 slots
-  const uint32_t key_lo = (uint32_t)xb << 19;
-  const uint32_t key_hi = xb == kTopPBins - 1 ? 0xffffffffu : ((uint32_t)(xb + 1) << 19);
+  const unsigned long long Z = ((unsigned long long)__shfl_sync(0xffffffffu, ih, 31) << 16) +
+                               __shfl_sync(0xffffffffu, il, 31);
+  ToppCross C;
+  C.target = (unsigned long long)((double)p * (double)Z);
+  C.lim = C.target > 0ull ? C.target : 1ull;
+  unsigned long long run = (((unsigned long long)(ih - sh)) << 16) + (il - sl);  // mass before this lane's bins
+  int q_hit = -1;
+  unsigned long long b_hit = 0ull;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const unsigned long long m = ((unsigned long long)bh[q] << 16) + bl[q];
+    if (q_hit < 0 && run + m >= C.lim) {
+      q_hit = q;
+      b_hit = run;
+    }
+    run += m;
+  }
+  const int F = __ffs(__ballot_sync(0xffffffffu, q_hit >= 0)) - 1;  // lim <= Z: some lane holds it
+  C.xb = 8 * F + __shfl_sync(0xffffffffu, q_hit, F);
+  C.base = __shfl_sync(0xffffffffu, b_hit, F);
+  return C;
+}
+
+__device__ __forceinline__ void topp_refine(int n, const ToppScratch& S, const ToppCross& C, uint32_t* bits,
+                                            float* dbgw, int lane);
+
+// The selection of step (6) on a band row whose keys are at S.d and whose
+// bin masses are in S.h (after a histogram pass); ORs the kept blocks into
+// bits[].  One pass over the keys keeps the blocks of earlier bins (lane u
+// collects the word of slot u of each batch of 32 slots) and lists the
+// crossing bin's members (the first 32, in block order) by ballot; with <= 32
+// members every member sums the masses of the members ranked ahead of it,
+// else the bin is refined.
+__device__ __forceinline__ void topp_select(int n, float p, const ToppScratch& S, uint32_t* bits, float* dbgw,
+                                            int lane) {
+  const unsigned lt = (1u << lane) - 1u;
+  const int ns = (n + 31) >> 5;
+  uint4* rec = reinterpret_cast<uint4*>(S.h);  // member records, over the bins once they are read
+  const ToppCross C = topp_cross_bin(p, S, lane);
+  __syncwarp();  // the bins are read before member records overwrite them
+  const uint32_t key_lo = (uint32_t)C.xb << 19;
+  const uint32_t key_hi = C.xb == kTopPBins - 1 ? 0xffffffffu : ((uint32_t)(C.xb + 1) << 19);
   int cnt = 0;
   for (int u0 = 0; u0 < ns; u0 += 32) {
     const int u1 = min(u0 + 32, ns);
-    uint32_t myw = 0u, mym = 0u;
-    auto sel = [&](int uu, uint32_t d) {
-      const unsigned kb = __ballot_sync(0xffffffffu, d < key_lo);
-      const unsigned mb = __ballot_sync(0xffffffffu, d < key_hi) & ~kb;
-      if (lane == uu - u0) {
-        myw = kb;
-        mym = mb;
-      }
-    };
-    const int uf = min(u1, n >> 5);  // whole slots
-    int uu = u0;
-#pragma unroll 8
-    for (; uu < uf; ++uu) sel(uu, S.d[uu * 32 + lane]);
-    for (; uu < u1; ++uu) {
+    uint32_t myw = 0u;
+#pragma unroll 4
+    for (int uu = u0; uu < u1; ++uu) {
       const int j = uu * 32 + lane;
-      sel(uu, j < n ? S.d[j] : 0xffffffffu);
+      const uint32_t d = j < n ? S.d[j] : 0xffffffffu;
+      const unsigned kb = __ballot_sync(0xffffffffu, d < key_lo);
+      const bool in = d >= key_lo && d < key_hi;
+      const unsigned mk = __ballot_sync(0xffffffffu, in);
+      const int pos = cnt + __popc(mk & lt);
+      if (in && pos < 32) rec[pos] = make_uint4(d, (uint32_t)j, fixmass(key_value(d)), 0u);
+      cnt += __popc(mk);
+      if (lane == uu - u0) myw = kb;
     }
-    if (lane < u1 - u0) {
-      bits[u0 + lane] |= myw;
-      S.memw[u0 + lane] = mym;
-    }
-    cnt += __reduce_add_sync(0xffffffffu, (unsigned)__popc(mym));
+    if (lane < u1 - u0) bits[u0 + lane] |= myw;
   }
   __syncwarp();
   if (cnt <= 32) {
-    // member x is kept iff base + (mass of the members ranked ahead of it) <
-    // lim; the members' records are read back with broadcast loads
-    list_flagged(S, ns, rec, lane);
-    __syncwarp();
     const uint4 me = lane < cnt ? rec[lane] : make_uint4(0xffffffffu, 0x7fffffffu, 0u, 0u);
-    unsigned long long ahead = base;
+    unsigned long long ahead = C.base;
 #pragma unroll 4
     for (int y = 0; y < cnt; ++y) {
       const uint4 o = rec[y];
       if (o.x < me.x || (o.x == me.x && o.y < me.y)) ahead += o.z;
     }
-    if (lane < cnt && ahead < lim) atomicOr(&bits[me.y >> 5], 1u << (me.y & 31));
+    if (lane < cnt && ahead < C.lim) atomicOr(&bits[me.y >> 5], 1u << (me.y & 31));
     if (dbgw)
       for (int j = lane; j < n; j += 32) dbgw[j] = key_value(S.d[j]);
     __syncwarp();
     return;
   }
+  topp_refine(n, S, C, bits, dbgw, lane);
+}
+
+// A crossing bin with more than 32 members: refine it on lower key bits (the
+// keys at S.d), then keep every block ranked at or ahead of the crossing.
+__device__ __forceinline__ void topp_refine(int n, const ToppScratch& S, const ToppCross& C, uint32_t* bits,
+                                            float* dbgw, int lane) {
+  const unsigned lt = (1u << lane) - 1u;
+  uint4* rec = reinterpret_cast<uint4*>(S.h);
+  const unsigned long long target = C.target, lim = C.lim;
+  unsigned long long base = C.base;
+  const int xb = C.xb;
+  const uint32_t key_lo = (uint32_t)xb << 19;
+  const uint32_t key_hi = xb == kTopPBins - 1 ? 0xffffffffu : ((uint32_t)(xb + 1) << 19);
+  (void)lim;
   // refine on lower key bits, 8-bit digits: a regular bin spans 2^19 keys
   // (digits at shifts 11, 3, 0), the catch-all bin up to 2^30 (22, 14, 6, 0).
   // The members are the row's keys in [rlo, rhi], found by scanning the keys.
@@ -813,21 +826,18 @@ __device__ __forceinline__ void topp_band_row(float rmax, int n, float p, const 
   for (int level = 0;; ++level) {
     const int sh = wide ? (level == 0 ? 22 : level == 1 ? 14 : level == 2 ? 6 : 0)
                         : (level == 0 ? 11 : level == 1 ? 3 : 0);
-    for (int b = lane; b < kTopPBins; b += 32) {
-      hlo[b] = 0u;
-      hhi[b] = 0u;
-    }
+    for (int b = lane; b < kTopPBins; b += 32) S.h[b] = 0ull;  // both halves: 2 x 256 words
     __syncwarp();
     for (int j = lane; j < n; j += 32) {
       const uint32_t d = S.d[j];
       if (d >= rlo && d <= rhi)
-        bin_add(hlo, hhi, (int)min((d - rlo) >> sh, (uint32_t)(kTopPBins - 1)), fixmass(key_value(d)));
+        bin_add(S.h, (int)min((d - rlo) >> sh, (uint32_t)(kTopPBins - 1)), fixmass(key_value(d)));
     }
     __syncwarp();
     unsigned long long h2[8], t2 = 0ull;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      h2[q] = bin_mass(hlo, hhi, lane * 8 + q);
+      h2[q] = bin_mass(S.h, lane * 8 + q);
       t2 += h2[q];
     }
     const unsigned long long inc2 = warp_scan_u64(t2, lane);
@@ -979,7 +989,8 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
   const int bi = g / P.hkv, kv = g - bi * P.hkv;
   const int nchunk = (P.nb + kScoreRows - 1) / kScoreRows;
   int chunk, part;
-  score_part_of(P, y / P.G, chunk, part);  // longest rows first
+  const int pb = score_part_blocks(P, g);
+  score_part_of(P, y / P.G, pb, chunk, part);  // longest rows first
   const int bh = bi * P.hq + kv * P.G + y % P.G;
   const int i0 = chunk * kScoreRows;
   const int nbb = seq_blocks(P, bi);
@@ -987,7 +998,7 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
   const uint32_t nch = (uint32_t)P.bl.dp / 64;
   const int ncolw = score_cols(P.bl.dp);  // N: key blocks per column chunk
   // this part's key blocks [j0, j1): column chunks c0 .. c0 + ncol - 1
-  const int j0 = part * kScorePartBlocks, j1 = min(j0 + kScorePartBlocks, max_i + 1);
+  const int j0 = part * pb, j1 = min(j0 + pb, max_i + 1);
   const int c0 = j0 / ncolw;
   const int ncol = (j1 - 1) / ncolw + 1 - c0;
   const int units = 3 * ncol;
@@ -1064,11 +1075,11 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
     // warp w reads TMEM lane quarter w % 4 in the 16 x 256-bit shape, 32
     // columns at a time: four threads share a row, each holding two adjacent
     // key blocks, so every store instruction writes eight whole 32-byte
-    // sectors of the score tiles.  The row maxima over j <= i are kept too.
+    // sectors of the score tiles.
     const float sc_hi = P.tau[bh * 4 + 2], sc_lo = P.tau[bh * 4 + 3];
     const int q4 = warp & 3;
     const int gr = lane >> 2, cq = (lane & 3) * 2;
-    float mx[2][2][2];  // [lane half][row of the pair][band]
+    float mx[2][2][2];  // [lane half][row of the pair][band]: row maxima over this part's j <= i
 #pragma unroll
     for (int a = 0; a < 8; ++a) (&mx[0][0][0])[a] = -INFINITY;
     for (int c = 0; c < ncol; ++c) {
@@ -1091,11 +1102,11 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
               const int rl = q4 * 32 + lh * 16 + gr + 8 * rr;  // row in the item
+              float* dst = score_tile(P, bh, chunk, j >> 7) + rl * 128 + (j & 127);
               const float h0 = __uint_as_float(vh[4 * k + 2 * rr]) * sc_hi;
               const float h1 = __uint_as_float(vh[4 * k + 2 * rr + 1]) * sc_hi;
               const float l0 = __uint_as_float(vl[4 * k + 2 * rr]) * sc_lo;
               const float l1 = __uint_as_float(vl[4 * k + 2 * rr + 1]) * sc_lo;
-              float* dst = score_tile(P, bh, chunk, j >> 7) + rl * 128 + (j & 127);
               *reinterpret_cast<float2*>(dst) = make_float2(h0, h1);
               *reinterpret_cast<float2*>(dst + 128 * 128) = make_float2(l0, l1);
               const int i = i0 + rl;
@@ -1115,7 +1126,8 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_e(c));
     }
-    // the four threads of a row combine their maxima
+    // the four threads of a row combine their maxima; one of them folds them
+    // into the row's maxima over every part
 #pragma unroll
     for (int a = 0; a < 8; ++a) {
       float& v = (&mx[0][0][0])[a];
@@ -1127,21 +1139,16 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
       for (int lh = 0; lh < 2; ++lh)
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
-          const int rl = q4 * 32 + lh * 16 + gr + 8 * rr;
-          sm.rmax[0][0][rl] = sm.rmax[1][0][rl] = mx[lh][rr][0];
-          sm.rmax[0][1][rl] = sm.rmax[1][1][rl] = mx[lh][rr][1];
+          const int i = i0 + q4 * 32 + lh * 16 + gr + 8 * rr;
+          if (i <= max_i && mx[lh][rr][0] > -INFINITY) {  // this part holds keys j <= i of the row
+            atomicMax(&P.rmax[((size_t)bh * P.nb + i) * 2 + 0], max_enc(mx[lh][rr][0]));
+            atomicMax(&P.rmax[((size_t)bh * P.nb + i) * 2 + 1], max_enc(mx[lh][rr][1]));
+          }
         }
     }
   }
-  named_barrier(kBarStream, kStreamThreads);  // score tiles and row maxima complete
-  // publish: the part's row maxima, then count the part for the chunk's Top-P items
-  const int st = stream_tid(t);
-  for (int q = st; q < 256; q += kStreamThreads) {
-    const int rl = q & 127, band = q >> 7, i = i0 + rl;
-    if (i <= max_i)
-      P.rmax[(((size_t)bh * P.nb + i) * P.rparts + part) * 2 + band] = fmaxf(sm.rmax[0][band][rl], sm.rmax[1][band][rl]);
-  }
-  named_barrier(kBarStream, kStreamThreads);
+  named_barrier(kBarStream, kStreamThreads);  // score tiles complete
+  // publish: count the part for the chunk's Top-P rows
   if (t == 0) {
     __threadfence();
     red_release_gpu_add(&P.sync[2 + 2 * P.n_groups + bh * nchunk + chunk], 1u);
@@ -1150,136 +1157,134 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
 }
 
 // ---------------------------------------------------------------------------
-// Top-P item: steps (5)-(7) for kToppRows consecutive query blocks of one
-// (batch, Q head): one warp per row at a time, both bands, union, whole mask
-// row.  A warp's tasks are (row, band) pairs; with two logit buffers the next
-// task's row streams in (cp.async) while the current one is ranked.  The
-// rows' score chunk has been published by its score item.  Run by a team of
-// nw warps (team-local index lw) with `stride` bytes of shared memory each
-// at `region`.
+// Top-P rows: steps (5)-(7) for one query-block row i of one (batch, Q head),
+// both bands, union, the whole mask row.  Every warp of the Top-P lane (and,
+// once the stream queue is empty, of the stream lane) claims rows one at a
+// time from a device queue -- no team barriers -- and waits (bounded) until
+// every part of the row's score chunk is written.  Rows are queued per KV
+// group in the order their score chunks complete (longest rows first).
 // ---------------------------------------------------------------------------
-struct ToppTeam {
-  unsigned char* region;
-  int lw, nw, stride, single;
-};
 
-__device__ __forceinline__ void topp_item(const EstParams& P, int g, int y, const ToppTeam& T) {
-  const int lane = threadIdx.x & 31;
-  const int bi = g / P.hkv, kv = g - bi * P.hkv;
-  const int nseg = (P.nb + kToppRows - 1) / kToppRows;
-  const int seg = nseg - 1 - y / P.G;  // longest rows first
-  const int bh = bi * P.hq + kv * P.G + y % P.G;
-  const int r0 = seg * kToppRows;
-  const int nbb = seq_blocks(P, bi);
-  const int max_i = min(nbb, r0 + kToppRows) - 1;
-  const int chunk = r0 / kScoreRows, i0 = chunk * kScoreRows;
-  const size_t tri = (size_t)P.nb * (P.nb + 1) / 2;
-  if (T.lw >= T.nw) return;
-  {  // rows of the layout past the sequence: empty mask rows
-    const int lo = max(r0, nbb), hi = min(P.nb, r0 + kToppRows);
-    for (int x = T.lw * 32 + (threadIdx.x & 31); x < (hi - lo) * P.W; x += T.nw * 32)
-      P.mask[((size_t)bh * P.nb + lo) * P.W + x] = 0u;
-  }
-  unsigned char* wb = T.region + (size_t)T.lw * T.stride;
-  const int nbp = (P.nb + 7) & ~7;
-  const int nbuf = T.single ? 1 : 2;
-  ToppScratch S;
-  // per warp: nbuf logit rows | bins (2 KB) | member words | bit row
-  S.h = reinterpret_cast<unsigned long long*>(wb + (size_t)nbp * 4 * nbuf);
-  S.memw = reinterpret_cast<uint32_t*>(wb + (size_t)nbp * 4 * nbuf + kTopPBins * 8);
-  uint32_t* bits = S.memw + nbp / 32 + 1;
-  const int nrows = max_i - r0 - T.lw >= 0 ? (max_i - r0 - T.lw) / T.nw + 1 : 0;
-  const int ntasks = 2 * nrows;
-  const float* tiles = score_tile(P, bh, chunk, 0);
-  auto fetch = [&](int task) {  // logits of task -> its buffer, 16-byte pieces
-    const int i = r0 + T.lw + (task >> 1) * T.nw;
-    const float* row = tiles + (i - i0) * 128 + (task & 1) * 128 * 128;
-    const uint32_t dst = smem_u32(wb) + (uint32_t)(task & (nbuf - 1)) * (uint32_t)nbp * 4u;
-    for (int c = lane; c * 4 <= i; c += 32)
-      cp_async16(dst + (uint32_t)c * 16u, row + (size_t)((c * 4) >> 7) * kTilePair + ((c * 4) & 127));
-    cp_async_commit();
-  };
-  if (!T.single && ntasks > 0) fetch(0);
-  // row maxima of the warp's first 32 tasks, one per lane, loaded up front
-  const int np = score_parts(chunk);
-  auto row_max = [&](int i, int band) {  // over the score parts of the row
-    const float* r = P.rmax + ((size_t)bh * P.nb + i) * P.rparts * 2 + band;
-    float m = r[0];
-    for (int q = 1; q < np; ++q) m = fmaxf(m, r[2 * q]);
-    return m;
-  };
-  float my_rmax = 0.f;
-  if (lane < ntasks) my_rmax = row_max(r0 + T.lw + (lane >> 1) * T.nw, lane & 1);
-  for (int task = 0; task < ntasks; ++task) {
-    if (T.single) {
-      fetch(task);  // the buffer is free: the last task ended with __syncwarp
-      cp_async_wait<0>();
-    } else {
-      if (task + 1 < ntasks)
-        fetch(task + 1);
-      else
-        cp_async_commit();  // an empty group keeps the count of groups in flight uniform
-      cp_async_wait<1>();   // this task's pieces have landed
-    }
-    __syncwarp();
-    const int i = r0 + T.lw + (task >> 1) * T.nw, band = task & 1;
-    const int n = i + 1;
-    const float rmax_t = __shfl_sync(0xffffffffu, my_rmax, task & 31);
-    const float rmax = task < 32 ? rmax_t : row_max(i, band);
-    S.d = reinterpret_cast<uint32_t*>(wb + (size_t)(task & (nbuf - 1)) * nbp * 4);
-    const size_t drow = (size_t)bh * 2 * tri + (size_t)band * tri + (size_t)i * (i + 1) / 2;
-    float* dbg = P.dbg_scores ? P.dbg_scores + drow : nullptr;
-    float* dbgw = P.dbg_weights ? P.dbg_weights + drow : nullptr;
-    uint32_t* dst = P.mask + ((size_t)bh * P.nb + i) * P.W;
-    if (band == 0) {
-      for (int w = lane; w < P.W; w += 32) bits[w] = 0u;
-      __syncwarp();
-    }
-    topp_band_row(rmax, n, P.p, S, bits, dbg, dbgw, lane);
-    if (band == 1) {
-      if (P.force && lane == 0) {  // optional additions to M_high | M_low
-        if (P.force & 1) bits[0] |= 1u;
-        if (P.force & 2) bits[i >> 5] |= 1u << (i & 31);
-      }
-      __syncwarp();
-      for (int w = lane; w < P.W; w += 32) dst[w] = bits[w];
-      __syncwarp();
-    }
-  }
-  cp_async_wait<0>();
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
 }
 
-// A lane's (or the stream team's) loop over the Top-P queue.  `leader` claims
-// each item and waits for its score chunk; every thread of the team passes
-// the team's barrier twice per item.
-__device__ __forceinline__ void topp_loop(const EstParams& P, const ToppTeam& T, bool leader, int bar, int nthreads,
-                                          volatile int* s_item, volatile int* s_ok) {
+__device__ __forceinline__ void l2_discard_line(const void* p) {
+  asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
+
+// The warp's shared memory for Top-P rows: keys [nbp] | bins (2 KB, then the
+// member records) | mask bit row [W].
+__device__ __forceinline__ ToppScratch topp_scratch(const EstParams& P, unsigned char* wb, uint32_t*& bits) {
+  const int nbp = (P.nb + 7) & ~7;
+  ToppScratch S;
+  S.d = reinterpret_cast<uint32_t*>(wb);
+  S.h = reinterpret_cast<unsigned long long*>(wb + (size_t)nbp * 4);
+  bits = reinterpret_cast<uint32_t*>(wb + (size_t)nbp * 4 + kTopPBins * 8);
+  return S;
+}
+
+// One query-block row i of one (batch, Q head), both bands: each band's
+// logits are read once, straight from the score tiles (L2, four 128-byte
+// lines per lane iteration in flight), and turned into weights, rank keys
+// (stored for the selection) and exact bin masses against the row maximum the
+// score items published; then the selection runs on shared memory.  Once a
+// band is read, the row's lines of its tiles are dropped from L2 (never read
+// again, so never written back).  The mask row is built in the warp's bit
+// row and written whole.  One compact routine for every row length: the
+// warps of an SM run several roles at once, and the code they share must
+// stay small.
+__device__ __forceinline__ void topp_row(const EstParams& P, int bh, int i, int chunk, unsigned char* wb, int lane) {
+  const int n = i + 1, ns = (n + 31) >> 5;
+  uint32_t* bits;
+  const ToppScratch T = topp_scratch(P, wb, bits);
+  const float* row = score_tile(P, bh, chunk, 0) + (size_t)(i - chunk * kScoreRows) * 128;
+  const size_t tri = (size_t)P.nb * (P.nb + 1) / 2;
+  const bool all = P.p >= 1.0f;
+  for (int w = lane; w < P.W; w += 32) bits[w] = 0u;
+  for (int band = 0; band < 2; ++band) {
+    // slot u of lane L = block 32 u + L: tile u / 4, columns 32 (u % 4) + L
+    const float* rb = row + band * (128 * 128);
+    const size_t drow = ((size_t)bh * 2 + band) * tri + (size_t)i * (i + 1) / 2;
+    float* dbg = P.dbg_scores ? P.dbg_scores + drow : nullptr;
+    const float m = max_dec(__ldcg(P.rmax + ((size_t)bh * P.nb + i) * 2 + band)) * kLog2e;
+    if (!all) topp_zero_bins(T, lane);
+    for (int u0 = 0; u0 < ns; u0 += 4) {
+      float v[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int u = u0 + q;
+        v[q] = 32 * u + lane < n ? __ldcg(rb + (size_t)(u >> 2) * kTilePair + ((u & 3) << 5) + lane) : 0.f;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int j = 32 * (u0 + q) + lane;
+        if (j < n) {
+          if (dbg) dbg[j] = v[q];
+          if (!all) topp_hist1(T, j, v[q], m);
+        }
+      }
+    }
+    __syncwarp();
+    // the row's 4 (chunk + 1) lines of this band, the unused ones above the
+    // diagonal included
+    for (int u = lane; u < 4 * (chunk + 1); u += 32) l2_discard_line(rb + (size_t)(u >> 2) * kTilePair + ((u & 3) << 5));
+    if (all)
+      topp_keep_all(n, bits, lane);
+    else
+      topp_select(n, P.p, T, bits, P.dbg_weights ? P.dbg_weights + drow : nullptr, lane);
+  }
+  if (P.force && lane == 0) {  // optional additions to M_high | M_low
+    if (P.force & 1) bits[0] |= 1u;
+    if (P.force & 2) bits[i >> 5] |= 1u << (i & 31);
+  }
+  __syncwarp();
+  uint32_t* dst = P.mask + ((size_t)bh * P.nb + i) * P.W;
+  for (int w = lane; w < P.W; w += 32) dst[w] = bits[w];
+  __syncwarp();
+}
+
+// A warp's loop over the Top-P queue: entries x = 0, 1, ... of P.n_groups *
+// P.topp_rows, one row per claim (finer claims balance the end of the launch
+// better than batches of rows); per group g, entry y -> score chunk nchunk -
+// 1 - y / (G 128) (longest rows first), Q head y / 128 % G, row y % 128 of the
+// chunk.  The warp claims its next row before it works on the current one,
+// so the claim's latency is hidden.  After its mask row is written a row is
+// counted for its kToppRows-row segment (the attention of a prefill waits on
+// the count).  `wb`: the warp's shared memory (topp_scratch).
+__device__ __forceinline__ void topp_warp_loop(const EstParams& P, unsigned char* wb) {
+  const int lane = threadIdx.x & 31;
   const int nchunk = (P.nb + kScoreRows - 1) / kScoreRows;
   const int nseg = (P.nb + kToppRows - 1) / kToppRows;
+  const int total = P.n_groups * P.topp_rows;
+  int xc = 0;
+  if (lane == 0) xc = (int)atomicAdd(&P.sync[1], 1u);
   for (;;) {
-    if (leader) {
-      const int x = (int)atomicAdd(&P.sync[1], 1u);
-      int g, y, ok = 0;
-      if (decode_topp(P, x, g, y) == kItemTopp) {
-        const int bh = (g / P.hkv) * P.hq + (g % P.hkv) * P.G + y % P.G;
-        const int chunk = (nseg - 1 - y / P.G) * kToppRows / kScoreRows;
-        ok = count_wait_ns(&P.sync[2 + 2 * P.n_groups + bh * nchunk + chunk], (uint32_t)score_parts(chunk),
-                           kWaitLimitNs) ? 1 : 0;
-      }
-      *s_item = x;
-      *s_ok = ok;
+    const int x = __shfl_sync(0xffffffffu, xc, 0);
+    if (x >= total) break;
+    if (lane == 0) xc = (int)atomicAdd(&P.sync[1], 1u);  // the next row, used in the next iteration
+    const int g = x / P.topp_rows, y = x - g * P.topp_rows;
+    const int chunk = nchunk - 1 - y / (P.G * kScoreRows);
+    const int hh = (y / kScoreRows) % P.G;
+    const int i = chunk * kScoreRows + y % kScoreRows;
+    if (i >= P.nb) continue;  // past the layout's last block
+    const int bi = g / P.hkv, kv = g - bi * P.hkv;
+    const int bh = bi * P.hq + kv * P.G + hh;
+    if (i >= seq_blocks(P, bi)) {  // past the sequence: an empty mask row
+      for (int w = lane; w < P.W; w += 32) P.mask[((size_t)bh * P.nb + i) * P.W + w] = 0u;
+    } else {
+      int ok = 1;
+      if (lane == 0)
+        ok = count_wait_ns(&P.sync[2 + 2 * P.n_groups + bh * nchunk + chunk],
+                           (uint32_t)score_parts(chunk, score_part_blocks(P, g)), kWaitLimitNs) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;  // (timed out: error recorded)
+      __syncwarp();  // orders the lanes' loads of the chunk after lane 0's acquire
+      topp_row(P, bh, i, chunk, wb, lane);
     }
-    named_barrier(bar, nthreads);
-    const int x = *s_item, ok = *s_ok;
-    int g, y;
-    if (decode_topp(P, x, g, y) == kItemNone) break;  // no thread passes a barrier after this
-    if (ok) topp_item(P, g, y, T);
-    named_barrier(bar, nthreads);  // the item's shared memory and s_item are reused
-    if (leader && ok) {  // the item's mask rows are final: attention may read them
-      const int bh = (g / P.hkv) * P.hq + (g % P.hkv) * P.G + y % P.G;
-      __threadfence();
-      st_release_gpu(&P.ready[(size_t)bh * nseg + (nseg - 1 - y / P.G)], 1u);
-    }
+    __syncwarp();  // every lane's mask words are written before lane 0 releases them
+    if (lane == 0) red_release_gpu_add(&P.ready[(size_t)bh * nseg + i / kToppRows], 1u);
   }
 }
 
@@ -1292,9 +1297,9 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
   __shared__ PoolSmem psm;
   // a kernel launched after this one with programmatic serialization (the
   // attention of a prefill) may be scheduled on SMs this grid leaves; it
-  // waits for the mask rows it reads through the `ready` flags
+  // waits for the mask rows it reads through the `ready` counters
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  __shared__ int s_next, s_ok, s_titem[2], s_tok[2];
+  __shared__ int s_next, s_ok;
   const int stages = P.pool_stages;
   PoolState pst = {0u, 0u, 0u, 0u, 0};
   ScoreState ss = {0u, 0u, 0u, 0u, 0u};
@@ -1329,7 +1334,8 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
   const int warp = threadIdx.x >> 5;
   if (in_stream_lane(warp)) {
     const int sid = stream_tid(threadIdx.x);
-    const int total = P.n_groups * (P.pool_items + P.score_items);
+    const int lag = min(kScoreLag, P.n_groups);
+    const int total = P.n_groups * P.pool_items + (P.n_groups - lag) * P.score_items + lag * P.score_items_fine;
     // During a pool item thread 0 already claims the lane's next item (the
     // claim's latency is hidden, and a following pool item's tiles can start
     // streaming); a score item claims its successor only when it is done, so
@@ -1356,12 +1362,13 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
       named_barrier(kBarStream, kStreamThreads);
       if (sid == 0) s_next = (int)atomicAdd(&P.sync[0], 1u);
     }
-    // the stream queue is empty: the lane's warps join the Top-P queue
-    const ToppTeam T = {est_smem, stream_warp(warp), P.team_warps, P.team_stride, P.team_single};
-    topp_loop(P, T, sid == 0, kBarStream, kStreamThreads, &s_titem[0], &s_tok[0]);
-  } else if (P.lane_warps > 0) {
-    const ToppTeam T = {est_smem + P.lane_off, lane_warp(warp), P.lane_warps, P.lane_stride, P.lane_single};
-    topp_loop(P, T, threadIdx.x == 64, kBarLane, kLaneThreads, &s_titem[1], &s_tok[1]);
+    // the stream queue is empty (this CTA's last item is done, its shared
+    // memory free): the lane's warps join the Top-P queue
+    const int sw = stream_warp(warp);
+    if (sw < P.team_warps) topp_warp_loop(P, est_smem + (size_t)sw * P.team_stride);
+  } else {
+    const int lw = lane_warp(warp);
+    if (lw < P.lane_warps) topp_warp_loop(P, est_smem + P.lane_off + (size_t)lw * P.lane_stride);
   }
   tc_fence_before();
   __syncthreads();

@@ -35,7 +35,7 @@ struct Plan {
   int force;
   int varlen;            // per-sequence lengths given
   int seq_n[kMaxSeqs];   // tokens of each batch element (n when not varlen)
-  size_t off_pool[kTerms], off_part, off_tau, off_scores, off_rmax, off_mask, off_sync, sync_bytes, total;
+  size_t off_pool[kTerms], off_part, off_tau, off_scores, off_sync, sync_bytes, est_bytes, off_mask, total;
 };
 static_assert(kMaxSeqs == attn::kMaxSeqs, "one sequence limit for both kernels");
 
@@ -129,17 +129,17 @@ int validate(const prism_config* cfg, Plan* pl) {
   P.off_scores = off;
   const size_t nch = ((size_t)P.nb + 127) / 128;
   off = align_up(off + (size_t)P.q_rows * (nch * (nch + 1) / 2) * 2 * 128 * 128 * sizeof(float), 256);
-  P.off_rmax = off;
-  off = align_up(off + (size_t)P.q_rows * P.nb * score_parts((int)nch - 1) * 2 * sizeof(float), 256);
-  P.off_mask = off;
-  off = align_up(off + (size_t)P.q_rows * P.nb * P.W * sizeof(uint32_t), 256);
   P.off_sync = off;
   // queue heads, per-group counters and ready flags, per (batch, Q head, score chunk) part counters,
-  // per (batch, Q head, Top-P segment) mask-rows-written flags
+  // per (batch, Q head, kToppRows-row segment) mask-rows-written counters
+  // and the row maxima of the band scores ([q_rows, nb, 2], combined with atomicMax from 0)
   P.sync_bytes = (2 + 2 * (size_t)P.kv_rows + (size_t)P.q_rows * nch +
-                  (size_t)P.q_rows * (((size_t)P.nb + kToppRows - 1) / kToppRows)) *
+                  (size_t)P.q_rows * (((size_t)P.nb + kToppRows - 1) / kToppRows) + (size_t)P.q_rows * P.nb * 2) *
                  sizeof(uint32_t);
   off = align_up(off + P.sync_bytes, 256);
+  P.est_bytes = off;  // the estimator uses [0, est_bytes); the mask slot after it is prism_prefill's
+  P.off_mask = off;
+  off = align_up(off + (size_t)P.q_rows * P.nb * P.W * sizeof(uint32_t), 256);
   P.total = off;
   return PRISM_OK;
 }
@@ -161,35 +161,32 @@ static_assert(kGemmSmemBytes + sizeof(PoolSmem) + 256 <= 232448, "estimator shar
 constexpr size_t kEstMaxDyn = 232448 - sizeof(PoolSmem) - 256;
 
 struct EstLaunch {
-  int lane_warps, lane_stride, lane_single;
-  int team_warps, team_stride, team_single;
+  int lane_warps, lane_stride;
+  int team_warps, team_stride;
   size_t stream, smem;
   int stages;
 };
-// Per Top-P warp: one or two logit rows (keys replace the logits in place),
-// 256 64-bit bins, a member bit row and the mask bit row.
-static size_t topp_stride(int nb, bool single) {
+// Per Top-P warp: a row's logits (replaced by their keys), 256 64-bit bins
+// and the mask bit row.
+static size_t topp_stride(int nb) {
   const size_t W = ((size_t)nb + 31) / 32, nbp = ((size_t)nb + 7) & ~(size_t)7;
-  return align_up(nbp * 4 * (single ? 1 : 2) + 256 * 8 + (nbp / 32 + 1) * 4 + W * 4, 16);
+  return align_up(nbp * 4 + kTopPBins * 8 + W * 4, 16);
 }
-// Fills L; false if not even one Top-P warp fits beside the product operands.
+// Fills L; false if the score operands or not even one Top-P warp fit.  The
+// Top-P lane takes what the score operands leave; the stream lane's warps use
+// the stream region once the stream queue is empty.
 bool est_launch_shape(int nb, int dp, EstLaunch& L) {
-  const size_t sd = topp_stride(nb, false), ss = topp_stride(nb, true);
-  const size_t base = (size_t)gemm_smem_bytes(dp);
-  const size_t rest = kEstMaxDyn - base;
-  const int nd = (int)std::min<size_t>(kLaneWarpsMax, rest / sd), ns = (int)std::min<size_t>(kLaneWarpsMax, rest / ss);
-  L.lane_single = ns > nd;
-  L.lane_warps = L.lane_single ? ns : nd;
-  L.lane_stride = (int)(L.lane_single ? ss : sd);
-  const size_t lane_bytes = (size_t)L.lane_warps * L.lane_stride;
+  const size_t gemm = (size_t)gemm_smem_bytes(dp);
+  const size_t st = topp_stride(nb);
+  L.lane_warps = gemm >= kEstMaxDyn ? 0 : (int)std::min<size_t>(kLaneWarpsMax, (kEstMaxDyn - gemm) / st);
+  L.lane_stride = (int)st;
+  const size_t lane_bytes = (size_t)L.lane_warps * st;
   L.stream = (kEstMaxDyn - lane_bytes) & ~(size_t)15;  // what the lane leaves: more ring stages
-  const int td = (int)std::min<size_t>(kTeamWarpsMax, L.stream / sd);
-  L.team_single = td == 0;
-  L.team_warps = td > 0 ? td : (int)std::min<size_t>(kTeamWarpsMax, L.stream / ss);
-  L.team_stride = (int)(td > 0 ? sd : ss);
+  L.team_warps = (int)std::min<size_t>(kTeamWarpsMax, L.stream / st);
+  L.team_stride = (int)st;
   L.smem = L.stream + lane_bytes;
   L.stages = (int)std::min<size_t>(kMaxPoolStages, (L.stream - 1024) / kTileBytes);  // 1 KB-aligned ring
-  return L.team_warps > 0;
+  return gemm <= L.stream && L.stages >= 2 && (L.lane_warps > 0 || L.team_warps > 0);
 }
 
 int g_num_sms[kMaxDevices];
@@ -323,9 +320,9 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   E.dbg_tau = dbg ? dbg->tau : nullptr;
   E.dbg_pooled = dbg ? dbg->pooled : nullptr;
   E.mask = mask;
-  E.rmax = reinterpret_cast<float*>(ws + P.off_rmax);
   E.sync = reinterpret_cast<uint32_t*>(ws + P.off_sync);
   E.ready = E.sync + ready_offset(P);
+  E.rmax = E.ready + (size_t)P.q_rows * (((size_t)P.nb + kToppRows - 1) / kToppRows);
   E.hq = P.hq;
   E.hkv = P.hkv;
   E.G = P.hq / P.hkv;
@@ -338,20 +335,21 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   E.pool_items = (E.G + 1) * E.pool_item_span;
   {
     const int nchunk = (P.nb + kScoreRows - 1) / kScoreRows;
-    E.score_span = 0;
-    for (int c = 0; c < nchunk; ++c) E.score_span += score_parts(c);
+    E.score_span = E.score_span_fine = 0;
+    for (int c = 0; c < nchunk; ++c) {
+      E.score_span += score_parts(c, kScorePartBlocks);
+      E.score_span_fine += score_parts(c, kScorePartFine);
+    }
     E.score_items = E.G * E.score_span;
-    E.rparts = score_parts(nchunk - 1);
+    E.score_items_fine = E.G * E.score_span_fine;
+    E.topp_rows = nchunk * E.G * kScoreRows;
   }
-  E.topp_items = E.G * ((P.nb + kToppRows - 1) / kToppRows);
   EstLaunch L;
   if (!est_launch_shape(P.nb, P.bl.dp, L)) return PRISM_ERR_UNSUPPORTED;
   E.lane_warps = L.lane_warps;
   E.lane_stride = L.lane_stride;
-  E.lane_single = L.lane_single;
   E.team_warps = L.team_warps;
   E.team_stride = L.team_stride;
-  E.team_single = L.team_single;
   E.lane_off = (int)L.stream;
   E.stream_bytes = (int)L.stream;
   E.pool_stages = L.stages;
@@ -368,7 +366,7 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, estimator_kernel, kEstThreads, L.smem) !=
           cudaSuccess)
     return PRISM_ERR_CUDA;
-  const long long items = (long long)E.n_groups * (E.pool_items + E.score_items + E.topp_items);
+  const long long items = (long long)E.n_groups * (E.pool_items + E.score_items + E.topp_rows / kScoreRows);
   const long long grid = std::min<long long>(items, (long long)g_num_sms[dev] * std::max(per_sm, 1));
   // the score items' operands: pooled rows as bf16 [rows, dp], boxes of 64
   // dims x 128 rows (A, and B when dp <= 128) or x 64 rows (B when dp = 192)
@@ -549,7 +547,7 @@ int prism_estimate_noalloc(const prism_config* cfg, const void* q, const void* k
   int s = validate(cfg, &P);
   if (s != PRISM_OK) return s;
   if (!q || !k || !mask) return PRISM_ERR_NULL;
-  if (P.total > kStaticScratchBytes) return PRISM_ERR_SCRATCH_LIMIT;
+  if (P.est_bytes > kStaticScratchBytes) return PRISM_ERR_SCRATCH_LIMIT;  // the estimator's part of the workspace
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(mask, 4)) return PRISM_ERR_ALIGN;
   if ((s = ensure_device()) != PRISM_OK) return s;
   void* scratch = nullptr;

@@ -79,12 +79,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   return mbar_wait_ns(bar, parity, kWaitLimitNs);
 }
 // Waits until a global word another CTA publishes (release) becomes nonzero.
+// Between polls the thread sleeps briefly, so a waiting warp leaves the SM's
+// issue slots and L2 bandwidth to the warps that work.
 __device__ __forceinline__ bool flag_wait_ns(const uint32_t* flag, uint64_t limit_ns) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
   if (v != 0u) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
+    __nanosleep(200);
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
     if (v != 0u) return true;
     if (globaltimer_ns() - t0 > limit_ns) {
@@ -101,6 +104,7 @@ __device__ __forceinline__ bool count_wait_ns(const uint32_t* ctr, uint32_t targ
   if (v >= target) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
+    __nanosleep(200);
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
     if (v >= target) return true;
     if (globaltimer_ns() - t0 > limit_ns) {
@@ -138,6 +142,21 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
       : "memory");
+}
+// The same with an L2 cache policy (createpolicy) for the loaded lines.
+__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                                 uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(policy)
+      : "memory");
+}
+// An L2 policy that evicts the lines it is applied to first (streamed data).
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
                                             uint32_t bar) {

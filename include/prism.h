@@ -226,10 +226,11 @@ int prism_prefill(const prism_config* cfg, const void* q, const void* k, const v
  * of prism_noalloc_scratch_bytes() = 32 MiB that every GPU loading the library
  * holds until the process exits.  The caller still passes q, k and mask
  * (device pointers, layouts as above); no dbg outputs.
- *   - Problems whose workspace (prism_workspace_size) exceeds 32 MiB are
- *     rejected with PRISM_ERR_SCRATCH_LIMIT before anything is enqueued
- *     (the Llama-3-8B shape, 32 Q / 8 KV heads, batch 1, fits up to 32,768
- *     tokens = 256 blocks).
+ *   - Problems whose estimator workspace (prism_workspace_size less the
+ *     mask slot only prism_prefill uses) exceeds 32 MiB are rejected with
+ *     PRISM_ERR_SCRATCH_LIMIT before anything is enqueued (the Llama-3-8B
+ *     shape, 32 Q / 8 KV heads, batch 1, fits up to 265 blocks = 33,920
+ *     tokens).
  *   - The first call on a device looks up the array's device address with
  *     cudaGetSymbolAddress while that device is current; make that first call
  *     before any stream capture.

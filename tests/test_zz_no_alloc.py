@@ -48,11 +48,17 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda_device):
         assert torch.equal(got, ref), f"{w.name}: {(got != ref).sum().item()} mask words differ"
 
 
+def _estimator_bytes(cfg):
+    """The workspace less the mask slot that only prism_prefill uses."""
+    mask_slot = -(-cfg.c.batch * cfg.c.hq * cfg.nb * cfg.words * 4 // 256) * 256
+    return pb.prism_workspace_size(cfg) - mask_slot
+
+
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda_device):
     hi, lo = gen.default_bands()
-    fits = pb.PrismConfig(1, 32, 8, 256 * 128, hi, lo, 0.95)
-    too_big = pb.PrismConfig(1, 32, 8, 257 * 128, hi, lo, 0.95)
-    assert pb.prism_workspace_size(fits) <= pb.prism_noalloc_scratch_bytes()
-    assert pb.prism_workspace_size(too_big) > pb.prism_noalloc_scratch_bytes()
+    fits = pb.PrismConfig(1, 32, 8, 265 * 128, hi, lo, 0.95)
+    too_big = pb.PrismConfig(1, 32, 8, 266 * 128, hi, lo, 0.95)
+    assert _estimator_bytes(fits) <= pb.prism_noalloc_scratch_bytes() < pb.prism_workspace_size(fits)
+    assert _estimator_bytes(too_big) > pb.prism_noalloc_scratch_bytes()
     a = 1 << 20  # never dereferenced: the size check runs before anything is enqueued
     assert pb.lib.prism_estimate_noalloc(too_big.ptr(), a, a, a, None) == -12
