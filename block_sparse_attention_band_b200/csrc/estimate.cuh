@@ -63,13 +63,18 @@ constexpr int kToppRows = 16;         // mask rows per ready counter (what the a
 constexpr uint32_t kOpChunk = 128 * 64 * 2;  // one 64-dim x 128-row bf16 operand chunk (SW128)
 constexpr int kTerms = 3;             // bf16 terms per pooled value
 // product operands: A (3 terms x dp/64 chunks of 128 rows) once, B one term at
-// a time in kBSlots slots (dp/64 chunks of N rows; N = 128, or 64 when dp = 192)
+// a time in kBSlots slots (dp/64 chunks of N rows)
 constexpr int kBSlots = 2;
-__host__ __device__ constexpr int score_cols(int dp) { return dp <= 128 ? 128 : 64; }
-__host__ __device__ constexpr int gemm_smem_bytes(int dp) {
-  return kTerms * (dp / 64) * (int)kOpChunk + kBSlots * (dp / 64) * score_cols(dp) * 128 + 1024;
+// N, the key blocks of one product: 128, or 64 when the pooled rows are 192
+// wide (the operands must fit) or the rows are long (from nb = 2048 on, the
+// Top-P warps' key buffers need the shared memory; halving the B slots leaves
+// room for more of them)
+constexpr int kWideRowsNb = 2048;
+__host__ __device__ constexpr int score_cols(int dp, int nb) { return dp <= 128 && nb < kWideRowsNb ? 128 : 64; }
+__host__ __device__ constexpr int gemm_smem_bytes(int dp, int ncolw) {
+  return kTerms * (dp / 64) * (int)kOpChunk + kBSlots * (dp / 64) * ncolw * 128 + 1024;
 }
-constexpr int kGemmSmemBytes = gemm_smem_bytes(192);  // the largest layout: 144 + 2 x 24 KB + alignment
+constexpr int kGemmSmemBytes = gemm_smem_bytes(192, 64);  // the largest layout: 144 + 2 x 24 KB + alignment
 
 // The CTA's warps form two lanes that take items from two queues at once:
 // the stream lane (warps 0, 1, 4-7) runs pool and score items, the Top-P
@@ -121,7 +126,7 @@ struct EstParams {
   int pool_items;      // per group
   int score_items;     // per group (kScorePartBlocks parts)
   int score_span;      // score items per head: (row chunk, key-block part) pairs
-  int score_items_fine, score_span_fine;  // the same with kScorePartFine parts (the last kScoreLag groups)
+  int score_items_fine, score_span_fine;  // the same with kScorePartFine parts (score_fine groups)
   int topp_rows;       // Top-P queue entries per group: nchunk x G x kScoreRows (rows past nb skipped)
   int pool_item_span;  // pool items per head row
   // Top-P warps of each lane: how many take rows and bytes of shared memory
@@ -130,6 +135,7 @@ struct EstParams {
   int team_warps, team_stride;
   int lane_off;      // byte offset of the Top-P lane's shared memory
   int stream_bytes;  // dynamic shared memory of the stream lane (pool ring, score operands)
+  int ncolw;         // key blocks per score product (score_cols)
   int pool_stages;   // TMA ring depth (<= kMaxPoolStages)
   float p;
   int explicit_tau;
@@ -160,8 +166,11 @@ __host__ __device__ __forceinline__ int score_parts(int chunk, int pb) {
   return (chunk * kScoreRows + kScoreRows + pb - 1) / pb;
 }
 constexpr int kScoreLag = 2;  // scoring of group g follows pooling of group g + kScoreLag
+__device__ __forceinline__ bool score_fine(const EstParams& P, int g) {
+  return g >= P.n_groups - min(kScoreLag, P.n_groups);
+}
 __device__ __forceinline__ int score_part_blocks(const EstParams& P, int g) {
-  return g >= P.n_groups - min(kScoreLag, P.n_groups) ? kScorePartFine : kScorePartBlocks;
+  return score_fine(P, g) ? kScorePartFine : kScorePartBlocks;
 }
 // Item z of one head (longest rows first) -> (row chunk, part).
 __device__ __forceinline__ void score_part_of(const EstParams& P, int z, int pb, int& chunk, int& part) {
@@ -344,14 +353,15 @@ struct PoolState {  // per-role counters of ring stages and items, carried acros
 // the group's items of that kind.
 enum : int { kItemPool = 0, kItemScore = 1, kItemNone = -1 };
 __device__ __forceinline__ int decode_stream(const EstParams& P, int x, int& g, int& y) {
-  const int n = P.n_groups, PI = P.pool_items, SI = P.score_items;
-  const int lag = min(kScoreLag, n), M = n - lag, L = PI + SI;
+  const int n = P.n_groups, PI = P.pool_items;
+  const int lag = min(kScoreLag, n), M = n - lag;
   if (x < lag * PI) {
     g = x / PI;
     y = x - g * PI;
     return kItemPool;
   }
   x -= lag * PI;
+  const int L = PI + P.score_items;
   if (x < M * L) {  // pairs p = 0 .. M-1: pool(p + lag) score(p)
     const int p = x / L, rem = x - p * L;
     if (rem < PI) {
@@ -996,7 +1006,7 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
   const int nbb = seq_blocks(P, bi);
   const int max_i = min(nbb, i0 + kScoreRows) - 1;  // < i0: the chunk is past the sequence, only counted
   const uint32_t nch = (uint32_t)P.bl.dp / 64;
-  const int ncolw = score_cols(P.bl.dp);  // N: key blocks per column chunk
+  const int ncolw = P.ncolw;  // N: key blocks per column chunk
   // this part's key blocks [j0, j1): column chunks c0 .. c0 + ncol - 1
   const int j0 = part * pb, j1 = min(j0 + pb, max_i + 1);
   const int c0 = j0 / ncolw;
@@ -1004,7 +1014,7 @@ __device__ __forceinline__ void score_item(const EstParams& P, const CUtensorMap
   const int units = 3 * ncol;
   const uint32_t idesc = ncolw == 128 ? idesc_bf16_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 64, 0, 0);
   const uint32_t sbase = (smem_u32(smem) + 1023u) & ~1023u;
-  if (sbase - smem_u32(smem) + (uint32_t)gemm_smem_bytes(P.bl.dp) - 1024u > (uint32_t)P.stream_bytes) {
+  if (sbase - smem_u32(smem) + (uint32_t)gemm_smem_bytes(P.bl.dp, ncolw) - 1024u > (uint32_t)P.stream_bytes) {
     if (t == 0) set_device_error(-6);  // PRISM_ERR_UNSUPPORTED (host sizing makes this unreachable)
     return;
   }
@@ -1187,15 +1197,19 @@ __device__ __forceinline__ ToppScratch topp_scratch(const EstParams& P, unsigned
 }
 
 // One query-block row i of one (batch, Q head), both bands: each band's
-// logits are read once, straight from the score tiles (L2, four 128-byte
-// lines per lane iteration in flight), and turned into weights, rank keys
-// (stored for the selection) and exact bin masses against the row maximum the
-// score items published; then the selection runs on shared memory.  Once a
-// band is read, the row's lines of its tiles are dropped from L2 (never read
-// again, so never written back).  The mask row is built in the warp's bit
-// row and written whole.  One compact routine for every row length: the
-// warps of an SM run several roles at once, and the code they share must
-// stay small.
+// logits are read once, straight from the score tiles in L2, and turned into
+// weights, rank keys (stored for the selection) and exact bin masses against
+// the row maximum the score items published; then the selection runs on
+// shared memory.  The loads are software-pipelined: eight 128-byte lines per
+// lane group, the next group's loads issued before the current group is
+// ranked, and the next band's first group issued before this band's
+// selection, so L2 latency is paid about once per band rather than once per
+// group.  Once a band is read, the row's lines of its tiles are dropped from
+// L2 (never read again, so never written back).  The mask row is built in the
+// warp's bit row and written whole.  One compact routine for every row
+// length: the warps of an SM run several roles at once, and the code they
+// share must stay small.
+constexpr int kToppGroup = 8;  // slots (32-block columns of a row) per load group
 __device__ __forceinline__ void topp_row(const EstParams& P, int bh, int i, int chunk, unsigned char* wb, int lane) {
   const int n = i + 1, ns = (n + 31) >> 5;
   uint32_t* bits;
@@ -1203,34 +1217,45 @@ __device__ __forceinline__ void topp_row(const EstParams& P, int bh, int i, int 
   const float* row = score_tile(P, bh, chunk, 0) + (size_t)(i - chunk * kScoreRows) * 128;
   const size_t tri = (size_t)P.nb * (P.nb + 1) / 2;
   const bool all = P.p >= 1.0f;
+  // slot u of lane L = block 32 u + L: tile u / 4, columns 32 (u % 4) + L
+  auto slot_ptr = [&](int band, int u) {
+    return row + band * (128 * 128) + (size_t)(u >> 2) * kTilePair + ((u & 3) << 5) + lane;
+  };
+  float v[kToppGroup];
+  auto load_group = [&](int band, int u0) {
+#pragma unroll
+    for (int q = 0; q < kToppGroup; ++q)
+      v[q] = 32 * (u0 + q) + lane < n ? __ldcg(slot_ptr(band, u0 + q)) : 0.f;
+  };
+  const uint32_t* rm = P.rmax + ((size_t)bh * P.nb + i) * 2;
+  const uint32_t rm0 = __ldcg(rm), rm1 = __ldcg(rm + 1);
   for (int w = lane; w < P.W; w += 32) bits[w] = 0u;
+  load_group(0, 0);
   for (int band = 0; band < 2; ++band) {
-    // slot u of lane L = block 32 u + L: tile u / 4, columns 32 (u % 4) + L
-    const float* rb = row + band * (128 * 128);
     const size_t drow = ((size_t)bh * 2 + band) * tri + (size_t)i * (i + 1) / 2;
     float* dbg = P.dbg_scores ? P.dbg_scores + drow : nullptr;
-    const float m = max_dec(__ldcg(P.rmax + ((size_t)bh * P.nb + i) * 2 + band)) * kLog2e;
+    const float m = max_dec(band == 0 ? rm0 : rm1) * kLog2e;
     if (!all) topp_zero_bins(T, lane);
-    for (int u0 = 0; u0 < ns; u0 += 4) {
-      float v[4];
+    for (int u0 = 0; u0 < ns; u0 += kToppGroup) {
+      float cur[kToppGroup];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int u = u0 + q;
-        v[q] = 32 * u + lane < n ? __ldcg(rb + (size_t)(u >> 2) * kTilePair + ((u & 3) << 5) + lane) : 0.f;
-      }
+      for (int q = 0; q < kToppGroup; ++q) cur[q] = v[q];
+      if (u0 + kToppGroup < ns) load_group(band, u0 + kToppGroup);  // in flight while this group is ranked
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < kToppGroup; ++q) {
         const int j = 32 * (u0 + q) + lane;
         if (j < n) {
-          if (dbg) dbg[j] = v[q];
-          if (!all) topp_hist1(T, j, v[q], m);
+          if (dbg) dbg[j] = cur[q];
+          if (!all) topp_hist1(T, j, cur[q], m);
         }
       }
     }
     __syncwarp();
     // the row's 4 (chunk + 1) lines of this band, the unused ones above the
     // diagonal included
-    for (int u = lane; u < 4 * (chunk + 1); u += 32) l2_discard_line(rb + (size_t)(u >> 2) * kTilePair + ((u & 3) << 5));
+    for (int u = lane; u < 4 * (chunk + 1); u += 32)
+      l2_discard_line(row + band * (128 * 128) + (size_t)(u >> 2) * kTilePair + ((u & 3) << 5));
+    if (band == 0) load_group(1, 0);  // in flight during this band's selection
     if (all)
       topp_keep_all(n, bits, lane);
     else
@@ -1334,8 +1359,8 @@ estimator_kernel(const __grid_constant__ EstParams P, const __grid_constant__ Te
   const int warp = threadIdx.x >> 5;
   if (in_stream_lane(warp)) {
     const int sid = stream_tid(threadIdx.x);
-    const int lag = min(kScoreLag, P.n_groups);
-    const int total = P.n_groups * P.pool_items + (P.n_groups - lag) * P.score_items + lag * P.score_items_fine;
+    int total = P.n_groups * P.pool_items;
+    for (int gg = 0; gg < P.n_groups; ++gg) total += score_fine(P, gg) ? P.score_items_fine : P.score_items;
     // During a pool item thread 0 already claims the lane's next item (the
     // claim's latency is hidden, and a following pool item's tiles can start
     // streaming); a score item claims its successor only when it is done, so

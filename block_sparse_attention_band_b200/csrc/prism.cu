@@ -176,7 +176,7 @@ static size_t topp_stride(int nb) {
 // Top-P lane takes what the score operands leave; the stream lane's warps use
 // the stream region once the stream queue is empty.
 bool est_launch_shape(int nb, int dp, EstLaunch& L) {
-  const size_t gemm = (size_t)gemm_smem_bytes(dp);
+  const size_t gemm = (size_t)gemm_smem_bytes(dp, score_cols(dp, nb));
   const size_t st = topp_stride(nb);
   L.lane_warps = gemm >= kEstMaxDyn ? 0 : (int)std::min<size_t>(kLaneWarpsMax, (kEstMaxDyn - gemm) / st);
   L.lane_stride = (int)st;
@@ -352,6 +352,7 @@ int run_estimate(const Plan& P, const void* q, const void* k, uint32_t* mask, un
   E.team_stride = L.team_stride;
   E.lane_off = (int)L.stream;
   E.stream_bytes = (int)L.stream;
+  E.ncolw = score_cols(P.bl.dp, P.nb);
   E.pool_stages = L.stages;
   E.p = P.p_eff;
   E.explicit_tau = P.explicit_tau;
