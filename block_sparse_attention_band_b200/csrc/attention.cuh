@@ -15,7 +15,9 @@
 // 384 threads (12 warps; registers re-split per warpgroup: warps 0-3 keep 72,
 // the two softmax warpgroups get 216 so a whole S row stays in registers):
 //   warp 0      TMA producer: Q_A, Q_B once; K_j, V_j of every visited block
-//               into a 2-stage ring (128-byte swizzled, two 16 KB halves each)
+//               into a 2-stage ring (128-byte swizzled, two 16 KB halves
+//               each).  A K stage is refilled once the Q K^T products that
+//               read it are done, a V stage once its P V products are.
 //   warp 1      MMA issuer (one thread), tcgen05.mma kind::f16, bf16 in /
 //               fp32 accumulate in tensor memory (512 columns):
 //                 S_A = cols [0,128)  S_B = [128,256)  O_A = [256,384)  O_B = [384,512)
@@ -25,6 +27,10 @@
 //               tile's softmax overlaps the other tile's matrix products;
 //               each P V product starts on keys 0-63 as soon as the softmax
 //               has published that half of P, while it computes the other.
+//               A tile that skips step t but takes step t + 1 gets its Q K^T
+//               at the start of step t when K(t + 1) has already landed, so
+//               its softmax runs beside the other tile's (at low density more
+//               than half the steps feed one tile only, mostly alternating).
 //   warps 2-3   idle
 //   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: thread =
 //               query row = tensor-memory lane 32*(warp%4)+lane.  Online
@@ -62,13 +68,14 @@ enum : uint32_t {
   kBarQ = 0,
   kBarKFull = 1,    // [2]
   kBarVFull = 3,    // [2]
-  kBarKVEmpty = 5,  // [2]
+  kBarKEmpty = 5,   // [2] the Q K^T products that read the K stage are done
   kBarSFull = 7,    // [2] per tile
   kBarPFull = 9,    // [2] per tile
   kBarODone = 11,   // [2] per tile
   kBarPHalf = 13,   // [2] per tile: P of keys 0-63 written
   kBarDone = 15,    // softmax threads finished with tensor memory
-  kNumBars = 16
+  kBarVEmpty = 16,  // [2] the P V products that read the V stage are done
+  kNumBars = 18
 };
 
 // Per-sequence token counts of a batch whose sequences differ in length
@@ -145,25 +152,28 @@ __device__ __forceinline__ int count_kept(const Tile& t) {
   return n;
 }
 
-__device__ __forceinline__ void mma_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+// S = Q K^T.  q_lo / k_lo: low words of the shared memory descriptors of the
+// Q tile and the K stage (K-major, 128-byte swizzle; hi the common high
+// word); the eight K steps of 16 dims move the address field (16-byte units).
+__device__ __forceinline__ void mma_qk(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo, uint32_t hi) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);  // Q K-major, K K-major
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-    mma_bf16_ss(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024), smem_desc_sw128(k_smem + off, 16, 1024),
-                idesc, kk > 0);
+    const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) / 16;
+    mma_bf16_ss_lo(d_tmem, q_lo + off, k_lo + off, hi, idesc, kk > 0);
   }
 }
 
 // O += P V over keys [64 part, 64 part + 64): four K steps of 16 keys
-__device__ __forceinline__ void mma_pv_part(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate,
-                                            int part) {
+// (v_lo: low word of the V stage's descriptor, MN-major, 2 KB per 16 keys)
+__device__ __forceinline__ void mma_pv_part(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_lo, uint32_t hi,
+                                            bool accumulate, int part) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 1);  // P K-major (TMEM), V MN-major
 #pragma unroll
   for (int k4 = 0; k4 < 4; ++k4) {
     const int kk = part * 4 + k4;
-    mma_bf16_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(v_smem + kk * 2048, kHalfBytes, 1024), idesc,
-                (accumulate || kk > 0) ? 1u : 0u);
+    mma_bf16_ts_lo(o_tmem, p_tmem + kk * 8, v_lo + (uint32_t)(kk * 2048 / 16), hi, idesc,
+                   (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -322,12 +332,16 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           const int j = it.next(ia, ib);
           if (j < 0) break;
           const int s = t & 1;
-          if (t >= 2 && !mbar_wait(bar(kBarKVEmpty + s), ((t >> 1) - 1) & 1)) break;
+          // a K stage is refilled once the Q K^T products that read it are
+          // done, a V stage once its P V products are: K(t + 1) then lands
+          // about a step ahead of its first use
+          if (t >= 2 && !mbar_wait(bar(kBarKEmpty + s), ((t >> 1) - 1) & 1)) break;
           const int kr = j * 128;
           const uint32_t kd = sbase + kOffK + s * kTileBytes, vd = sbase + kOffV + s * kTileBytes;
           mbar_arrive_expect_tx(bar(kBarKFull + s), kTileBytes);
           tma_load_3d(kd, &tmK, 0, kr, kv_global, bar(kBarKFull + s));
           tma_load_3d(kd + kHalfBytes, &tmK, 64, kr, kv_global, bar(kBarKFull + s));
+          if (t >= 2 && !mbar_wait(bar(kBarVEmpty + s), ((t >> 1) - 1) & 1)) break;
           mbar_arrive_expect_tx(bar(kBarVFull + s), kTileBytes);
           tma_load_3d(vd, &tmV, 0, kr, kv_global, bar(kBarVFull + s));
           tma_load_3d(vd + kHalfBytes, &tmV, 64, kr, kv_global, bar(kBarVFull + s));
@@ -341,7 +355,14 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       if (nA + nB > 0 && mbar_wait(bar(kBarQ), 0)) {
         const uint32_t tS[2] = {tmem, tmem + 128};
         const uint32_t tO[2] = {tmem + 256, tmem + 384};
-        const uint32_t qs[2] = {sbase + kOffQ, sbase + kOffQ + kTileBytes};
+        // descriptor low words: Q tile x, K / V stage s at + x (s) * kStep
+        constexpr uint32_t kStep = kTileBytes / 16;
+        const uint64_t qdesc = smem_desc_sw128(sbase + kOffQ, 16, 1024);
+        const uint32_t hi = (uint32_t)(qdesc >> 32);  // the same for every descriptor here
+        const uint32_t qs0 = (uint32_t)qdesc;
+        const uint32_t qs[2] = {qs0, qs0 + kStep};
+        const uint32_t kd0 = qs0 + (kOffK - kOffQ) / 16;
+        const uint32_t vd0 = (uint32_t)smem_desc_sw128(sbase + kOffV, kHalfBytes, 1024);
         int u[2] = {0, 0};  // per-tile count of P V products issued
         UnionIter it;
         it.init(&tiles[0], &tiles[1]);
@@ -352,38 +373,57 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           tc_fence_after();
           for (int x = 0; x < 2; ++x)
             if (in_cur[x]) {
-              mma_qk(tS[x], qs[x], sbase + kOffK);
+              mma_qk(tS[x], qs[x], kd0, hi);
               mma_commit(bar(kBarSFull + x));
             }
+          mma_commit(bar(kBarKEmpty + 0));
         }
         for (int t = 0; ok && j >= 0; ++t) {
           const int s = t & 1;
           const int jn = it.next(in_nxt[0], in_nxt[1]);
-          if (!(ok = mbar_wait(bar(kBarVFull + s), (t >> 1) & 1))) break;
           bool k_ready = false;
+          // a tile that skips step t but takes step t + 1 gets its Q K^T right
+          // away if K(t + 1) has landed (no wait here), so its softmax runs
+          // beside this step's; else in its place below
+          const uint32_t late =
+              jn >= 0 ? ((in_nxt[0] && !in_cur[0]) ? 1u : 0u) | ((in_nxt[1] && !in_cur[1]) ? 2u : 0u) : 0u;
+          uint32_t early = 0;
+          if (late && mbar_test_wait(bar(kBarKFull + (s ^ 1)), ((t + 1) >> 1) & 1)) {
+            tc_fence_after();
+            k_ready = true;
+            early = late;
+#pragma unroll 1
+            for (int x = 0; x < 2; ++x)
+              if ((late >> x) & 1u) {
+                mma_qk(tmem + 128 * x, qs0 + x * kStep, kd0 + (s ^ 1) * kStep, hi);
+                mma_commit(bar(kBarSFull + x));
+              }
+          }
+          if (!(ok = mbar_wait(bar(kBarVFull + s), (t >> 1) & 1))) break;
           for (int x = 0; x < 2; ++x) {
             if (in_cur[x]) {
               if (!(ok = mbar_wait(bar(kBarPHalf + x), u[x] & 1))) break;
               tc_fence_after();
-              mma_pv_part(tO[x], tS[x], sbase + kOffV + s * kTileBytes, u[x] > 0, 0);
+              mma_pv_part(tO[x], tS[x], vd0 + s * kStep, hi, u[x] > 0, 0);
               if (!(ok = mbar_wait(bar(kBarPFull + x), u[x] & 1))) break;
               tc_fence_after();
-              mma_pv_part(tO[x], tS[x], sbase + kOffV + s * kTileBytes, true, 1);
+              mma_pv_part(tO[x], tS[x], vd0 + s * kStep, hi, true, 1);
               mma_commit(bar(kBarODone + x));
               ++u[x];
             }
-            if (jn >= 0 && in_nxt[x]) {
+            if (jn >= 0 && in_nxt[x] && !((early >> x) & 1u)) {
               if (!k_ready) {
                 if (!(ok = mbar_wait(bar(kBarKFull + (s ^ 1)), ((t + 1) >> 1) & 1))) break;
                 tc_fence_after();
                 k_ready = true;
               }
-              mma_qk(tS[x], qs[x], sbase + kOffK + (s ^ 1) * kTileBytes);
+              mma_qk(tS[x], qs[x], kd0 + (s ^ 1) * kStep, hi);
               mma_commit(bar(kBarSFull + x));
             }
           }
           if (!ok) break;
-          mma_commit(bar(kBarKVEmpty + s));
+          mma_commit(bar(kBarVEmpty + s));
+          if (jn >= 0) mma_commit(bar(kBarKEmpty + (s ^ 1)));
           j = jn;
           in_cur[0] = in_nxt[0];
           in_cur[1] = in_nxt[1];
