@@ -13,7 +13,8 @@ each step every rank runs its share, the step time is the max over ranks and
 ``value`` is ms per whole layer (strong scaling).  ``--impl reference`` times
 the fp64 CPU oracle on a bounded sample of the same layer (rank 0 only).
 ``--record-traffic CSV`` turns an ncu capture of the DRAM-byte counters into
-``gpurun_out/dram_traffic.json`` keyed by the hash of the CUDA sources.
+a record keyed by the hash of the CUDA sources (``--traffic-out``, by default
+the ``profiles/dram_traffic.json`` that the roofline objects read).
 """
 from __future__ import annotations
 
@@ -506,14 +507,15 @@ def main():
                     help="comma list of Top-P thresholds: prefill time and density per p on --workload, vs dense")
     ap.add_argument("--record-traffic", default=None,
                     help="comma list of ncu CSV files (dram__bytes_*.sum, --print-units base) of --workload")
+    ap.add_argument("--traffic-out", default=TRAFFIC_FILE,
+                    help="with --record-traffic: where to write the record")
     ap.add_argument("--traffic-scale", default="",
                     help="with --record-traffic: comma list workload=factor (bytes per launch there / here)")
     args = ap.parse_args()
     if args.record_traffic:
         scales = dict((kv.split("=")[0], float(kv.split("=")[1])) for kv in args.traffic_scale.split(",") if kv)
-        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-        record_traffic(args.record_traffic.split(","), args.workload, scales,
-                       os.path.join(ROOT, "gpurun_out", "dram_traffic.json"))
+        os.makedirs(os.path.dirname(os.path.abspath(args.traffic_out)), exist_ok=True)
+        record_traffic(args.record_traffic.split(","), args.workload, scales, args.traffic_out)
         return
     if args.table:
         run_table(args)
