@@ -25,8 +25,10 @@
 //               with P read from tensor memory (bf16, written over S).
 //               Issue order: PV_A(t), QK_A(t+1), PV_B(t), QK_B(t+1), so one
 //               tile's softmax overlaps the other tile's matrix products;
-//               each P V product starts on keys 0-63 as soon as the softmax
-//               has published that half of P, while it computes the other.
+//               each P V product starts on keys 0-95 as soon as the softmax
+//               has published that part of P, while it computes keys 96-127,
+//               so only a 32-key product separates the end of a tile's
+//               softmax from its next Q K^T.
 //               A tile that skips step t but takes step t + 1 gets its Q K^T
 //               at the start of step t when K(t + 1) has already landed, so
 //               its softmax runs beside the other tile's (at low density more
@@ -62,6 +64,11 @@ constexpr int kMaxMaskWords = 16384 / 32;  // mask words of one row at the large
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + slack for 1024-byte alignment
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// P is published in two parts: keys [0, 16 kPFirstSteps) first, so the P V
+// product on them runs while the softmax computes the rest; only the short
+// second part's product then stands between the end of the softmax and the
+// tile's next Q K^T
+constexpr int kPFirstSteps = 6;
 
 // Barrier slots (8 bytes each) after kOffBar.
 enum : uint32_t {
@@ -72,7 +79,7 @@ enum : uint32_t {
   kBarSFull = 7,    // [2] per tile
   kBarPFull = 9,    // [2] per tile
   kBarODone = 11,   // [2] per tile
-  kBarPHalf = 13,   // [2] per tile: P of keys 0-63 written
+  kBarPHalf = 13,   // [2] per tile: P of keys [0, 16 kPFirstSteps) written
   kBarDone = 15,    // softmax threads finished with tensor memory
   kBarVEmpty = 16,  // [2] the P V products that read the V stage are done
   kNumBars = 18
@@ -165,16 +172,17 @@ __device__ __forceinline__ void mma_qk(uint32_t d_tmem, uint32_t q_lo, uint32_t 
 }
 
 // O += P V over keys [64 part, 64 part + 64): four K steps of 16 keys
-// (v_lo: low word of the V stage's descriptor, MN-major, 2 KB per 16 keys)
+// O += P V over keys [16 k0, 16 k1): K steps of 16 keys; P in tensor memory at
+// p_tmem (two bf16 per column), v_lo: low word of the V stage's descriptor
+// (MN-major, 2 KB per 16 keys)
+template <int K0, int K1>
 __device__ __forceinline__ void mma_pv_part(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_lo, uint32_t hi,
-                                            bool accumulate, int part) {
+                                            bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 1);  // P K-major (TMEM), V MN-major
 #pragma unroll
-  for (int k4 = 0; k4 < 4; ++k4) {
-    const int kk = part * 4 + k4;
+  for (int kk = K0; kk < K1; ++kk)
     mma_bf16_ts_lo(o_tmem, p_tmem + kk * 8, v_lo + (uint32_t)(kk * 2048 / 16), hi, idesc,
                    (accumulate || kk > 0) ? 1u : 0u);
-  }
 }
 
 // Row max of this thread's S row held in registers; DIAG skips keys c > r.
@@ -193,42 +201,55 @@ __device__ __forceinline__ float row_max(const uint32_t (&sv)[128], int r) {
   return fmaxf(max3f(mc[0], mc[1], mc[2]), mc[3]);
 }
 
+// P = exp2(S * scale_log2 - m) for the key pairs [e0, e0 + ne) of this
+// thread's S row (keys 2 e, 2 e + 1), two bf16 per word into pk; the fp32
+// values are added into acc.  Packed f32x2 arithmetic for the scale/shift and
+// the sums; four independent partial sums keep the dependency chains short.
+// DIAG zeroes keys c > r (causal diagonal).
+template <bool DIAG>
+__device__ __forceinline__ void p_pairs(const uint32_t (&sv)[128], int e0, int ne, uint64_t sc2, uint64_t nm2, int r,
+                                        uint64_t (&acc)[4], uint32_t* pk) {
+#pragma unroll
+  for (int e = 0; e < ne; ++e) {
+    const int c = 2 * (e0 + e);
+    const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sc2, nm2);
+    float x0, x1;
+    f2_unpack(x2, x0, x1);
+    float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+    if (DIAG) {
+      if (c > r) p0 = 0.f;
+      if (c + 1 > r) p1 = 0.f;
+    }
+    acc[e & 3] = f2_add(acc[e & 3], f2_pack(p0, p1));
+    pk[e] = pack_bf16x2(p0, p1);
+  }
+}
+
 // Writes P = exp2(S * scale_log2 - m) as bf16 over columns [0, 64) of this
-// thread's S row and returns the row sum of the fp32 values.  Packed f32x2
-// arithmetic for the scale/shift and the sum; four independent partial sums
-// keep the dependency chains short.  DIAG zeroes keys c > r (causal diagonal).
-// The first half (keys 0-63) is published on bar_half as soon as it is in
-// tensor memory, so the P V product can start on it while the second half is
+// thread's S row and returns the row sum of the fp32 values.  Keys
+// [0, 16 kPFirstSteps) are published on bar_first as soon as they are in
+// tensor memory, so the P V product can start on them while the rest is
 // computed.
 template <bool DIAG>
 __device__ __forceinline__ float softmax_p(const uint32_t (&sv)[128], uint32_t tS, float scale_log2, float m,
-                                           int r, uint32_t bar_half) {
+                                           int r, uint32_t bar_first) {
+  static_assert(kPFirstSteps == 6, "the store shapes below assume 96 + 32 keys");
   const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
   const uint64_t nm2 = f2_pack(-m, -m);
   uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-  for (int h2 = 0; h2 < 2; ++h2) {
-    uint32_t pk[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int c = h2 * 64 + 2 * e;
-      const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sc2, nm2);
-      float x0, x1;
-      f2_unpack(x2, x0, x1);
-      float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-      if (DIAG) {
-        if (c > r) p0 = 0.f;
-        if (c + 1 > r) p1 = 0.f;
-      }
-      acc[e & 3] = f2_add(acc[e & 3], f2_pack(p0, p1));
-      pk[e] = pack_bf16x2(p0, p1);
-    }
-    tmem_st32(tS + h2 * 32, pk);
-    if (h2 == 0) {
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar_half);
-    }
+  {
+    uint32_t pk[48];
+    p_pairs<DIAG>(sv, 0, 48, sc2, nm2, r, acc, pk);
+    tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+    tmem_st16(tS + 32, *reinterpret_cast<const uint32_t(*)[16]>(pk + 32));
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(bar_first);
+  }
+  {
+    uint32_t pk[16];
+    p_pairs<DIAG>(sv, 48, 16, sc2, nm2, r, acc, pk);
+    tmem_st16(tS + 48, pk);
   }
   const uint64_t t2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
   float a0, a1;
@@ -404,10 +425,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             if (in_cur[x]) {
               if (!(ok = mbar_wait(bar(kBarPHalf + x), u[x] & 1))) break;
               tc_fence_after();
-              mma_pv_part(tO[x], tS[x], vd0 + s * kStep, hi, u[x] > 0, 0);
+              mma_pv_part<0, kPFirstSteps>(tO[x], tS[x], vd0 + s * kStep, hi, u[x] > 0);
               if (!(ok = mbar_wait(bar(kBarPFull + x), u[x] & 1))) break;
               tc_fence_after();
-              mma_pv_part(tO[x], tS[x], vd0 + s * kStep, hi, true, 1);
+              mma_pv_part<kPFirstSteps, 8>(tO[x], tS[x], vd0 + s * kStep, hi, true);
               mma_commit(bar(kBarODone + x));
               ++u[x];
             }
