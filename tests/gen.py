@@ -87,6 +87,31 @@ def rope_tables(seqlen: int, head_dim: int, base: float, start: int = 0, theta=N
     return torch.cos(ang), torch.sin(ang)
 
 
+def mrope_tables(pos_thw: torch.Tensor, head_dim: int, base: float, sections=(16, 24, 24)):
+    """Multimodal RoPE (M-RoPE) cos/sin tables [N, head_dim/2]: every token has a
+    (temporal, height, width) position and the frequency pairs are split into
+    consecutive sections, pair j taking the position component of its section
+    (the fastest ``sections[0]`` pairs the temporal one, then height, then
+    width; 16 / 24 / 24 pairs at head_dim 128).  A text token has t = h = w =
+    its index, which makes the tables those of plain RoPE."""
+    half = head_dim // 2
+    assert sum(sections) == half
+    j = torch.arange(half, dtype=torch.float64)
+    theta = base ** (-2.0 * j / head_dim)
+    comp = torch.cat([torch.full((n,), c, dtype=torch.long) for c, n in enumerate(sections)])
+    pos = torch.as_tensor(pos_thw, dtype=torch.float64)[:, comp]  # [N, half]: each pair's position
+    ang = pos * theta[None, :]
+    return torch.cos(ang), torch.sin(ang)
+
+
+def video_positions(frames: int, height: int, width: int, t0: int = 0) -> torch.Tensor:
+    """(t, h, w) positions of a video's patch tokens, frame by frame, row by row."""
+    t = torch.arange(frames).repeat_interleave(height * width) + t0
+    h = torch.arange(height).repeat_interleave(width).repeat(frames)
+    w = torch.arange(width).repeat(frames * height)
+    return torch.stack([t, h, w], dim=1)
+
+
 def apply_rope(x: torch.Tensor, cos: torch.Tensor, sin: torch.Tensor, interleaved: bool = False) -> torch.Tensor:
     """RoPE on the last dim of fp64 ``x`` [..., N, D]: pair j = (j, j+D/2)
     (half-split) or (2j, 2j+1) (interleaved)."""
@@ -183,5 +208,5 @@ def rope_theta(head_dim: int, base: float):
     return [base ** (-2.0 * j / head_dim) for j in range(half)]
 
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "rope_tables", "apply_rope",
-           "small_workload", "default_bands", "rope_theta", "HEAD_DIM", "BLOCK"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "rope_tables", "apply_rope", "mrope_tables",
+           "video_positions", "small_workload", "default_bands", "rope_theta", "HEAD_DIM", "BLOCK"]

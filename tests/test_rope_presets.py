@@ -121,3 +121,44 @@ def test_pooling_attenuation_by_layout_and_ladder(layout, ladder):
     kept_hi = e_out[hi].sum() / e_in[hi].sum()
     kept_lo = e_out[lo].sum() / e_in[lo].sum()
     assert kept_hi < 0.75 and kept_lo > 0.85 and kept_hi < kept_lo
+
+
+def test_mrope_on_text_is_plain_rope():
+    """Text tokens under M-RoPE (t = h = w = index) rotate exactly as under
+    plain RoPE, so the presets, the pooling attenuation and the whole estimate
+    are unchanged (gist.science Technical Summary, results: Prism carries over
+    to M-RoPE)."""
+    n, d, base = 1024, 128, 1e6
+    idx = torch.arange(n)
+    cos_m, sin_m = gen.mrope_tables(torch.stack([idx, idx, idx], dim=1), d, base)
+    cos_r, sin_r = gen.rope_tables(n, d, base)
+    assert torch.equal(cos_m, cos_r) and torch.equal(sin_m, sin_r)
+
+
+@pytest.mark.parametrize("height,width", [(8, 16), (4, 32)])
+def test_mrope_video_block_attenuation(height, width):
+    """One frame of height x width = 128 patch tokens pooled as one block: the
+    temporal pairs do not rotate inside it (no attenuation), the height pairs
+    step once per row (Dirichlet kernel over `height` positions), the width
+    pairs once per token within a row (Dirichlet kernel over `width`).  So on
+    video the fastest pairs are not the most attenuated ones: the text-derived
+    high band holds the unattenuated temporal section."""
+    d, base = 128, 1e6
+    sections = (16, 24, 24)
+    pos = gen.video_positions(1, height, width, t0=3)
+    assert pos.shape[0] == 128
+    cos, sin = gen.mrope_tables(pos, d, base, sections)
+    rng = np.random.default_rng(5)
+    c = torch.from_numpy(rng.standard_normal(d))
+    x = gen.apply_rope(c[None, :].expand(128, d).clone(), cos, sin).numpy()
+    pooled = oracle.mean_pool(x, 128)[0]
+    lam = np.hypot(pooled[:64], pooled[64:]) / np.hypot(c.numpy()[:64], c.numpy()[64:])
+    theta = np.array(gen.rope_theta(d, base))
+    expect = np.concatenate([np.ones(sections[0]),
+                             _dirichlet(theta[16:40], height),
+                             _dirichlet(theta[40:64], width)])
+    np.testing.assert_allclose(lam, expect, rtol=0, atol=1e-12)
+    hi, lo = pb.rope_band_sets("half_split")
+    e_in, e_out = c.numpy() ** 2, pooled ** 2
+    temporal_hi = [k for k in hi if k % 64 < 16]
+    assert np.isclose(e_out[temporal_hi].sum(), e_in[temporal_hi].sum(), rtol=1e-12)
