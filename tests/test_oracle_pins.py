@@ -348,6 +348,48 @@ def test_top_p_p1_keeps_all_and_monotone():
         prev = r
 
 
+def test_top_p_p1_keeps_blocks_of_zero_probability():
+    """p >= 1 keeps every causal block even where the mass ahead of a block
+    already rounds to 1 (probabilities that underflow to 0): the rule is
+    stated for p, not left to the floating-point sum reaching 1."""
+    mat = np.array([[1.0, 0, 0], [1.0, 0.0, 0], [1.0, 0.0, 0.0]])
+    keep, c_excl = oracle.top_p(mat, 1.0)
+    np.testing.assert_array_equal(keep, np.tril(np.ones((3, 3), dtype=bool)))
+    assert c_excl[2, 1] == 1.0 and c_excl[2, 2] == 1.0
+    # the same through the estimator: a temperature small enough that every
+    # row's softmax puts all its mass on one block
+    rng = np.random.default_rng(21)
+    q = rng.standard_normal((1, 1, 8 * 16, 128))
+    k = rng.standard_normal((1, 1, 8 * 16, 128))
+    r = oracle.estimate(q, k, list(range(64)), list(range(32, 128)), 1.0, block=16,
+                        tau_mode="explicit", tau_explicit=(1e-4, 1e-4))
+    assert np.any(r["probs"][0, 0][:, np.tril(np.ones((8, 8), dtype=bool))] == 0.0)
+    np.testing.assert_array_equal(r["mask"][0, 0], np.tril(np.ones((8, 8), dtype=bool)))
+
+
+def test_zero_queries_give_unit_tau_and_uniform_rows():
+    """A head whose queries are all zero: every pooled RMS of Q is 0, so both
+    temperatures fall back to 1, every causal logit is 0, each row's softmax is
+    uniform over its i + 1 blocks, and Top-P (ties to the lower block index)
+    keeps exactly the first ceil(p (i + 1)) blocks."""
+    rng = np.random.default_rng(22)
+    nb, p = 12, 0.61  # p (i + 1) is never within 0.01 of an integer for i < 12
+    q = np.zeros((1, 1, nb * 16, 128))
+    k = rng.standard_normal((1, 1, nb * 16, 128))
+    r = oracle.estimate(q, k, list(range(64)), list(range(32, 128)), p, block=16)
+    np.testing.assert_array_equal(r["tau"][0, 0], [1.0, 1.0])
+    causal = np.tril(np.ones((nb, nb), dtype=bool))
+    for z in range(2):
+        np.testing.assert_array_equal(r["logits"][0, 0, z][causal], 0.0)
+        np.testing.assert_allclose(r["probs"][0, 0, z], causal / np.arange(1, nb + 1)[:, None],
+                                   rtol=1e-15, atol=0)
+    want = np.zeros((nb, nb), dtype=bool)
+    for i in range(nb):
+        want[i, :math.ceil(p * (i + 1))] = True
+    for key in ("keep_hi", "keep_lo", "mask"):
+        np.testing.assert_array_equal(r[key][0, 0], want)
+
+
 def test_union_identities():
     q, k = _small_inputs(seed=10)
     hi, lo = gen.default_bands()
@@ -419,6 +461,29 @@ def test_attention_sparse_mask_vs_library():
             rows_visible = tok[i * 128:(i + 1) * 128].any(axis=1)
             np.testing.assert_allclose(o[rows_visible], ref[0, h, i * 128:(i + 1) * 128][rows_visible],
                                        rtol=1e-10, atol=1e-12)
+
+
+def test_attention_batch_elements_vs_library():
+    """Batch element b reads its own Q, K and V: every element of a batch of two
+    matches the library's attention of that element alone (same block mask)."""
+    w = gen.small_workload("pin_attn_b2", 2, 2, 1, 512, 14)
+    q, k, v = (x.double().numpy() for x in gen.make_inputs(w))
+    nb = 4
+    rng = np.random.default_rng(6)
+    blk = np.tril(rng.random((nb, nb)) < 0.6)
+    blk[np.arange(nb), np.arange(nb)] = True
+    tok = np.repeat(np.repeat(blk, 128, axis=0), 128, axis=1) & np.tril(np.ones((512, 512), dtype=bool))
+    dense = oracle.dense_causal_attention(q, k, v, group=2)
+    for b in range(2):
+        ref = _sdpa_ref(q[b:b + 1], k[b:b + 1], v[b:b + 1], torch.from_numpy(tok), 2).numpy()
+        causal_ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[b]), torch.from_numpy(k[b]).repeat_interleave(2, dim=0),
+            torch.from_numpy(v[b]).repeat_interleave(2, dim=0), is_causal=True).numpy()
+        np.testing.assert_allclose(dense[b], causal_ref, rtol=1e-10, atol=1e-12)
+        for h in range(2):
+            for i in range(nb):
+                o = oracle.sparse_attention_block(q, k, v, blk[i], b, h, i, group=2)
+                np.testing.assert_allclose(o, ref[0, h, i * 128:(i + 1) * 128], rtol=1e-10, atol=1e-12)
 
 
 def test_attention_diagonal_only_is_local_and_empty_is_zero():
