@@ -133,8 +133,8 @@ def rope_band_sets(layout: str = "half_split", d_high: int = 64, d_low: int = 96
 
     RoPE rotates dimension pairs; pair j turns at theta_j = base^(-2j / D), j = 0
     the fastest.  The high band is the d_high / 2 fastest pairs, the low band the
-    d_low / 2 slowest (the review's method step (1): "first d_high / last d_low",
-    read in frequency-pair order).  Pair j occupies dims (j, j + D/2) in the
+    d_low / 2 slowest (the review's method step (1) takes the leading d_high and the trailing
+    d_low dims, read here in frequency-pair order).  Pair j occupies dims (j, j + D/2) in the
     half-split layout (GPT-NeoX / Llama-style checkpoints) and (2j, 2j + 1) in
     the interleaved layout (GPT-J-style).  RoPE variants that keep the
     frequencies monotone in j -- YaRN's per-band interpolation, M-RoPE's
